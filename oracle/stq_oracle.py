@@ -31,7 +31,8 @@ Readings taken where the pages are silent (each also listed in the design doc):
     bits [b*j, b*j + b).
   * Degenerate cases: a zero row scale gives an all-zero row of Q and no weight; a
     zero column scale gives an all-zero column of Q; a column whose least-squares
-    denominator is 0 keeps its previous scale.
+    denominator is 0 keeps its previous scale. A scale below 2^-126 (the smallest
+    normal float32) is treated as zero when its reciprocal is taken.
   * FP16 pivot rows are stored as the float16 rounding of the updated float32 state
     and take no part in the refit.
 """
@@ -248,11 +249,16 @@ def _quantise(y, inv_c, qm):
     return np.clip(np.rint(x), -qm[..., :, None], qm[..., :, None]).astype(F32)
 
 
+TINY = F32(np.finfo(np.float32).tiny)   # 2^-126, the smallest normal float32
+
+
 def _recip(a):
-    """float32 1/a where a > 0, else 0."""
+    """float32 1/a for a scale a >= 2^-126; a smaller scale counts as zero and gets 0
+    (its reciprocal would overflow)."""
     a = np.asarray(a, dtype=F32)
-    safe = np.where(a > 0, a, F32(1))
-    return np.where(a > 0, F32(1) / safe, F32(0)).astype(F32)
+    ok = a >= TINY
+    safe = np.where(ok, a, F32(1))
+    return np.where(ok, F32(1) / safe, F32(0)).astype(F32)
 
 
 def refit(S, omega, row_bits, n_ls=2):

@@ -155,6 +155,15 @@ def test_zero_state_and_zero_rows():
     assert np.all(O.dequantize(u, r, c, np.zeros((128, 128), np.float16), bits)[5] == 0)
 
 
+def test_subnormal_scale_counts_as_zero():
+    # a column of subnormal values: its start scale is below 2^-126, so its codes are 0
+    # rather than the NaN that 0 * (1/c) = 0 * inf would give
+    S = np.random.default_rng(12).standard_normal((128, 128)).astype(F32)
+    S[:, 3] = np.float32(1e-44)
+    u, r, c, _ = O.refit(S, np.ones(128, F32), np.full(128, 6))
+    assert np.all(np.isfinite(c)) and np.all(u[:, 3] == 32) and np.all((u >= 1) & (u <= 63))
+
+
 def test_dequantize_hand_example():
     # X_ij = r_i c_j z_ij (bloombook section 4) with z = u - 2^(b-1)
     bits = np.array([4, 4, 16, 2])
@@ -198,7 +207,7 @@ def _scalar_refit(S, omega, bits):
         m = _tsum([abs(S[i][j]) for j in range(d)]) * f(1.0 / d)
         ri = f(0) if piv[i] else m * g[i]
         r.append(ri)
-        inv_r.append(f(1) / ri if ri > 0 else f(0))
+        inv_r.append(f(1) / ri if ri >= f(2.0 ** -126) else f(0))
     y = [[S[i][j] * inv_r[i] for j in range(d)] for i in range(d)]
     c = []
     for j in range(d):
@@ -212,7 +221,7 @@ def _scalar_refit(S, omega, bits):
     def quant(c):
         Q = [[f(0)] * d for _ in range(d)]
         for j in range(d):
-            ic = f(1) / c[j] if c[j] > 0 else f(0)
+            ic = f(1) / c[j] if c[j] >= f(2.0 ** -126) else f(0)
             for i in range(d):
                 x = float(y[i][j]) * float(ic)
                 Q[i][j] = f(max(-qm[i], min(qm[i], np.rint(x))))
