@@ -1,0 +1,401 @@
+#!/usr/bin/env python
+"""Throughput of the packed Delta-rule state decode step on B200.
+
+One step = one stq_decode_step over every (request, head) of the workload: restore
+the packed state, gated delta update, float32 readout, refit, packed write-back.
+Default workload: GDN, B = 512 requests x H = 48 heads, d = 128, nominal 6-bit
+allocation ({4,6,8} bits at 0.2/0.5/0.3 of the heads plus 2% FP16 pivot heads),
+lognormal row influence, x10 row/column outliers; states built by 256 FP32 warm-up
+steps from zero.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl stq|reference]
+
+Under torchrun each rank runs its own B requests on its own GPU (weak scaling, no
+collective on the data path); rank 0 prints one JSON line. `--impl reference` times
+the CPU oracle on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from quantized_linear_attention_02_b200 import workload as W  # noqa: E402
+
+D = 128
+METRIC = "head-state decode steps/s and HBM GB/s (% of B200 peak), B=512 6-bit"
+UNIT = "head-state steps/s"
+
+# Peaks: MEASURED_PEAKS.json when present, else the pool's earlier measurement.
+FALLBACK_HBM_GBS = 6650.0
+SMS = 148
+FP32_LANES_PER_SM = 128
+
+# ncu dram bytes (read + write) per launch of decode_kernel on the default workload,
+# and the sha256 of the kernel source they were taken with (a changed kernel voids them).
+TRAFFIC = {"bytes": None, "kernel_sha256": None, "source": None}
+
+
+def kernel_sha():
+    p = os.path.join(ROOT, "quantized_linear_attention_02_b200", "csrc", "stq_kernels.cu")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return float(j["hbm_gbs"]), float(j.get("sm_max_mhz", 1965.0)), "measured"
+    return FALLBACK_HBM_GBS, 1965.0, "fallback"
+
+
+# ---------------------------------------------------------------------------------
+# algorithmic counts per step
+# ---------------------------------------------------------------------------------
+def algorithmic_bytes(w, B):
+    """Bytes a decode step must move: every head's packed codes (or FP16 pivot rows)
+    read and written, its scales r[128], c[128] read and written (heads with any
+    quantised row), q, k, v, gate, beta read and o written."""
+    rb = W.row_bits(w)
+    per_req = 0
+    for h in range(w.H):
+        piv = rb[h] == 16
+        codes = int((D * rb[h][~piv] // 8).sum()) + int(piv.sum()) * D * 2
+        scales = 2 * D * 4 if (~piv).any() else 0
+        per_req += 2 * (codes + scales)
+        per_req += 3 * D * 4 + (4 if w.kind == "gdn" else D * 4) + 4 + D * 4
+    return per_req * B
+
+
+def algorithmic_flops(w, B):
+    """float32 operations the rule prescribes per step (each rounded IEEE operation
+    of the oracle's definition): per quantised element 31 for GDN (restore 2, k^T S 2,
+    update 2, readout 2, |S| row sum 1, y 1, column max 1, least-squares step one 7,
+    step two 9 with the clamp, final code 4), one more for KDA's per-row 1/qmax in
+    the column max; per FP16 pivot element 7 (decay, k^T S, update, readout)."""
+    rb = W.row_bits(w)
+    per_q = 31 + (1 if w.kind == "kda" else 0)
+    nq = int((rb != 16).sum()) * D
+    npv = int((rb == 16).sum()) * D
+    return B * (per_q * nq + 7 * npv)
+
+
+# ---------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------------
+# CPU oracle timing (reported baseline only)
+# ---------------------------------------------------------------------------------
+def oracle_rate(w, budget_s=10.0, reqs=1):
+    """Head-state steps/s of the CPU oracle on one thread, timed on a sample of the
+    workload (`reqs` requests x all heads per call) for about budget_s seconds."""
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(limits=1)
+    except Exception:  # pragma: no cover
+        limiter = None
+    from oracle import stq_oracle as O
+    rb, om = W.row_bits(w), W.omega(w)
+    rng = np.random.default_rng(0)
+    S = (rng.standard_normal((reqs, w.H, D, D)) * 0.1).astype(np.float32)
+    u, r, c, piv = O.refit(S, om, rb)
+    heads, t0, calls = 0, time.perf_counter(), 0
+    while True:
+        x = W.step_inputs(w, "decode", calls, 0, reqs)
+        u, r, c, piv, o, X = O.decode_step(u, r, c, piv, rb, om, x.q, x.k, x.v,
+                                           O.gate_rows(x.gate, w.kind, D), x.beta)
+        heads += reqs * w.H
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    if limiter is not None:
+        limiter.unregister()
+    return heads / el, {"kind": "oracle", "cores": 1,
+                        "sample": f"{calls} oracle decode steps of {reqs} request(s) x {w.H} heads "
+                                  f"of {w.name} in {el:.1f} s, one thread"}
+
+
+def reference_arm(args, rank, world):
+    w = W.WORKLOADS[args.workload]
+    if rank != 0:
+        return
+    # size each step's sample so that warmup + steps take about args.ref_budget seconds
+    from oracle import stq_oracle as O
+    rb, om = W.row_bits(w), W.omega(w)
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(limits=1)
+    except Exception:  # pragma: no cover
+        pass
+    rng = np.random.default_rng(0)
+    S = (rng.standard_normal((1, w.H, D, D)) * 0.1).astype(np.float32)
+    u0, r0, c0, p0 = O.refit(S, om, rb)
+    x = W.step_inputs(w, "decode", 0, 0, 1)
+    t0 = time.perf_counter()
+    O.decode_step(u0, r0, c0, p0, rb, om, x.q, x.k, x.v, O.gate_rows(x.gate, w.kind, D), x.beta)
+    per_head = (time.perf_counter() - t0) / w.H
+    n_steps = args.steps + args.warmup
+    heads = int(max(1, min(w.H, args.ref_budget / max(n_steps, 1) / per_head)))
+    sub = slice(0, heads)
+    rbs, oms = rb[sub], om[sub]
+    u, r, c, p = u0[:, sub], r0[:, sub], c0[:, sub], p0[:, sub]
+
+    def step(t):
+        nonlocal u, r, c, p
+        x = W.step_inputs(w, "decode", t, 0, 1)
+        u, r, c, p, o, X = O.decode_step(u, r, c, p, rbs, oms, x.q[:, sub], x.k[:, sub], x.v[:, sub],
+                                         O.gate_rows(x.gate[:, sub], w.kind, D), x.beta[:, sub])
+
+    for t in range(args.warmup):
+        step(t)
+    t0 = time.perf_counter()
+    for t in range(args.steps):
+        step(args.warmup + t)
+    el = time.perf_counter() - t0
+    value = heads * args.steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "d": D, "sample_heads_per_step": heads},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"each step: oracle decode of 1 request x {heads} heads of {w.name}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------
+# the CUDA arm
+# ---------------------------------------------------------------------------------
+def stq_arm(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from quantized_linear_attention_02_b200 import build, stq
+    build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = W.WORKLOADS[args.workload]
+    B, H = w.B, w.H
+    ub, om = W.unit_bits(w), W.omega(w)
+    n_slots = W.n_slots(B)
+    pool = stq.Pool(w.kind, n_slots, ub, om, device=dev)
+    slots = torch.tensor([W.slot_of_request(b) for b in range(B)], dtype=torch.int32, device=dev)
+    gen = torch.Generator(device=dev).manual_seed(1000 * args.workload + rank)
+
+    # initial states: FP32 warm-up steps from zero on the GPU, outlier rows, quantise
+    S = torch.zeros((B, H, D, D), device=dev)
+    out = torch.empty((B, H, D), device=dev)
+    for t in range(w.warmup_steps):
+        q, k, v, g, b = W.torch_step_inputs(w, B, gen, dev)
+        stq.fp32_decode_step(w.kind, S, q, k, v, g, b, out)
+    W.torch_scale_outlier_rows(S, w)
+    pool.quantize_init(slots, S)
+    pool.check()
+    del S
+    torch.cuda.empty_cache()
+
+    n_sets = 8
+    inputs = [W.torch_step_inputs(w, B, gen, dev) for _ in range(n_sets)]
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        q, k, v, g, b = inputs[i % n_sets]
+        pool.decode_step(slots, q, k, v, g, b, out, stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    clk = clocks.stop()
+    pool.check()
+
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_step = ms_max / args.steps
+    heads_per_step = B * H * world
+    value = heads_per_step / (ms_step * 1e-3)
+
+    # end to end through the host-buffer entry point: pinned inputs in, readout out
+    e2e = None
+    if args.e2e_steps > 0:
+        n_e = args.e2e_steps
+        pin = [[x.cpu().pin_memory() for x in s] for s in inputs[:2]]
+        h_out = torch.empty((B, H, D), dtype=torch.float32).pin_memory()
+        staging = torch.empty(pool.host_staging_bytes(B), dtype=torch.uint8, device=dev)
+        for i in range(3):
+            pool.decode_step_host(slots, *pin[i % 2], h_out, staging, stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(n_e):
+            pool.decode_step_host(slots, *pin[i % 2], h_out, staging, stream)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.barrier()
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        h2d = sum(x.numel() * 4 for x in pin[0])
+        e2e = {"value": heads_per_step / (float(te.item()) / n_e * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": B * H * D * 4, "steps": n_e}
+
+    if rank != 0:
+        return
+    hbm_peak, smax, which = peaks()
+    nbytes = algorithmic_bytes(w, B)
+    flops = algorithmic_flops(w, B)
+    sec = ms_step * 1e-3                 # one launch per step: the step time is the launch time
+    hbm_ach = nbytes / sec / 1e9
+    alu_peak = SMS * FP32_LANES_PER_SM * smax * 1e6 / 1e12
+    alu_ach = flops / sec / 1e12
+    traffic = TRAFFIC["bytes"] if TRAFFIC["kernel_sha256"] == kernel_sha() else None
+    hbm = {"bound": "hbm", "achieved": hbm_ach, "peak": hbm_peak, "unit": "GB/s",
+           "frac": hbm_ach / hbm_peak, "traffic": traffic, "peak_source": which,
+           "algorithmic_bytes_per_launch": nbytes}
+    alu = {"bound": "alu", "achieved": alu_ach, "peak": alu_peak, "unit": "TFLOP/s",
+           "frac": alu_ach / alu_peak, "traffic": traffic,
+           "peak_source": f"{SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x {smax:.0f} MHz",
+           "algorithmic_flops_per_launch": flops}
+    roofline = alu if alu["frac"] >= hbm["frac"] else hbm
+    other = hbm if roofline is alu else alu
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "kind": w.kind, "B": B, "H": H, "d": D,
+                   "global_batch": B * world, "bits": {str(b): int((ub == b).sum()) for b in sorted(set(ub.tolist()))},
+                   "n_slots": n_slots, "l2": "inputs larger than L2 (packed state of the active slots "
+                   f"{pool.sizes['slot_code_bytes'] * B / 1e9:.2f} GB, 8 rotating input sets)",
+                   "parallelism": f"dp{world}"},
+        "hbm_gbs": hbm_ach, "hbm_frac": hbm["frac"],
+        "roofline": roofline, "roofline_other": other,
+        "clocks": clk, "e2e": e2e, "gpu_launches": args.steps,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        rate, info = oracle_rate(w, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, **info}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["stq", "reference"], default="stq")
+    ap.add_argument("--workload", type=int, default=3, help="index into the workload list (3 = GDN B=512 6-bit)")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--ref-budget", type=float, default=90.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        stq_arm(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

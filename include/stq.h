@@ -1,0 +1,164 @@
+/*
+ * stq.h -- C ABI of the B200 packed Delta-rule state decode step.
+ *
+ * The operation is the per-(request, head) decode step over a low-bit recurrent
+ * state from "STEPQuant: When and Where Errors Matter in Delta-Rule Recurrent State
+ * Quantization" (arXiv 2609.38169), as these web pages describe it:
+ *   - gated delta rule S_t = (I - beta_t k_t k_t^T) D_t S_{t-1} + beta_t k_t v_t^T,
+ *     D_t a per-head scalar alpha_t (Gated DeltaNet, "GDN") or a per-key-channel
+ *     diagonal (Kimi Delta Attention, "KDA")  [bloombook.cn tutorial, section 2];
+ *   - readout o_t = S_t^T q_t from the updated floating-point state, then
+ *     requantise and store, so this step's error only reaches later steps
+ *     [singularity-lens.com summary, decode-order paragraph];
+ *   - dual-axis codes X_ij = r_i c_j z_ij with a key-row scale r_i and a value-column
+ *     scale c_j fitted under omega-weighted squared error  [bloombook section 4;
+ *     singularity-lens dual-axis paragraph];
+ *   - per-unit widths (unit = head for GDN, key row for KDA) from {2,4,6,8} and FP16
+ *     pivot units kept unquantised, fixed offline for all requests  [ai-trend.me
+ *     review, Method; singularity-lens calibration paragraph].
+ * The exact float32 evaluation order (tree sums, where the decay is folded, the
+ * refit rule) is the one the CPU oracle restates; both sides follow it.
+ *
+ * Conventions for every call:
+ *   - d_k = d_v = d = 128.
+ *   - Pointers named d_* are device pointers; h_* are host pointers. Every device
+ *     pointer must be 16-byte aligned (else STQ_ERR_ALIGNMENT).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Calls only enqueue work: the status covers argument checks and launch errors.
+ *   - The caller owns every buffer. The library never allocates device memory; the
+ *     pool handle owns only host memory (freed by stq_pool_destroy).
+ *   - Kernels check slot indices against n_slots; a bad index sets a sticky error
+ *     bit in the pool's device metadata and that (request, head) is skipped.
+ *     stq_pool_check() reads and clears it.
+ *   - No call may list the same slot twice in one batch.
+ *   - Errors: a non-zero stq_status; stq_last_error() gives a message (thread-local).
+ *   - No C++ exception crosses this boundary.
+ */
+#ifndef STQ_H
+#define STQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  STQ_OK = 0,
+  STQ_ERR_INVALID_ARG = 1,   /* a size, kind, width or pointer is invalid */
+  STQ_ERR_ALIGNMENT = 2,     /* a device pointer is not 16-byte aligned */
+  STQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+  STQ_ERR_DEVICE_CHECK = 4   /* a kernel found a bad slot index (stq_pool_check) */
+} stq_status;
+
+typedef enum { STQ_GDN = 0, STQ_KDA = 1 } stq_kind;
+
+#define STQ_D 128
+#define STQ_PIVOT_BITS 16
+
+/* Static description of a state pool: the per-unit widths and row influences are
+ * fixed offline and shared by every request (ai-trend review, Method (1)). */
+typedef struct {
+  int kind;                  /* stq_kind */
+  int n_slots;               /* number of state slots, > 0 */
+  int H;                     /* heads per slot, > 0 */
+  int d;                     /* must be STQ_D */
+  const uint8_t* unit_bits;  /* host; GDN: [H] (one width per head), KDA: [H*d]
+                                (one width per key row); each 2, 4, 6, 8 or 16 (FP16
+                                pivot unit) */
+  const float* omega;        /* host; [H*d] row influence omega_i, finite and > 0 */
+} stq_pool_desc;
+
+/* Buffer sizes (bytes) the caller allocates for a pool, from stq_pool_layout. */
+typedef struct {
+  size_t codes_bytes;        /* packed codes, all slots */
+  size_t scales_bytes;       /* float32 r[d], c[d] per (slot, head) */
+  size_t pivots_bytes;       /* float16 pivot rows, all slots */
+  size_t meta_bytes;         /* device metadata the library writes at create time */
+  size_t slot_code_bytes;    /* bytes of packed codes per slot */
+  int n_pivot_rows;          /* pivot rows per slot */
+  int max_head_bytes;        /* largest per-head code + pivot bytes */
+} stq_pool_sizes;
+
+typedef struct stq_pool stq_pool;
+
+/* Layout of one pool, host only (no CUDA call). Slot s holds, for head h, the rows
+ * of its non-pivot units back to back (row i of width b takes 16*b bytes; code j of a
+ * row is bits [b*j, b*j+b) of a little-endian bit stream, stored as
+ * u = Q + 2^(b-1)); the float16 rows of its pivot units in (head, row) order; and
+ * r[128], c[128] per head. Returns STQ_ERR_INVALID_ARG on a bad description. */
+stq_status stq_pool_layout(const stq_pool_desc* desc, stq_pool_sizes* out);
+
+/* Bind caller-allocated device buffers (sizes from stq_pool_layout) to a new pool
+ * handle and upload the static metadata (offsets, widths, omega_i and the row gain
+ * g_i = (omega_i / mean omega)^(-1/2)) into d_meta with a synchronous copy. The
+ * state buffers are not touched: fill them with stq_quantize_init. d_pivots may be
+ * NULL when the pool has no pivot rows. */
+stq_status stq_pool_create(const stq_pool_desc* desc, void* d_codes, void* d_scales,
+                           void* d_pivots, void* d_meta, stq_pool** out);
+
+/* Free the host handle. Device buffers stay the caller's. NULL is ignored. */
+void stq_pool_destroy(stq_pool* pool);
+
+/* Quantise float32 states into the pool: for b < B, slot d_slots[b] receives
+ * d_S[b] ([H, 128, 128], row-major, key row i, value column j) under the refit rule
+ * (row scale, column scale start, two omega-weighted least-squares steps, final
+ * codes; bloombook section 4). Pivot units store float16(S). */
+stq_status stq_quantize_init(stq_pool* pool, const int32_t* d_slots, int B,
+                             const float* d_S, void* stream);
+
+/* One decode step for B requests (THE hot path). For request b and head h, with
+ * slot s = d_slots[b]:
+ *   restore S' = D_t * dequantised state of (s, h), update with the gated delta rule,
+ *   write out[b, h, :] = S_t^T q (float32, from the updated unquantised state), refit
+ *   the scales and store S_t back into slot s packed.
+ * q, k, v: [B, H, 128] float32 device. gate: GDN [B, H] retention alpha_t, KDA
+ * [B, H, 128] per-key-row retention; values in [0, 1] (the host takes exp of the
+ * log-retention). beta: [B, H] in [0, 1]. out: [B, H, 128] float32 device. */
+stq_status stq_decode_step(stq_pool* pool, const int32_t* d_slots, int B,
+                           const float* d_q, const float* d_k, const float* d_v,
+                           const float* d_gate, const float* d_beta, float* d_out,
+                           void* stream);
+
+/* Bytes of device staging stq_decode_step_host needs for B requests. */
+size_t stq_decode_step_host_staging_bytes(const stq_pool* pool, int B);
+
+/* The same decode step with its per-step inputs and output in HOST memory (pinned
+ * for asynchronous copies): copies h_q, h_k, h_v, h_gate, h_beta into d_staging,
+ * runs stq_decode_step, and copies the output back into h_out, all on `stream`.
+ * d_slots stays a device array. The caller synchronises the stream before reading
+ * h_out. staging_bytes must be >= stq_decode_step_host_staging_bytes(pool, B). */
+stq_status stq_decode_step_host(stq_pool* pool, const int32_t* d_slots, int B,
+                                const float* h_q, const float* h_k, const float* h_v,
+                                const float* h_gate, const float* h_beta, float* h_out,
+                                void* d_staging, size_t staging_bytes, void* stream);
+
+/* Dequantise slots d_slots[0..B) into d_S_out [B, H, 128, 128] float32:
+ * S_ij = (Q_ij * r_i) * c_j, pivot rows float32(h_ij). */
+stq_status stq_dequantize(stq_pool* pool, const int32_t* d_slots, int B, float* d_S_out,
+                          void* stream);
+
+/* FP32-state decode step (the unquantised state the pages compare against), in place
+ * on d_S [B, H, 128, 128]: S <- (I - beta k k^T) D S + beta k v^T, out = S^T q.
+ * Same inputs as stq_decode_step; kind selects the gate shape. */
+stq_status stq_fp32_decode_step(int kind, int B, int H, int d, float* d_S,
+                                const float* d_q, const float* d_k, const float* d_v,
+                                const float* d_gate, const float* d_beta, float* d_out,
+                                void* stream);
+
+/* Synchronise `stream`, read the pool's sticky device error bits, clear them, and
+ * return STQ_ERR_DEVICE_CHECK if any was set (message names the check). */
+stq_status stq_pool_check(stq_pool* pool, void* stream);
+
+/* Message of the last failing call on this thread ("" if none). */
+const char* stq_last_error(void);
+
+/* Library version string. */
+const char* stq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STQ_H */

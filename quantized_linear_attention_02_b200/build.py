@@ -1,0 +1,48 @@
+"""Build step of the CUDA library: compiles csrc/ into libstq.so in this directory
+(sm_100a, in-tree, so the built library travels with the source tree)."""
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+LIB = os.path.join(HERE, "libstq.so")
+SOURCES = ["csrc/stq_abi.cpp", "csrc/stq_kernels.cu"]
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+
+FLAGS = [
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-lineinfo", "-O3", "-std=c++17",
+    "--fmad=false",                 # products are rounded before they are added
+    "-Xcompiler", "-fPIC,-O2,-Wall",
+    "-shared",
+]
+
+
+def needs_build() -> bool:
+    if not os.path.exists(LIB):
+        return True
+    t = os.path.getmtime(LIB)
+    deps = [os.path.join(HERE, s) for s in SOURCES]
+    deps += [os.path.join(HERE, "csrc", "stq_internal.h"), os.path.join(ROOT, "include", "stq.h")]
+    return any(os.path.getmtime(p) > t for p in deps)
+
+
+def build(force: bool = False, verbose: bool = False, extra=None) -> str:
+    if not force and not needs_build():
+        return LIB
+    cmd = [NVCC] + FLAGS + (extra or []) + ["-I", os.path.join(ROOT, "include"),
+                                            "-I", os.path.join(HERE, "csrc"), "-o", LIB]
+    cmd += [os.path.join(HERE, s) for s in SOURCES]
+    if verbose:
+        print(" ".join(cmd), file=sys.stderr)
+    tmp = LIB + ".tmp"
+    cmd[cmd.index(LIB)] = tmp
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    build(force="--force" in sys.argv, verbose=True,
+          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None)

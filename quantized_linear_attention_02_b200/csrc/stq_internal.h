@@ -1,0 +1,62 @@
+// Internal declarations shared by the C ABI (stq_abi.cpp) and the kernels
+// (stq_kernels.cu). Not part of the public interface.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+namespace stq {
+
+constexpr int D = 128;           // d_k = d_v
+constexpr int PIVOT = 16;        // width marker of an FP16 pivot unit
+
+// Error bits written by kernels into the pool's device error word.
+constexpr uint32_t ERR_SLOT_RANGE = 1u;   // a slot index was outside [0, n_slots)
+
+// Device view of a pool: caller-owned state buffers plus the metadata the library
+// uploaded into the caller-owned meta buffer. Passed to kernels by value.
+struct PoolDev {
+  int kind;                 // 0 = GDN, 1 = KDA
+  int n_slots;
+  int H;
+  int n_pivot_rows;         // pivot rows per slot
+  int max_head_bytes;       // largest per-head code + pivot bytes (staging size)
+  uint64_t slot_code_bytes;
+  uint8_t* codes;           // [n_slots, slot_code_bytes]
+  float* scales;            // [n_slots, H, 2, D]
+  uint16_t* pivots;         // [n_slots, n_pivot_rows, D] float16 bits
+  // metadata (device)
+  const uint32_t* head_code_off;    // [H] byte offset of head h's codes in a slot
+  const uint32_t* head_code_bytes;  // [H]
+  const uint32_t* head_piv_first;   // [H] index of head h's first pivot row in a slot
+  const uint32_t* head_piv_count;   // [H]
+  const uint32_t* row_info;         // [H*D] bits (low 8) | byte offset in head << 8
+                                    //   (pivot rows: index in head's pivot block << 8)
+  const float* g;                   // [H*D] row gain (omega_i / mean omega)^(-1/2)
+  const float* omega;               // [H*D]
+  uint32_t* err;                    // [4] sticky error bits
+};
+
+// Byte layout of the meta buffer, computed on the host.
+struct MetaLayout {
+  size_t head_code_off, head_code_bytes, head_piv_first, head_piv_count;
+  size_t row_info, g, omega, err, total;
+};
+
+MetaLayout meta_layout(int H);
+
+// Launchers (stq_kernels.cu). They return the cudaGetLastError() of the launch.
+cudaError_t launch_decode(const PoolDev& P, const int32_t* slots, int B, const float* q,
+                          const float* k, const float* v, const float* gate,
+                          const float* beta, float* out, cudaStream_t s);
+cudaError_t launch_quantize(const PoolDev& P, const int32_t* slots, int B, const float* S,
+                            cudaStream_t s);
+cudaError_t launch_dequantize(const PoolDev& P, const int32_t* slots, int B, float* S_out,
+                              cudaStream_t s);
+cudaError_t launch_fp32_step(int kind, int B, int H, float* S, const float* q,
+                             const float* k, const float* v, const float* gate,
+                             const float* beta, float* out, cudaStream_t s);
+
+}  // namespace stq

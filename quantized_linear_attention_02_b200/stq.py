@@ -1,0 +1,233 @@
+"""Thin Python binding of the C ABI in include/stq.h (argument marshalling only).
+
+Every step of the decode path runs in the CUDA library libstq.so built from csrc/;
+torch only provides device memory and streams. Nothing here computes on the host,
+and there is no fallback: a missing library raises at load time.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libstq.so")
+
+STQ_GDN, STQ_KDA = 0, 1
+D = 128
+PIVOT_BITS = 16
+KINDS = {"gdn": STQ_GDN, "kda": STQ_KDA}
+
+
+class StqError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"stq status {status}: {msg}")
+        self.status = status
+
+
+class _Desc(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("n_slots", ctypes.c_int), ("H", ctypes.c_int),
+                ("d", ctypes.c_int), ("unit_bits", ctypes.POINTER(ctypes.c_uint8)),
+                ("omega", ctypes.POINTER(ctypes.c_float))]
+
+
+class _Sizes(ctypes.Structure):
+    _fields_ = [("codes_bytes", ctypes.c_size_t), ("scales_bytes", ctypes.c_size_t),
+                ("pivots_bytes", ctypes.c_size_t), ("meta_bytes", ctypes.c_size_t),
+                ("slot_code_bytes", ctypes.c_size_t), ("n_pivot_rows", ctypes.c_int),
+                ("max_head_bytes", ctypes.c_int)]
+
+
+_lib = None
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+
+
+def lib():
+    """Load libstq.so (built in-tree by build.py); raise if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m quantized_linear_attention_02_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "stq_pool_layout": (_i, [ctypes.POINTER(_Desc), ctypes.POINTER(_Sizes)]),
+        "stq_pool_create": (_i, [ctypes.POINTER(_Desc), _vp, _vp, _vp, _vp, ctypes.POINTER(_vp)]),
+        "stq_pool_destroy": (None, [_vp]),
+        "stq_quantize_init": (_i, [_vp, _vp, _i, _vp, _vp]),
+        "stq_decode_step": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+        "stq_decode_step_host_staging_bytes": (ctypes.c_size_t, [_vp, _i]),
+        "stq_decode_step_host": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                      ctypes.c_size_t, _vp]),
+        "stq_dequantize": (_i, [_vp, _vp, _i, _vp, _vp]),
+        "stq_fp32_decode_step": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+        "stq_pool_check": (_i, [_vp, _vp]),
+        "stq_last_error": (ctypes.c_char_p, []),
+        "stq_version": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+def _check(status):
+    if status != 0:
+        raise StqError(status, lib().stq_last_error().decode())
+
+
+def _desc(kind, n_slots, unit_bits, omega):
+    ub = np.ascontiguousarray(unit_bits, dtype=np.uint8)
+    om = np.ascontiguousarray(omega, dtype=np.float32)
+    H = om.shape[0]
+    d = _Desc(KINDS[kind] if isinstance(kind, str) else int(kind), int(n_slots), int(H), D,
+              ub.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+              om.ctypes.data_as(ctypes.POINTER(ctypes.c_float)))
+    return d, (ub, om)   # keep the arrays alive with the struct
+
+
+def layout(kind, n_slots, unit_bits, omega) -> dict:
+    """Buffer sizes of a pool (host only; no CUDA call)."""
+    d, keep = _desc(kind, n_slots, unit_bits, omega)
+    s = _Sizes()
+    _check(lib().stq_pool_layout(ctypes.byref(d), ctypes.byref(s)))
+    return {f: getattr(s, f) for f, _ in _Sizes._fields_}
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t, dtype, name, numel=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name} must have {numel} elements, got {t.numel()}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+class Pool:
+    """A packed state pool on the current CUDA device. The buffers are torch tensors
+    owned here; the library handle only references them."""
+
+    def __init__(self, kind, n_slots, unit_bits, omega, device=None):
+        import torch
+        self.kind = kind
+        self.kind_id = KINDS[kind]
+        self.n_slots = int(n_slots)
+        self.unit_bits = np.ascontiguousarray(unit_bits, dtype=np.uint8)
+        self.omega = np.ascontiguousarray(omega, dtype=np.float32)
+        self.H = self.omega.shape[0]
+        self.sizes = layout(kind, n_slots, self.unit_bits, self.omega)
+        dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        s = self.sizes
+        self.codes = torch.zeros(max(s["codes_bytes"], 16), dtype=torch.uint8, device=dev)
+        self.scales = torch.zeros(s["scales_bytes"] // 4, dtype=torch.float32, device=dev)
+        self.pivots = torch.zeros(max(s["pivots_bytes"] // 2, 8), dtype=torch.float16, device=dev)
+        self.meta = torch.zeros(s["meta_bytes"], dtype=torch.uint8, device=dev)
+        d, keep = _desc(kind, n_slots, self.unit_bits, self.omega)
+        h = ctypes.c_void_p()
+        _check(lib().stq_pool_create(ctypes.byref(d), ctypes.c_void_p(self.codes.data_ptr()),
+                                     ctypes.c_void_p(self.scales.data_ptr()),
+                                     ctypes.c_void_p(self.pivots.data_ptr()),
+                                     ctypes.c_void_p(self.meta.data_ptr()), ctypes.byref(h)))
+        self.handle = h
+
+    def close(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            lib().stq_pool_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # views of the buffers in the pool's layout
+    def codes_view(self):
+        return self.codes[: self.sizes["codes_bytes"]].view(self.n_slots, -1)
+
+    def scales_view(self):
+        return self.scales.view(self.n_slots, self.H, 2, D)
+
+    def pivots_view(self):
+        n = self.sizes["n_pivot_rows"]
+        return self.pivots[: self.n_slots * n * D].view(self.n_slots, n, D)
+
+    def _slots(self, slots):
+        import torch
+        return _ptr(slots, torch.int32, "slots")
+
+    def quantize_init(self, slots, S, stream=None):
+        import torch
+        B = slots.numel()
+        _check(lib().stq_quantize_init(self.handle, self._slots(slots), B,
+                                       _ptr(S, torch.float32, "S", B * self.H * D * D), _stream(stream)))
+
+    def decode_step(self, slots, q, k, v, gate, beta, out, stream=None):
+        import torch
+        B = slots.numel()
+        n = B * self.H * D
+        ng = B * self.H if self.kind_id == STQ_GDN else n
+        _check(lib().stq_decode_step(self.handle, self._slots(slots), B,
+                                     _ptr(q, torch.float32, "q", n), _ptr(k, torch.float32, "k", n),
+                                     _ptr(v, torch.float32, "v", n), _ptr(gate, torch.float32, "gate", ng),
+                                     _ptr(beta, torch.float32, "beta", B * self.H),
+                                     _ptr(out, torch.float32, "out", n), _stream(stream)))
+
+    def host_staging_bytes(self, B):
+        return int(lib().stq_decode_step_host_staging_bytes(self.handle, int(B)))
+
+    def decode_step_host(self, slots, h_q, h_k, h_v, h_gate, h_beta, h_out, staging, stream=None):
+        """Decode step with host (pinned) input/output tensors; copies run inside the
+        library call on `stream`."""
+        import torch
+        B = slots.numel()
+        for name, t in (("q", h_q), ("k", h_k), ("v", h_v), ("gate", h_gate), ("beta", h_beta), ("out", h_out)):
+            if t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+                raise ValueError(f"host {name} must be a contiguous float32 CPU tensor")
+        _check(lib().stq_decode_step_host(
+            self.handle, self._slots(slots), B, ctypes.c_void_p(h_q.data_ptr()),
+            ctypes.c_void_p(h_k.data_ptr()), ctypes.c_void_p(h_v.data_ptr()),
+            ctypes.c_void_p(h_gate.data_ptr()), ctypes.c_void_p(h_beta.data_ptr()),
+            ctypes.c_void_p(h_out.data_ptr()), _ptr(staging, torch.uint8, "staging"),
+            ctypes.c_size_t(staging.numel()), _stream(stream)))
+
+    def dequantize(self, slots, S_out, stream=None):
+        import torch
+        B = slots.numel()
+        _check(lib().stq_dequantize(self.handle, self._slots(slots), B,
+                                    _ptr(S_out, torch.float32, "S_out", B * self.H * D * D),
+                                    _stream(stream)))
+
+    def check(self, stream=None):
+        """Synchronise and raise StqError if a kernel flagged a bad slot index."""
+        _check(lib().stq_pool_check(self.handle, _stream(stream)))
+
+
+def fp32_decode_step(kind, S, q, k, v, gate, beta, out, stream=None):
+    """FP32-state decode step in place on S [B, H, 128, 128]."""
+    import torch
+    B, H = S.shape[0], S.shape[1]
+    n = B * H * D
+    kid = KINDS[kind]
+    ng = B * H if kid == STQ_GDN else n
+    _check(lib().stq_fp32_decode_step(kid, B, H, D, _ptr(S, torch.float32, "S", n * D),
+                                      _ptr(q, torch.float32, "q", n), _ptr(k, torch.float32, "k", n),
+                                      _ptr(v, torch.float32, "v", n), _ptr(gate, torch.float32, "gate", ng),
+                                      _ptr(beta, torch.float32, "beta", B * H),
+                                      _ptr(out, torch.float32, "out", n), _stream(stream)))

@@ -200,3 +200,36 @@ def scale_outlier_rows(S: np.ndarray, w: Workload) -> np.ndarray:
     hh = np.arange(w.H)[:, None]
     S[:, hh, rows, :] *= np.float32(OUTLIER_FACTOR)
     return S
+
+
+def torch_step_inputs(w: Workload, B: int, generator, device="cuda"):
+    """The same input recipe drawn with torch's device RNG (fast, for large batches
+    whose exact values no oracle needs): returns q, k, v, gate, beta tensors."""
+    import torch
+    H, d = w.H, w.d
+    g = generator
+    q = torch.nn.functional.normalize(torch.randn((B, H, d), device=device, generator=g), dim=-1)
+    k = torch.nn.functional.normalize(torch.randn((B, H, d), device=device, generator=g), dim=-1)
+    v = torch.randn((B, H, d), device=device, generator=g)
+    _, cols = outlier_sets(w)
+    if cols.shape[1]:
+        scale = torch.ones((H, d), device=device)
+        hh = torch.arange(H, device=device)[:, None]
+        scale[hh, torch.as_tensor(cols, device=device)] = OUTLIER_FACTOR
+        v = v * scale
+    gshape = (B, H) if w.kind == "gdn" else (B, H, d)
+    gate = torch.exp(torch.empty(gshape, device=device, dtype=torch.float64)
+                     .uniform_(w.gate_low, w.gate_high, generator=g)).float()
+    beta = torch.sigmoid(torch.randn((B, H), device=device, generator=g))
+    return q.contiguous(), k.contiguous(), v.contiguous(), gate.contiguous(), beta.contiguous()
+
+
+def torch_scale_outlier_rows(S, w: Workload):
+    """Device version of scale_outlier_rows for a [B, H, d, d] tensor (in place)."""
+    import torch
+    rows, _ = outlier_sets(w)
+    if rows.shape[1] == 0:
+        return S
+    hh = torch.arange(w.H, device=S.device)[:, None]
+    S[:, hh, torch.as_tensor(rows, device=S.device), :] *= OUTLIER_FACTOR
+    return S

@@ -1,0 +1,91 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every entry point
+include/stq.h declares, computes pool layouts that agree with the oracle's own layout,
+and rejects bad descriptions with the documented status codes."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import stq_oracle as O
+from quantized_linear_attention_02_b200 import build, stq
+from quantized_linear_attention_02_b200 import workload as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return stq.lib()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "stq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(stq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    # and nothing else in the header is left without a definition
+    assert "stq_decode_step" in names and "stq_quantize_init" in names
+
+
+def test_version(lib):
+    assert b"sm_100a" in lib.stq_version()
+
+
+@pytest.mark.parametrize("w", W.WORKLOADS, ids=lambda w: w.name)
+def test_layout_matches_oracle_layout(lib, w):
+    ub, rb = W.unit_bits(w), W.row_bits(w)
+    om = W.omega(w)
+    n_slots = W.n_slots(w.B)
+    got = stq.layout(w.kind, n_slots, ub, om)
+    L = O.Layout(rb)
+    assert got["slot_code_bytes"] == L.slot_code_bytes
+    assert got["codes_bytes"] == n_slots * L.slot_code_bytes
+    assert got["n_pivot_rows"] == L.n_pivot_rows
+    assert got["scales_bytes"] == n_slots * w.H * 2 * 128 * 4
+    assert got["pivots_bytes"] == n_slots * L.n_pivot_rows * 128 * 2
+    heads = [int(L.code_len[h].sum() + 256 * (rb[h] == 16).sum()) for h in range(w.H)]
+    assert got["max_head_bytes"] == max(heads)
+
+
+def test_six_bit_head_size(lib):
+    got = stq.layout("gdn", 1, np.array([6], np.uint8), np.ones((1, 128), np.float32))
+    assert got["slot_code_bytes"] == 128 * 96        # 4 codes in 3 bytes
+
+
+@pytest.mark.parametrize("bad", ["width", "omega_zero", "omega_nan", "kind", "slots"])
+def test_invalid_descriptions_rejected(lib, bad):
+    ub = np.full(4, 6, np.uint8)
+    om = np.ones((4, 128), np.float32)
+    kind, n_slots = "gdn", 3
+    if bad == "width":
+        ub[2] = 5
+    elif bad == "omega_zero":
+        om[1, 7] = 0
+    elif bad == "omega_nan":
+        om[0, 0] = np.nan
+    elif bad == "kind":
+        kind = 7
+    elif bad == "slots":
+        n_slots = 0
+    with pytest.raises(stq.StqError) as e:
+        stq.layout(kind, n_slots, ub, om)
+    assert e.value.status == 1
+    assert lib.stq_last_error()
+
+
+def test_null_arguments(lib):
+    assert lib.stq_pool_layout(None, None) == 1
+    assert lib.stq_decode_step(None, None, 1, None, None, None, None, None, None, None) == 1
+    assert lib.stq_pool_check(None, None) == 1
+    lib.stq_pool_destroy(None)
+    assert lib.stq_fp32_decode_step(3, 1, 1, 128, None, None, None, None, None, None, None, None) == 1
+    assert lib.stq_fp32_decode_step(0, 1, 1, 64, None, None, None, None, None, None, None, None) == 1

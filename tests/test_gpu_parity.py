@@ -1,0 +1,291 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, on the five
+workloads. Every expected value comes from the oracle on the same seeded inputs;
+the initial states the GPU receives are oracle-built too."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+from oracle import stq_oracle as O  # noqa: E402
+from quantized_linear_attention_02_b200 import build, stq  # noqa: E402
+from quantized_linear_attention_02_b200 import workload as W  # noqa: E402
+
+import stq_testlib as T  # noqa: E402
+
+D = 128
+F32 = np.float32
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    build.build()
+    stq.lib()
+
+
+def dev(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def slots_t(reqs):
+    return dev(np.array([W.slot_of_request(b) for b in reqs], np.int32))
+
+
+def make_pool(w, n_slots=None):
+    ub = W.unit_bits(w)
+    om = W.omega(w)
+    return stq.Pool(w.kind, n_slots or W.n_slots(w.B), ub, om), O.Layout(W.row_bits(w)), om
+
+
+def oracle_quantised(w, reqs):
+    S0 = T.warm_state(w.index, tuple(reqs))
+    u, r, c, piv = O.refit(S0, W.omega(w), W.row_bits(w))
+    return S0, u, r, c, piv
+
+
+# ---------------------------------------------------------------------------------
+# FP32 step
+# ---------------------------------------------------------------------------------
+@pytest.mark.parametrize("widx", [0, 2])
+def test_fp32_step_bit_exact_state(widx):
+    w = W.WORKLOADS[widx]
+    reqs = list(range(min(w.B, 2)))
+    S0 = T.warm_state(widx, tuple(reqs), steps=8)
+    x = T.inputs_for(w, "decode", 0, reqs)
+    S_or, o_or = O.fp32_step(S0, x.q, x.k, x.v, O.gate_rows(x.gate, w.kind, D), x.beta)
+    S = dev(S0)
+    out = torch.empty((len(reqs), w.H, D), device="cuda")
+    stq.fp32_decode_step(w.kind, S, dev(x.q), dev(x.k), dev(x.v), dev(x.gate), dev(x.beta), out)
+    torch.cuda.synchronize()
+    assert np.array_equal(S.cpu().numpy(), S_or)
+    assert T.per_vector_rel_l2(out.cpu().numpy(), o_or).max() <= T.OUT_REL_L2
+
+
+# ---------------------------------------------------------------------------------
+# dequantise / quantise
+# ---------------------------------------------------------------------------------
+@pytest.mark.parametrize("widx", [0, 1, 2])
+def test_dequantize_bit_exact(widx):
+    w = W.WORKLOADS[widx]
+    reqs = [0, min(3, w.B - 1)] if w.B > 1 else [0]
+    pool, L, _ = make_pool(w)
+    S0, u, r, c, piv = oracle_quantised(w, reqs)
+    slots = [W.slot_of_request(b) for b in reqs]
+    T.write_oracle_state(pool, L, slots, u, r, c, piv)
+    out = torch.empty((len(reqs), w.H, D, D), device="cuda")
+    pool.dequantize(slots_t(reqs), out)
+    pool.check()
+    assert np.array_equal(out.cpu().numpy(), O.dequantize(u, r, c, piv, W.row_bits(w)))
+
+
+@pytest.mark.parametrize("widx", [0, 1, 2])
+def test_quantize_init_matches_oracle(widx):
+    w = W.WORKLOADS[widx]
+    reqs = [0, min(5, w.B - 1)] if w.B > 1 else [0]
+    pool, L, _ = make_pool(w)
+    S0, u, r, c, piv = oracle_quantised(w, reqs)
+    pool.quantize_init(slots_t(reqs), dev(S0))
+    pool.check()
+    ug, rg, cg, pg = T.read_pool_state(pool, L, [W.slot_of_request(b) for b in reqs])
+    rb = W.row_bits(w)
+    n = T.compare_codes(ug, u, S0, r, c, rb, "quantize_init")
+    if n == 0:
+        assert np.array_equal(rg, r) and np.array_equal(cg, c)
+    piv_rows = (rb == 16)
+    assert np.array_equal(pg[:, piv_rows], piv[:, piv_rows])
+
+
+# ---------------------------------------------------------------------------------
+# decode step, teacher-forced from an identical packed state
+# ---------------------------------------------------------------------------------
+def _single_step(w, reqs, t, pool, L):
+    S0, u, r, c, piv = oracle_quantised(w, reqs)
+    slots = [W.slot_of_request(b) for b in reqs]
+    T.write_oracle_state(pool, L, slots, u, r, c, piv)
+    x = T.inputs_for(w, "decode", t, reqs)
+    rb = W.row_bits(w)
+    u2, r2, c2, p2, o, X = O.decode_step(u, r, c, piv, rb, W.omega(w), x.q, x.k, x.v,
+                                         O.gate_rows(x.gate, w.kind, D), x.beta)
+    out = torch.empty((len(reqs), w.H, D), device="cuda")
+    pool.decode_step(slots_t(reqs), dev(x.q), dev(x.k), dev(x.v), dev(x.gate), dev(x.beta), out)
+    pool.check()
+    ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
+    n = T.compare_codes(ug, u2, X, r2, c2, rb, f"{w.name} step {t}")
+    if n == 0:
+        assert np.array_equal(rg, r2), "row scales differ"
+        assert np.array_equal(cg, c2), "column scales differ"
+    piv_rows = rb == 16
+    assert np.array_equal(pg[:, piv_rows], p2[:, piv_rows])
+    assert T.per_vector_rel_l2(out.cpu().numpy(), o).max() <= T.OUT_REL_L2
+    return n
+
+
+@pytest.mark.parametrize("widx,t", [(0, 0), (0, 7), (1, 0), (1, 31), (2, 0), (2, 17)])
+def test_decode_step_teacher_forced(widx, t):
+    w = W.WORKLOADS[widx]
+    reqs = [0, w.B - 1] if w.B > 1 else [0]
+    pool, L, _ = make_pool(w)
+    _single_step(w, reqs, t, pool, L)
+
+
+# ---------------------------------------------------------------------------------
+# chained steps: each side runs on its own from the same start
+# ---------------------------------------------------------------------------------
+@pytest.mark.parametrize("widx,steps", [(0, 16), (1, 64), (2, 64)])
+def test_decode_chain(widx, steps):
+    w = W.WORKLOADS[widx]
+    reqs = [1, w.B - 2] if w.B > 2 else [0]
+    pool, L, _ = make_pool(w)
+    S0, u, r, c, piv = oracle_quantised(w, reqs)
+    slots = [W.slot_of_request(b) for b in reqs]
+    T.write_oracle_state(pool, L, slots, u, r, c, piv)
+    rb, om = W.row_bits(w), W.omega(w)
+    st = slots_t(reqs)
+    out = torch.empty((len(reqs), w.H, D), device="cuda")
+    worst_o = 0.0
+    for t in range(steps):
+        x = T.inputs_for(w, "decode", t, reqs)
+        u, r, c, piv, o, X = O.decode_step(u, r, c, piv, rb, om, x.q, x.k, x.v,
+                                           O.gate_rows(x.gate, w.kind, D), x.beta)
+        pool.decode_step(st, dev(x.q), dev(x.k), dev(x.v), dev(x.gate), dev(x.beta), out)
+        worst_o = max(worst_o, T.per_vector_rel_l2(out.cpu().numpy(), o).max())
+    pool.check()
+    Sg = torch.empty((len(reqs), w.H, D, D), device="cuda")
+    pool.dequantize(st, Sg)
+    S_or = O.dequantize(u, r, c, piv, rb)
+    assert T.rel_l2(Sg.cpu().numpy(), S_or) <= T.CHAIN_REL_L2
+    assert worst_o <= T.OUT_REL_L2
+
+
+# ---------------------------------------------------------------------------------
+# full-size workloads in the launch configuration the bench times
+# ---------------------------------------------------------------------------------
+@pytest.mark.parametrize("widx", [3, 4])
+def test_full_size_sampled(widx):
+    w = W.WORKLOADS[widx]
+    pool, L, om = make_pool(w)
+    sample = [int(b) for b in W.parity_sample(w, 3)]
+    # every request gets a state; the sampled ones get oracle-built ones
+    g = torch.Generator(device="cuda").manual_seed(1234 + widx)
+    S_all = torch.randn((w.B, w.H, D, D), device="cuda", generator=g) * 0.05
+    S0 = T.warm_state(widx, tuple(sample))
+    S_all[sample] = dev(S0)
+    all_slots = slots_t(range(w.B))
+    pool.quantize_init(all_slots, S_all)
+    del S_all
+    pool.check()
+    u, r, c, piv = O.refit(S0, om, W.row_bits(w))
+    ug, rg, cg, pg = T.read_pool_state(pool, L, [W.slot_of_request(b) for b in sample])
+    T.compare_codes(ug, u, S0, r, c, W.row_bits(w), "full-size quantize_init")
+    # one decode step over all B requests: random inputs, the sampled requests' from
+    # the seeded generator
+    gen = torch.Generator(device="cuda").manual_seed(99)
+    xin = {
+        "q": torch.nn.functional.normalize(torch.randn((w.B, w.H, D), device="cuda", generator=gen), dim=-1),
+        "k": torch.nn.functional.normalize(torch.randn((w.B, w.H, D), device="cuda", generator=gen), dim=-1),
+        "v": torch.randn((w.B, w.H, D), device="cuda", generator=gen),
+        "gate": torch.exp(torch.empty((w.B, w.H) if w.kind == "gdn" else (w.B, w.H, D),
+                                      device="cuda").uniform_(w.gate_low, w.gate_high, generator=gen)),
+        "beta": torch.sigmoid(torch.randn((w.B, w.H), device="cuda", generator=gen)),
+    }
+    xs = T.inputs_for(w, "decode", 0, sample)
+    for name in xin:
+        xin[name][sample] = dev(getattr(xs, name))
+    out = torch.empty((w.B, w.H, D), device="cuda")
+    pool.decode_step(all_slots, xin["q"], xin["k"], xin["v"], xin["gate"], xin["beta"], out)
+    pool.check()
+    u2, r2, c2, p2, o, X = O.decode_step(u, r, c, piv, W.row_bits(w), om, xs.q, xs.k, xs.v,
+                                         O.gate_rows(xs.gate, w.kind, D), xs.beta)
+    ug, rg, cg, pg = T.read_pool_state(pool, L, [W.slot_of_request(b) for b in sample])
+    T.compare_codes(ug, u2, X, r2, c2, W.row_bits(w), "full-size decode")
+    assert T.per_vector_rel_l2(out[sample].cpu().numpy(), o).max() <= T.OUT_REL_L2
+    assert torch.isfinite(out).all()
+
+
+# ---------------------------------------------------------------------------------
+# edge cases and error paths
+# ---------------------------------------------------------------------------------
+def test_bad_slot_is_flagged_and_skipped():
+    w = W.WORKLOADS[0]
+    pool, L, _ = make_pool(w, n_slots=3)
+    S = torch.zeros((2, w.H, D, D), device="cuda")
+    pool.quantize_init(dev(np.array([0, 2], np.int32)), S)
+    pool.check()
+    before = pool.codes.clone()
+    x = W.step_inputs(w, "decode", 0, 0, 1)
+    out = torch.zeros((2, w.H, D), device="cuda")
+    rep = lambda a: dev(np.concatenate([a, a]))
+    pool.decode_step(dev(np.array([1, 7], np.int32)), rep(x.q), rep(x.k), rep(x.v), rep(x.gate),
+                     rep(x.beta), out)
+    with pytest.raises(stq.StqError) as e:
+        pool.check()
+    assert e.value.status == 4
+    pool.check()            # the error bit was cleared
+    sz = pool.sizes["slot_code_bytes"]
+    assert torch.equal(pool.codes[:sz], before[:sz])           # slot 0 untouched
+    assert torch.count_nonzero(out[1]) == 0                    # skipped request
+
+
+def test_empty_batch_is_a_no_op():
+    w = W.WORKLOADS[0]
+    pool, L, _ = make_pool(w, n_slots=2)
+    e = torch.empty(0, device="cuda")
+    pool.decode_step(torch.empty(0, dtype=torch.int32, device="cuda"), e, e, e, e, e, e)
+    pool.check()
+
+
+def test_zero_state_stays_zero_and_all_pivot_kda_head():
+    # a KDA head whose rows are all FP16 pivots, next to a zero state
+    ub = np.full(2 * D, 6, np.uint8)
+    ub[D:] = 16
+    om = np.ones((2, D), F32)
+    rb = ub.reshape(2, D)
+    pool = stq.Pool("kda", 2, ub, om)
+    L = O.Layout(rb)
+    rng = np.random.default_rng(0)
+    S0 = np.zeros((1, 2, D, D), F32)
+    S0[0, 1] = rng.standard_normal((D, D)).astype(F32)
+    st = dev(np.array([1], np.int32))
+    pool.quantize_init(st, dev(S0))
+    u, r, c, piv = O.refit(S0, om, rb)
+    ug, rg, cg, pg = T.read_pool_state(pool, L, [1])
+    assert np.array_equal(ug, u) and np.array_equal(rg, r) and np.array_equal(cg, c)
+    assert np.array_equal(pg[:, rb == 16], piv[:, rb == 16])
+    q = rng.standard_normal((1, 2, D)).astype(F32)
+    k = (q / np.linalg.norm(q, axis=-1, keepdims=True)).astype(F32)
+    v = rng.standard_normal((1, 2, D)).astype(F32)
+    gate = np.full((1, 2, D), 0.9, F32)
+    beta = np.full((1, 2), 0.5, F32)
+    out = torch.empty((1, 2, D), device="cuda")
+    pool.decode_step(st, dev(k), dev(k), dev(v), dev(gate), dev(beta), out)
+    pool.check()
+    u2, r2, c2, p2, o, X = O.decode_step(u, r, c, piv, rb, om, k, k, v, gate, beta)
+    ug, rg, cg, pg = T.read_pool_state(pool, L, [1])
+    T.compare_codes(ug, u2, X, r2, c2, rb, "pivot head")
+    assert np.array_equal(pg[:, rb == 16], p2[:, rb == 16])
+    assert T.per_vector_rel_l2(out.cpu().numpy(), o).max() <= T.OUT_REL_L2
+
+
+def test_host_entry_point_matches_device_entry_point():
+    w = W.WORKLOADS[1]
+    reqs = [0, 1, 2]
+    pool, L, _ = make_pool(w)
+    S0, u, r, c, piv = oracle_quantised(w, reqs)
+    slots = [W.slot_of_request(b) for b in reqs]
+    x = T.inputs_for(w, "decode", 3, reqs)
+    out_dev = torch.empty((len(reqs), w.H, D), device="cuda")
+    T.write_oracle_state(pool, L, slots, u, r, c, piv)
+    pool.decode_step(slots_t(reqs), dev(x.q), dev(x.k), dev(x.v), dev(x.gate), dev(x.beta), out_dev)
+    pool.check()
+    codes_dev = pool.codes.clone()
+    T.write_oracle_state(pool, L, slots, u, r, c, piv)
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    h_out = torch.empty((len(reqs), w.H, D)).pin_memory()
+    staging = torch.empty(pool.host_staging_bytes(len(reqs)), dtype=torch.uint8, device="cuda")
+    pool.decode_step_host(slots_t(reqs), pin(x.q), pin(x.k), pin(x.v), pin(x.gate), pin(x.beta),
+                          h_out, staging)
+    pool.check()
+    assert torch.equal(pool.codes, codes_dev)
+    assert torch.equal(h_out, out_dev.cpu())
