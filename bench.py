@@ -66,7 +66,7 @@ def algorithmic_bytes(w, B):
     """Bytes a decode step must move: every head's packed codes (or FP16 pivot rows)
     read and written, its scales r[128], c[128] read and written (heads with any
     quantised row), q, k, v, gate, beta read and o written."""
-    rb = W.row_bits(w)
+    rb = W.row_bits(w).astype(np.int64)
     per_req = 0
     for h in range(w.H):
         piv = rb[h] == 16
@@ -236,17 +236,23 @@ def stq_arm(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = W.WORKLOADS[args.workload]
-    B, H = w.B, w.H
+    B, H = (args.batch or w.B), w.H
     ub, om = W.unit_bits(w), W.omega(w)
-    n_slots = W.n_slots(B)
+    if args.compact_slots:       # profiling captures: one slot per request, smaller pool
+        n_slots = B
+        slot_ids = list(range(B))
+    else:
+        n_slots = W.n_slots(B)
+        slot_ids = [W.slot_of_request(b) for b in range(B)]
     pool = stq.Pool(w.kind, n_slots, ub, om, device=dev)
-    slots = torch.tensor([W.slot_of_request(b) for b in range(B)], dtype=torch.int32, device=dev)
+    slots = torch.tensor(slot_ids, dtype=torch.int32, device=dev)
     gen = torch.Generator(device=dev).manual_seed(1000 * args.workload + rank)
 
     # initial states: FP32 warm-up steps from zero on the GPU, outlier rows, quantise
     S = torch.zeros((B, H, D, D), device=dev)
     out = torch.empty((B, H, D), device=dev)
-    for t in range(w.warmup_steps):
+    warm = w.warmup_steps if args.warm_steps < 0 else args.warm_steps
+    for t in range(warm):
         q, k, v, g, b = W.torch_step_inputs(w, B, gen, dev)
         stq.fp32_decode_step(w.kind, S, q, k, v, g, b, out)
     W.torch_scale_outlier_rows(S, w)
@@ -372,6 +378,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-budget", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="override B (profiling captures only)")
+    ap.add_argument("--compact-slots", action="store_true", help="B slots instead of 5B+1 (profiling captures only)")
+    ap.add_argument("--warm-steps", type=int, default=-1, help="override the FP32 warm-up length (profiling only)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
