@@ -44,7 +44,7 @@ size_t up16(size_t x) { return (x + 15) & ~size_t(15); }
 // Host-side layout of one pool, derived from the description.
 struct HostLayout {
   int kind = 0, n_slots = 0, H = 0;
-  std::vector<uint32_t> head_code_off, head_code_bytes, head_piv_first, head_piv_count;
+  std::vector<uint32_t> head_code_off, head_code_bytes, head_piv_first, head_piv_count, head_bits;
   std::vector<uint32_t> row_info;
   std::vector<float> g, omega;
   uint64_t slot_code_bytes = 0;
@@ -69,6 +69,7 @@ stq_status build_layout(const stq_pool_desc* desc, HostLayout& L) {
   L.head_code_bytes.assign(H, 0);
   L.head_piv_first.assign(H, 0);
   L.head_piv_count.assign(H, 0);
+  L.head_bits.assign(H, 0);
   L.row_info.assign(size_t(H) * D, 0);
   L.g.assign(size_t(H) * D, 0.0f);
   L.omega.assign(size_t(H) * D, 0.0f);
@@ -104,6 +105,10 @@ stq_status build_layout(const stq_pool_desc* desc, HostLayout& L) {
         in_head += uint32_t(D * b / 8);
       }
     }
+    uint32_t hb0 = L.row_info[size_t(h) * D] & 0xFFu;
+    for (int i = 1; i < D; ++i)
+      if ((L.row_info[size_t(h) * D + i] & 0xFFu) != hb0) hb0 = 0;
+    L.head_bits[h] = hb0;
     L.head_code_bytes[h] = in_head;
     L.head_piv_count[h] = piv_in_head;
     off += in_head;
@@ -127,6 +132,7 @@ MetaLayout meta_layout(int H) {
   m.head_code_bytes = o; o = up16(o + size_t(H) * 4);
   m.head_piv_first = o;  o = up16(o + size_t(H) * 4);
   m.head_piv_count = o;  o = up16(o + size_t(H) * 4);
+  m.head_bits = o;       o = up16(o + size_t(H) * 4);
   m.row_info = o;        o = up16(o + size_t(H) * D * 4);
   m.g = o;               o = up16(o + size_t(H) * D * 4);
   m.omega = o;           o = up16(o + size_t(H) * D * 4);
@@ -191,6 +197,7 @@ stq_status stq_pool_create(const stq_pool_desc* desc, void* d_codes, void* d_sca
   put(m.head_code_bytes, L.head_code_bytes.data(), L.H * 4);
   put(m.head_piv_first, L.head_piv_first.data(), L.H * 4);
   put(m.head_piv_count, L.head_piv_count.data(), L.H * 4);
+  put(m.head_bits, L.head_bits.data(), L.H * 4);
   put(m.row_info, L.row_info.data(), L.row_info.size() * 4);
   put(m.g, L.g.data(), L.g.size() * 4);
   put(m.omega, L.omega.data(), L.omega.size() * 4);
@@ -211,6 +218,7 @@ stq_status stq_pool_create(const stq_pool_desc* desc, void* d_codes, void* d_sca
   dv.head_code_bytes = reinterpret_cast<const uint32_t*>(mb + m.head_code_bytes);
   dv.head_piv_first = reinterpret_cast<const uint32_t*>(mb + m.head_piv_first);
   dv.head_piv_count = reinterpret_cast<const uint32_t*>(mb + m.head_piv_count);
+  dv.head_bits = reinterpret_cast<const uint32_t*>(mb + m.head_bits);
   dv.row_info = reinterpret_cast<const uint32_t*>(mb + m.row_info);
   dv.g = reinterpret_cast<const float*>(mb + m.g);
   dv.omega = reinterpret_cast<const float*>(mb + m.omega);

@@ -7,20 +7,22 @@
 // per-unit widths and FP16 pivot units (ai-trend review, Method).
 //
 // One CTA of 256 threads owns one (request, head) 128x128 state. Warp w holds key rows
-// 16w..16w+15, lane l holds value columns 4l..4l+3, so a thread keeps 64 state values
-// in registers for the whole step. A row's width is therefore uniform across a warp
-// instruction (KDA widths vary per key row without divergence).
+// 16w..16w+15, lane l holds value columns 4l..4l+3 as two float2 pairs, so a thread keeps
+// 64 state values in registers for the whole step. A row's width is uniform across a
+// warp instruction (KDA widths vary per key row without divergence); heads whose rows
+// share one width run a code path specialised for it.
 //
 // Float32 evaluation order (the CPU oracle restates the same order):
-//   * every product is rounded before it is added (explicit __fmul_rn/__fadd_rn; the
-//     file is also built with --fmad=false);
+//   * every product is rounded before it is added (explicit _rn intrinsics, including
+//     the packed float2 forms __fmul2_rn/__fadd2_rn; the file is also built with
+//     --fmad=false);
 //   * sums over the 128 rows of a column or the 128 columns of a row are balanced
-//     binary trees: adjacent pairs first. Column sums: a thread's 16 rows form the
-//     lower 4 levels, the 8 warps (smem) the top 3. Row sums: a thread's 4 columns form
-//     the lower 2 levels, 5 butterfly shuffle steps (xor 1,2,...,16) the top 5;
+//     binary trees, adjacent pairs first. Column sums: a thread's 16 rows form the
+//     lower 4 levels, the 8 warps (shared memory) the top 3. Row sums: a thread's 4
+//     columns form the lower 2 levels, butterfly shuffle steps xor 1,2,...,16 the top 5;
 //   * the quantiser's x = y * inv_c is taken exactly: fma(y, inv_c, 1.5*2^23) rounds the
 //     exact product to the nearest integer (ties to even) inside the 2^23 binade, and
-//     clamping is done in that same binade.
+//     clamping is done in that binade, where the low bits are the (biased) code.
 #include <cuda_fp16.h>
 
 #include "stq_internal.h"
@@ -33,10 +35,21 @@ constexpr int NW = 8;     // warps per head-state
 constexpr int RPW = 16;   // key rows per warp
 constexpr float MAGIC = 12582912.0f;        // 1.5 * 2^23
 constexpr float TWO23 = 8388608.0f;         // 2^23
+constexpr uint32_t FLOAT_2P23 = 0x4B000000u;
 constexpr float SMALLEST_NORMAL = 1.17549435e-38f;  // 2^-126
+constexpr int MIXED = 0;
+
+using f2 = float2;
 
 __device__ __forceinline__ float fmul(float a, float b) { return __fmul_rn(a, b); }
 __device__ __forceinline__ float fadd(float a, float b) { return __fadd_rn(a, b); }
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ f2 add2(f2 a, f2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ f2 dup(float x) { return make_float2(x, x); }
+__device__ __forceinline__ float at4(const float4& v, int i) {
+  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
 
 // 1/a correctly rounded for a >= 2^-126; 0 for a smaller (or zero) scale.
 __device__ __forceinline__ float recip_scale(float a) {
@@ -44,21 +57,21 @@ __device__ __forceinline__ float recip_scale(float a) {
 }
 
 template <int N>
-struct Vec {
-  float x[N];
+struct V2 {
+  f2 x[N];
 };
 
-// Balanced binary tree over leaves f(LO), ..., f(LO+N-1); each leaf is a Vec<M> of
-// independent sums (one per value column held by the thread).
+// Balanced binary tree over leaves f(LO), ..., f(LO+N-1), each a V2<M> of independent
+// column sums.
 template <int LO, int N, int M, class F>
-__device__ __forceinline__ Vec<M> tree(F&& f) {
+__device__ __forceinline__ V2<M> tree(F&& f) {
   if constexpr (N == 1) {
     return f(LO);
   } else {
-    Vec<M> a = tree<LO, N / 2, M>(f);
-    Vec<M> b = tree<LO + N / 2, N / 2, M>(f);
+    V2<M> a = tree<LO, N / 2, M>(f);
+    V2<M> b = tree<LO + N / 2, N / 2, M>(f);
 #pragma unroll
-    for (int m = 0; m < M; ++m) a.x[m] = fadd(a.x[m], b.x[m]);
+    for (int m = 0; m < M; ++m) a.x[m] = add2(a.x[m], b.x[m]);
     return a;
   }
 }
@@ -69,58 +82,82 @@ struct __align__(16) HeadSmem {
   float inv_r[D];    // 1/r_i of the refit
   float b[D];        // omega_i * r_i^2
   float qm[D];       // qmax_i (0 for pivot rows)
-  float inv_qm[D];   // 1/qmax_i (0 for pivot rows)
+  float iq[D];       // 1/qmax_i (0 for pivot rows)
   float mb[D];       // 1.5*2^23 + 2^(b-1): magic that yields the biased code
+  float tb[D];       // 2^23 + 2^(b-1): magic that turns a code into its value
   uint32_t info[D];  // bits | offset << 8
-  float red[2][2][NW][D];  // ping-pong partial sums: [buffer][quantity][warp][column]
+  float4 red[2][2][NW][D / 4];  // ping-pong partials: [buffer][quantity][warp][col/4]
   float beta;
 };
 
 __device__ __forceinline__ int row_bits(uint32_t info) { return int(info & 0xFFu); }
 __device__ __forceinline__ int row_off(uint32_t info) { return int(info >> 8); }
 
-// The 4*bits-bit field holding codes 4*lane .. 4*lane+3 of one row: code j of a b-bit
-// row is bits [b*j, b*j+b) of a little-endian bit stream. `row` is 16-byte aligned.
-__device__ __forceinline__ uint32_t lane_field(const uint8_t* row, int bits, int lane) {
-  if (bits == 8) return reinterpret_cast<const uint32_t*>(row)[lane];
-  if (bits == 4) return reinterpret_cast<const uint16_t*>(row)[lane];
-  if (bits == 2) return row[lane];
-  // 6 bits: bytes 3*lane .. 3*lane+2, within word 3*lane/4 and possibly the next one
-  const uint32_t* wp = reinterpret_cast<const uint32_t*>(row);
-  const int byte = 3 * lane, wi = byte >> 2, sh = (byte & 3) * 8;
-  const uint32_t lo = wp[wi];
-  const uint32_t hi = (sh > 8) ? wp[wi + 1] : 0u;  // wi + 1 <= 23 whenever sh > 8
-  return __funnelshift_r(lo, hi, sh) & 0xFFFFFFu;
-}
+// ---------------------------------------------------------------------------------
+// code formats: code j of a b-bit row is bits [b*j, b*j+b) of a little-endian stream;
+// lane l owns codes 4l..4l+3 = bits [4bl, 4bl+4b) = bytes [bl/2, bl/2 + b/2)
+// ---------------------------------------------------------------------------------
 
-__device__ __forceinline__ void store_field(uint8_t* row, int bits, int lane, uint32_t f) {
-  if (bits == 8) {
-    reinterpret_cast<uint32_t*>(row)[lane] = f;
-  } else if (bits == 4) {
-    reinterpret_cast<uint16_t*>(row)[lane] = static_cast<uint16_t>(f);
-  } else if (bits == 2) {
-    row[lane] = static_cast<uint8_t>(f);
+// The four codes of a lane as floats 2^23 + u (exact), from a 16-byte aligned row.
+template <int BITS>
+__device__ __forceinline__ void load_codes(const uint8_t* row, int lane, uint32_t (&c)[4]) {
+  if constexpr (BITS == 8) {
+    const uint32_t w = reinterpret_cast<const uint32_t*>(row)[lane];
+    c[0] = __byte_perm(w, FLOAT_2P23, 0x7540);
+    c[1] = __byte_perm(w, FLOAT_2P23, 0x7541);
+    c[2] = __byte_perm(w, FLOAT_2P23, 0x7542);
+    c[3] = __byte_perm(w, FLOAT_2P23, 0x7543);
   } else {
-    uint8_t* p = row + 3 * lane;
-    p[0] = static_cast<uint8_t>(f);
-    p[1] = static_cast<uint8_t>(f >> 8);
-    p[2] = static_cast<uint8_t>(f >> 16);
+    uint32_t f;
+    if constexpr (BITS == 4) {
+      f = reinterpret_cast<const uint16_t*>(row)[lane];
+    } else if constexpr (BITS == 2) {
+      f = row[lane];
+    } else {
+      // 6 bits: bytes 3l..3l+2, inside word 3l/4 and possibly the next one
+      const uint32_t* wp = reinterpret_cast<const uint32_t*>(row);
+      const int byte = 3 * lane, wi = byte >> 2, sh = (byte & 3) * 8;
+      const uint32_t lo = wp[wi];
+      const uint32_t hi = (sh > 8) ? wp[wi + 1] : 0u;  // wi + 1 <= 23 whenever sh > 8
+      f = __funnelshift_r(lo, hi, sh);
+    }
+    constexpr uint32_t M = (1u << BITS) - 1u;
+    c[0] = (f & M) | FLOAT_2P23;
+    c[1] = ((f >> BITS) & M) | FLOAT_2P23;
+    c[2] = ((f >> (2 * BITS)) & M) | FLOAT_2P23;
+    c[3] = ((f >> (3 * BITS)) & M) | FLOAT_2P23;
   }
 }
 
-// Code u (< 2^22) minus its bias, as an exact float: (2^23 + u) - (2^23 + bias).
-__device__ __forceinline__ float code_value(uint32_t u, float two23_plus_bias) {
-  return __fsub_rn(__uint_as_float(u | 0x4B000000u), two23_plus_bias);
+// Pack four biased codes (low bits of t = 1.5*2^23 + u) and store them into a row.
+template <int BITS>
+__device__ __forceinline__ void store_codes(uint8_t* row, int lane, const uint32_t (&t)[4]) {
+  if constexpr (BITS == 8) {
+    const uint32_t p01 = __byte_perm(t[0], t[1], 0x0040);
+    const uint32_t p23 = __byte_perm(t[2], t[3], 0x0040);
+    reinterpret_cast<uint32_t*>(row)[lane] = __byte_perm(p01, p23, 0x5410);
+  } else {
+    constexpr uint32_t M = (1u << BITS) - 1u;
+    const uint32_t f = (t[0] & M) | ((t[1] & M) << BITS) | ((t[2] & M) << (2 * BITS)) |
+                       ((t[3] & M) << (3 * BITS));
+    if constexpr (BITS == 4) {
+      reinterpret_cast<uint16_t*>(row)[lane] = static_cast<uint16_t>(f);
+    } else if constexpr (BITS == 2) {
+      row[lane] = static_cast<uint8_t>(f);
+    } else {
+      // 24 bits at byte 3l: one 16-bit and one 8-bit store, the 16-bit one aligned
+      const bool odd = lane & 1;
+      uint8_t* p = row + 3 * lane;
+      uint8_t* p8 = odd ? p : p + 2;
+      uint16_t* p16 = reinterpret_cast<uint16_t*>(odd ? p + 1 : p);
+      *p8 = static_cast<uint8_t>(odd ? f : (f >> 16));
+      *p16 = static_cast<uint16_t>(odd ? (f >> 8) : f);
+    }
+  }
 }
 
-// Copy `bytes` (multiple of 16) from global to shared with 16-byte accesses.
+// Copy `bytes` (multiple of 16) with 16-byte accesses by the whole CTA.
 __device__ __forceinline__ void copy16(void* dst, const void* src, int bytes) {
-  const uint4* s = reinterpret_cast<const uint4*>(src);
-  uint4* d = reinterpret_cast<uint4*>(dst);
-  for (int t = threadIdx.x; t < (bytes >> 4); t += NT) d[t] = s[t];
-}
-
-__device__ __forceinline__ void copy16_out(void* dst, const void* src, int bytes) {
   const uint4* s = reinterpret_cast<const uint4*>(src);
   uint4* d = reinterpret_cast<uint4*>(dst);
   for (int t = threadIdx.x; t < (bytes >> 4); t += NT) d[t] = s[t];
@@ -132,6 +169,7 @@ struct HeadRef {
   float* scales;       // global: r[D], c[D] of this head in its slot
   int code_bytes;
   int piv_count;
+  int bits;            // uniform width of the head, 16 if all pivot, 0 if mixed
   int piv_stage_off;   // byte offset of the pivot rows in the staging buffer
 };
 
@@ -139,6 +177,7 @@ __device__ __forceinline__ HeadRef head_ref(const PoolDev& P, int slot, int h) {
   HeadRef r;
   r.code_bytes = int(P.head_code_bytes[h]);
   r.piv_count = int(P.head_piv_count[h]);
+  r.bits = int(P.head_bits[h]);
   r.codes = P.codes + uint64_t(slot) * P.slot_code_bytes + P.head_code_off[h];
   r.pivots = P.pivots + (uint64_t(slot) * P.n_pivot_rows + P.head_piv_first[h]) * D;
   r.scales = P.scales + (uint64_t(slot) * P.H + h) * 2 * D;
@@ -155,35 +194,73 @@ __device__ __forceinline__ void load_row_meta(const PoolDev& P, int h, HeadSmem&
     sm.info[i] = info;
     if (bits == PIVOT) {
       sm.qm[i] = 0.0f;
-      sm.inv_qm[i] = 0.0f;
+      sm.iq[i] = 0.0f;
       sm.mb[i] = MAGIC;
+      sm.tb[i] = TWO23;
     } else {
       const int bias = 1 << (bits - 1);
       sm.qm[i] = float(bias - 1);
-      sm.inv_qm[i] = __frcp_rn(float(bias - 1));
+      sm.iq[i] = __frcp_rn(float(bias - 1));
       sm.mb[i] = MAGIC + float(bias);
+      sm.tb[i] = TWO23 + float(bias);
     }
   }
 }
 
+__device__ __forceinline__ uint2 half4_bits(f2 a, f2 b) {
+  const uint32_t lo = uint32_t(__half_as_ushort(__float2half_rn(a.x))) |
+                      (uint32_t(__half_as_ushort(__float2half_rn(a.y))) << 16);
+  const uint32_t hi = uint32_t(__half_as_ushort(__float2half_rn(b.x))) |
+                      (uint32_t(__half_as_ushort(__float2half_rn(b.y))) << 16);
+  return make_uint2(lo, hi);
+}
+
+__device__ __forceinline__ void half4_floats(uint2 hv, f2& a, f2& b) {
+  a.x = __half2float(__ushort_as_half(uint16_t(hv.x & 0xFFFFu)));
+  a.y = __half2float(__ushort_as_half(uint16_t(hv.x >> 16)));
+  b.x = __half2float(__ushort_as_half(uint16_t(hv.y & 0xFFFFu)));
+  b.y = __half2float(__ushort_as_half(uint16_t(hv.y >> 16)));
+}
+
+// Sum of the 8 warps' partials of one quantity for this lane's 4 columns, as a tree
+// ((w0+w1)+(w2+w3))+((w4+w5)+(w6+w7)).
+__device__ __forceinline__ void warp_tree(const float4 (*red)[D / 4], int lane, f2& lo, f2& hi) {
+  f2 a[NW], b[NW];
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const float4 v = red[w][lane];
+    a[w] = make_float2(v.x, v.y);
+    b[w] = make_float2(v.z, v.w);
+  }
+  lo = add2(add2(add2(a[0], a[1]), add2(a[2], a[3])), add2(add2(a[4], a[5]), add2(a[6], a[7])));
+  hi = add2(add2(add2(b[0], b[1]), add2(b[2], b[3])), add2(add2(b[4], b[5]), add2(b[6], b[7])));
+}
+
+__device__ __forceinline__ void put_partial(float4 (*red)[D / 4], int w, int lane, f2 lo, f2 hi) {
+  red[w][lane] = make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
 // ---------------------------------------------------------------------------------
 // Refit: row scale, column scale start, two omega-weighted least-squares steps, final
-// codes (bloombook section 4; singularity-lens dual-axis paragraph). On entry the
-// thread's 64 values s[][] hold the float32 state (pivot rows already stored) and the
-// caller may have put readout partials into red[1][0]. On exit the packed codes of the
-// head are in `stage`, r has been written to global, and c is returned in c_out.
+// codes (bloombook section 4; singularity-lens dual-axis paragraph). On entry s[][]
+// holds the float32 state (pivot rows already stored) and the caller may have put
+// readout partials into red[1][0]. On exit the head's packed codes are in `stage`,
+// r has been written to global, and c is returned in c_out (this lane's columns).
+// BITS is the head's uniform width, or MIXED for per-row widths.
 // ---------------------------------------------------------------------------------
+template <int BITS>
 __device__ __forceinline__ void refit_pack(const PoolDev& P, int h, HeadSmem& sm, uint8_t* stage,
-                                           float (&s)[RPW][4], float* r_global,
-                                           float (&c_out)[4], float* o_global) {
+                                           f2 (&s)[RPW][2], float* r_global, f2 (&c_out)[2],
+                                           float* o_global) {
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r0 = w * RPW;
 
   // --- row scale r_i = (tree sum_j |S_ij|) / 128 * g_i -------------------------------
   float a[RPW];
 #pragma unroll
   for (int rr = 0; rr < RPW; ++rr)
-    a[rr] = fadd(fadd(fabsf(s[rr][0]), fabsf(s[rr][1])), fadd(fabsf(s[rr][2]), fabsf(s[rr][3])));
-  // reduce-scatter over lanes: step m keeps half of the rows, pairs lane l with l^m
+    a[rr] = fadd(fadd(fabsf(s[rr][0].x), fabsf(s[rr][0].y)), fadd(fabsf(s[rr][1].x), fabsf(s[rr][1].y)));
+  // reduce-scatter over lanes: step m keeps half of the rows and pairs lane l with l^m
 #pragma unroll
   for (int t = 0; t < 8; ++t) {
     const bool up = lane & 1;
@@ -213,10 +290,10 @@ __device__ __forceinline__ void refit_pack(const PoolDev& P, int h, HeadSmem& sm
   }
   a[0] = fadd(a[0], __shfl_xor_sync(0xffffffffu, a[0], 16));
   {
-    // lane l now holds the full sum of row R(l): bits 0..3 of l select halves 8,4,2,1
+    // lane l now holds the sum of row R(l): bits 0..3 of l chose halves 8, 4, 2, 1
     const int R = ((lane & 1) << 3) | ((lane & 2) << 1) | ((lane & 4) >> 1) | ((lane & 8) >> 3);
-    const int i = w * RPW + R;
-    const bool pivot = row_bits(sm.info[i]) == PIVOT;
+    const int i = r0 + R;
+    const bool pivot = (BITS == MIXED) ? (row_bits(sm.info[i]) == PIVOT) : false;
     const float g = P.g[h * D + i];
     const float om = P.omega[h * D + i];
     const float r = pivot ? 0.0f : fmul(fmul(a[0], 0.0078125f), g);
@@ -231,96 +308,316 @@ __device__ __forceinline__ void refit_pack(const PoolDev& P, int h, HeadSmem& sm
   // --- y = S * inv_r; column start c0_j = max_i |y_ij| / qmax_i -----------------------
   float mx[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-  for (int rr = 0; rr < RPW; ++rr) {
-    const int i = w * RPW + rr;
-    const float ir = sm.inv_r[i], iq = sm.inv_qm[i];
+  for (int g4 = 0; g4 < RPW / 4; ++g4) {
+    const float4 ir4 = *reinterpret_cast<const float4*>(&sm.inv_r[r0 + 4 * g4]);
+    float4 iq4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if constexpr (BITS == MIXED) iq4 = *reinterpret_cast<const float4*>(&sm.iq[r0 + 4 * g4]);
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      s[rr][cc] = fmul(s[rr][cc], ir);
-      mx[cc] = fmaxf(mx[cc], fmul(fabsf(s[rr][cc]), iq));
+    for (int j = 0; j < 4; ++j) {
+      const int rr = 4 * g4 + j;
+      const f2 ir = dup(at4(ir4, j));
+      s[rr][0] = mul2(s[rr][0], ir);
+      s[rr][1] = mul2(s[rr][1], ir);
+      if constexpr (BITS == MIXED) {
+        const float iq = at4(iq4, j);
+        mx[0] = fmaxf(mx[0], fmul(fabsf(s[rr][0].x), iq));
+        mx[1] = fmaxf(mx[1], fmul(fabsf(s[rr][0].y), iq));
+        mx[2] = fmaxf(mx[2], fmul(fabsf(s[rr][1].x), iq));
+        mx[3] = fmaxf(mx[3], fmul(fabsf(s[rr][1].y), iq));
+      } else {
+        mx[0] = fmaxf(mx[0], fabsf(s[rr][0].x));
+        mx[1] = fmaxf(mx[1], fabsf(s[rr][0].y));
+        mx[2] = fmaxf(mx[2], fabsf(s[rr][1].x));
+        mx[3] = fmaxf(mx[3], fabsf(s[rr][1].y));
+      }
     }
   }
-  *reinterpret_cast<float4*>(&sm.red[1][1][w][4 * lane]) = make_float4(mx[0], mx[1], mx[2], mx[3]);
+  sm.red[1][1][w][lane] = make_float4(mx[0], mx[1], mx[2], mx[3]);
   __syncthreads();
 
   if (o_global != nullptr && w == 0) {
-    float o[4];
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      const int j = 4 * lane + cc;
-      o[cc] = fadd(fadd(fadd(sm.red[1][0][0][j], sm.red[1][0][1][j]), fadd(sm.red[1][0][2][j], sm.red[1][0][3][j])),
-                   fadd(fadd(sm.red[1][0][4][j], sm.red[1][0][5][j]), fadd(sm.red[1][0][6][j], sm.red[1][0][7][j])));
-    }
-    *reinterpret_cast<float4*>(o_global + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
+    f2 lo, hi;
+    warp_tree(sm.red[1][0], lane, lo, hi);
+    *reinterpret_cast<float4*>(o_global + 4 * lane) = make_float4(lo.x, lo.y, hi.x, hi.y);
   }
-  float c[4];
+  f2 c[2];
+  {
+    float m[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-  for (int cc = 0; cc < 4; ++cc) {
-    float m = 0.0f;
+    for (int ww = 0; ww < NW; ++ww) {
+      const float4 v = sm.red[1][1][ww][lane];
+      m[0] = fmaxf(m[0], v.x); m[1] = fmaxf(m[1], v.y); m[2] = fmaxf(m[2], v.z); m[3] = fmaxf(m[3], v.w);
+    }
+    if constexpr (BITS != MIXED) {
+      // max_i RN(|y| / qmax) = RN(max_i |y| / qmax): rounding is monotone
+      constexpr float QM = float((1 << (BITS - 1)) - 1);
+      const float iq = __frcp_rn(QM);
 #pragma unroll
-    for (int ww = 0; ww < NW; ++ww) m = fmaxf(m, sm.red[1][1][ww][4 * lane + cc]);
-    c[cc] = m;
+      for (int t = 0; t < 4; ++t) m[t] = fmul(m[t], iq);
+    }
+    c[0] = make_float2(m[0], m[1]);
+    c[1] = make_float2(m[2], m[3]);
   }
 
   // --- two least-squares steps: c_j <- sum_i p y / sum_i p Q, p = b_i Q_ij -------------
 #pragma unroll
   for (int it = 0; it < 2; ++it) {
-    float ic[4];
+    const f2 ic[2] = {make_float2(recip_scale(c[0].x), recip_scale(c[0].y)),
+                      make_float2(recip_scale(c[1].x), recip_scale(c[1].y))};
+    float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f), q4 = b4;
+    V2<4> nd = tree<0, RPW, 4>([&](int rr) {
+      if ((rr & 3) == 0) {
+        b4 = *reinterpret_cast<const float4*>(&sm.b[r0 + rr]);
+        if constexpr (BITS == MIXED) q4 = *reinterpret_cast<const float4*>(&sm.qm[r0 + rr]);
+      }
+      const f2 bb = dup(at4(b4, rr & 3));
+      float lo_b, hi_b;
+      if constexpr (BITS == MIXED) {
+        lo_b = MAGIC - at4(q4, rr & 3);
+        hi_b = MAGIC + at4(q4, rr & 3);
+      } else {
+        lo_b = MAGIC - float((1 << (BITS - 1)) - 1);
+        hi_b = MAGIC + float((1 << (BITS - 1)) - 1);
+      }
+      V2<4> leaf;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) ic[cc] = recip_scale(c[cc]);
-    Vec<8> nd = tree<0, RPW, 8>([&](int rr) {
-      const int i = w * RPW + rr;
-      const float bi = sm.b[i], q = sm.qm[i];
-      Vec<8> leaf;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        float t = __fmaf_rn(s[rr][cc], ic[cc], MAGIC);
-        if (it > 0) t = fminf(fmaxf(t, MAGIC - q), MAGIC + q);  // step one never clips
-        const float Q = __fsub_rn(t, MAGIC);
-        const float p = fmul(bi, Q);
-        leaf.x[cc] = fmul(p, s[rr][cc]);
-        leaf.x[4 + cc] = fmul(p, Q);
+      for (int hh = 0; hh < 2; ++hh) {
+        f2 t = fma2(s[rr][hh], ic[hh], dup(MAGIC));
+        if (it > 0) {  // step one never clips: c0 is the column maximum
+          t.x = fminf(fmaxf(t.x, lo_b), hi_b);
+          t.y = fminf(fmaxf(t.y, lo_b), hi_b);
+        }
+        const f2 Q = add2(t, dup(-MAGIC));
+        const f2 p = mul2(bb, Q);
+        leaf.x[hh] = mul2(p, s[rr][hh]);
+        leaf.x[2 + hh] = mul2(p, Q);
       }
       return leaf;
     });
-    float(*buf)[NW][D] = sm.red[it];
-    *reinterpret_cast<float4*>(&buf[0][w][4 * lane]) = make_float4(nd.x[0], nd.x[1], nd.x[2], nd.x[3]);
-    *reinterpret_cast<float4*>(&buf[1][w][4 * lane]) = make_float4(nd.x[4], nd.x[5], nd.x[6], nd.x[7]);
+    float4 (*const num)[D / 4] = sm.red[it][0];
+    float4 (*const den)[D / 4] = sm.red[it][1];
+    put_partial(num, w, lane, nd.x[0], nd.x[1]);
+    put_partial(den, w, lane, nd.x[2], nd.x[3]);
     __syncthreads();
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      const int j = 4 * lane + cc;
-      const float num = fadd(fadd(fadd(buf[0][0][j], buf[0][1][j]), fadd(buf[0][2][j], buf[0][3][j])),
-                             fadd(fadd(buf[0][4][j], buf[0][5][j]), fadd(buf[0][6][j], buf[0][7][j])));
-      const float den = fadd(fadd(fadd(buf[1][0][j], buf[1][1][j]), fadd(buf[1][2][j], buf[1][3][j])),
-                             fadd(fadd(buf[1][4][j], buf[1][5][j]), fadd(buf[1][6][j], buf[1][7][j])));
-      if (den > 0.0f) c[cc] = __fdiv_rn(num, den);
-    }
+    f2 nlo, nhi, dlo, dhi;
+    warp_tree(num, lane, nlo, nhi);
+    warp_tree(den, lane, dlo, dhi);
+    if (dlo.x > 0.0f) c[0].x = __fdiv_rn(nlo.x, dlo.x);
+    if (dlo.y > 0.0f) c[0].y = __fdiv_rn(nlo.y, dlo.y);
+    if (dhi.x > 0.0f) c[1].x = __fdiv_rn(nhi.x, dhi.x);
+    if (dhi.y > 0.0f) c[1].y = __fdiv_rn(nhi.y, dhi.y);
   }
 
   // --- final codes with the final c, packed into the staging buffer --------------------
-  float ic[4];
-#pragma unroll
-  for (int cc = 0; cc < 4; ++cc) ic[cc] = recip_scale(c[cc]);
+  const f2 ic[2] = {make_float2(recip_scale(c[0].x), recip_scale(c[0].y)),
+                    make_float2(recip_scale(c[1].x), recip_scale(c[1].y))};
 #pragma unroll
   for (int rr = 0; rr < RPW; ++rr) {
-    const int i = w * RPW + rr;
-    const uint32_t info = sm.info[i];
-    const int bits = row_bits(info);
-    if (bits == PIVOT) continue;
-    const float mb = sm.mb[i], q = sm.qm[i];
-    uint32_t field = 0;
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      float t = __fmaf_rn(s[rr][cc], ic[cc], mb);
-      t = fminf(fmaxf(t, mb - q), mb + q);
-      const uint32_t u = __float_as_uint(t) & 0xFFu;
-      field |= u << (bits * cc);
+    const int i = r0 + rr;
+    if constexpr (BITS == MIXED) {
+      const uint32_t info = sm.info[i];
+      const int bits = row_bits(info);
+      if (bits == PIVOT) continue;
+      const float mb = sm.mb[i], q = sm.qm[i];
+      const f2 t01 = fma2(s[rr][0], ic[0], dup(mb));
+      const f2 t23 = fma2(s[rr][1], ic[1], dup(mb));
+      const float lo_b = mb - q, hi_b = mb + q;
+      const uint32_t t[4] = {__float_as_uint(fminf(fmaxf(t01.x, lo_b), hi_b)),
+                             __float_as_uint(fminf(fmaxf(t01.y, lo_b), hi_b)),
+                             __float_as_uint(fminf(fmaxf(t23.x, lo_b), hi_b)),
+                             __float_as_uint(fminf(fmaxf(t23.y, lo_b), hi_b))};
+      uint8_t* row = stage + row_off(info);
+      switch (bits) {
+        case 2: store_codes<2>(row, lane, t); break;
+        case 4: store_codes<4>(row, lane, t); break;
+        case 6: store_codes<6>(row, lane, t); break;
+        default: store_codes<8>(row, lane, t); break;
+      }
+    } else {
+      constexpr float MB = MAGIC + float(1 << (BITS - 1));
+      constexpr float QM = float((1 << (BITS - 1)) - 1);
+      const f2 t01 = fma2(s[rr][0], ic[0], dup(MB));
+      const f2 t23 = fma2(s[rr][1], ic[1], dup(MB));
+      const uint32_t t[4] = {__float_as_uint(fminf(fmaxf(t01.x, MB - QM), MB + QM)),
+                             __float_as_uint(fminf(fmaxf(t01.y, MB - QM), MB + QM)),
+                             __float_as_uint(fminf(fmaxf(t23.x, MB - QM), MB + QM)),
+                             __float_as_uint(fminf(fmaxf(t23.y, MB - QM), MB + QM))};
+      store_codes<BITS>(stage + rr * (D * BITS / 8) + r0 * (D * BITS / 8), lane, t);
     }
-    store_field(stage + row_off(info), bits, lane, field);
   }
+  c_out[0] = c[0];
+  c_out[1] = c[1];
+}
+
+// Restore one row of S' = D (r c Q) for this lane's 4 columns.
+template <int BITS>
+__device__ __forceinline__ void restore_row(const uint8_t* row, int lane, float rd, float tb,
+                                            const f2 (&cin)[2], f2& s01, f2& s23) {
+  uint32_t cd[4];
+  load_codes<BITS>(row, lane, cd);
+  const f2 ntb = dup(-tb);
+  const f2 q01 = add2(make_float2(__uint_as_float(cd[0]), __uint_as_float(cd[1])), ntb);
+  const f2 q23 = add2(make_float2(__uint_as_float(cd[2]), __uint_as_float(cd[3])), ntb);
+  s01 = mul2(mul2(q01, dup(rd)), cin[0]);
+  s23 = mul2(mul2(q23, dup(rd)), cin[1]);
+}
+
+// ---------------------------------------------------------------------------------
+// One (request, head) of stq_decode_step.
+// ---------------------------------------------------------------------------------
+template <int BITS>
+__device__ __forceinline__ void decode_head(const PoolDev& P, int h, HeadSmem& sm, uint8_t* stage,
+                                            const HeadRef& hr, const f2 (&cin)[2], float* o_out) {
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int r0 = w * RPW;
+  f2 s[RPW][2];
+
+  // ---- restore S' and the column sums u_j = sum_i k_i S'_ij ---------------------------
 #pragma unroll
-  for (int cc = 0; cc < 4; ++cc) c_out[cc] = c[cc];
+  for (int g4 = 0; g4 < RPW / 4; ++g4) {
+    const float4 rd4 = *reinterpret_cast<const float4*>(&sm.rd[r0 + 4 * g4]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int rr = 4 * g4 + j, i = r0 + rr;
+      if constexpr (BITS == MIXED) {
+        const uint32_t info = sm.info[i];
+        const int bits = row_bits(info);
+        const uint8_t* row = stage + row_off(info);
+        const float tb = sm.tb[i];
+        switch (bits) {
+          case 2: restore_row<2>(row, lane, at4(rd4, j), tb, cin, s[rr][0], s[rr][1]); break;
+          case 4: restore_row<4>(row, lane, at4(rd4, j), tb, cin, s[rr][0], s[rr][1]); break;
+          case 6: restore_row<6>(row, lane, at4(rd4, j), tb, cin, s[rr][0], s[rr][1]); break;
+          case 8: restore_row<8>(row, lane, at4(rd4, j), tb, cin, s[rr][0], s[rr][1]); break;
+          default: {
+            const uint2 hv = *reinterpret_cast<const uint2*>(stage + hr.piv_stage_off +
+                                                              row_off(info) * (D * 2) + 8 * lane);
+            f2 a, b;
+            half4_floats(hv, a, b);
+            const f2 dd = dup(sm.dec[i]);
+            s[rr][0] = mul2(dd, a);
+            s[rr][1] = mul2(dd, b);
+          }
+        }
+      } else {
+        constexpr float TB = TWO23 + float(1 << (BITS - 1));
+        restore_row<BITS>(stage + i * (D * BITS / 8), lane, at4(rd4, j), TB, cin, s[rr][0], s[rr][1]);
+      }
+    }
+  }
+  {
+    float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    V2<2> u = tree<0, RPW, 2>([&](int rr) {
+      if ((rr & 3) == 0) k4 = *reinterpret_cast<const float4*>(&sm.k[r0 + rr]);
+      const f2 kk = dup(at4(k4, rr & 3));
+      V2<2> leaf;
+      leaf.x[0] = mul2(kk, s[rr][0]);
+      leaf.x[1] = mul2(kk, s[rr][1]);
+      return leaf;
+    });
+    put_partial(sm.red[0][0], w, lane, u.x[0], u.x[1]);
+  }
+  __syncthreads();
+
+  // ---- delta_j = beta (v_j - u_j); S = S' + k delta^T; readout partials ----------------
+  f2 delta[2];
+  {
+    f2 ulo, uhi;
+    warp_tree(sm.red[0][0], lane, ulo, uhi);
+    const float4 v4 = *reinterpret_cast<const float4*>(&sm.v[4 * lane]);
+    const f2 bt = dup(sm.beta);
+    delta[0] = mul2(bt, add2(make_float2(v4.x, v4.y), make_float2(-ulo.x, -ulo.y)));
+    delta[1] = mul2(bt, add2(make_float2(v4.z, v4.w), make_float2(-uhi.x, -uhi.y)));
+  }
+  {
+    float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f), q4 = k4;
+    V2<2> o = tree<0, RPW, 2>([&](int rr) {
+      if ((rr & 3) == 0) {
+        k4 = *reinterpret_cast<const float4*>(&sm.k[r0 + rr]);
+        q4 = *reinterpret_cast<const float4*>(&sm.q[r0 + rr]);
+      }
+      const f2 kk = dup(at4(k4, rr & 3)), qq = dup(at4(q4, rr & 3));
+      s[rr][0] = add2(s[rr][0], mul2(kk, delta[0]));
+      s[rr][1] = add2(s[rr][1], mul2(kk, delta[1]));
+      V2<2> leaf;
+      leaf.x[0] = mul2(qq, s[rr][0]);
+      leaf.x[1] = mul2(qq, s[rr][1]);
+      return leaf;
+    });
+    put_partial(sm.red[1][0], w, lane, o.x[0], o.x[1]);
+  }
+  if constexpr (BITS == MIXED) {
+    // pivot rows: store float16(S) now (they take no part in the refit)
+#pragma unroll
+    for (int rr = 0; rr < RPW; ++rr) {
+      const uint32_t info = sm.info[r0 + rr];
+      if (row_bits(info) == PIVOT)
+        *reinterpret_cast<uint2*>(hr.pivots + row_off(info) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
+    }
+  }
+  f2 c[2];
+  refit_pack<BITS>(P, h, sm, stage, s, hr.scales, c, o_out);
+  __syncthreads();
+  copy16(hr.codes, stage, hr.code_bytes);
+  if (w == 0) *reinterpret_cast<float4*>(hr.scales + D + 4 * lane) = make_float4(c[0].x, c[0].y, c[1].x, c[1].y);
+}
+
+// A head whose rows are all FP16 pivots: decay, update, readout, store float16; r = c = 0.
+__device__ __forceinline__ void decode_pivot_head(HeadSmem& sm, uint8_t* stage, const HeadRef& hr,
+                                                  float* o_out) {
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int r0 = w * RPW;
+  f2 s[RPW][2];
+#pragma unroll
+  for (int rr = 0; rr < RPW; ++rr) {
+    const int i = r0 + rr;
+    const uint2 hv = *reinterpret_cast<const uint2*>(stage + i * (D * 2) + 8 * lane);
+    f2 a, b;
+    half4_floats(hv, a, b);
+    const f2 dd = dup(sm.dec[i]);
+    s[rr][0] = mul2(dd, a);
+    s[rr][1] = mul2(dd, b);
+  }
+  {
+    V2<2> u = tree<0, RPW, 2>([&](int rr) {
+      const f2 kk = dup(sm.k[r0 + rr]);
+      V2<2> leaf;
+      leaf.x[0] = mul2(kk, s[rr][0]);
+      leaf.x[1] = mul2(kk, s[rr][1]);
+      return leaf;
+    });
+    put_partial(sm.red[0][0], w, lane, u.x[0], u.x[1]);
+  }
+  __syncthreads();
+  f2 delta[2];
+  {
+    f2 ulo, uhi;
+    warp_tree(sm.red[0][0], lane, ulo, uhi);
+    const float4 v4 = *reinterpret_cast<const float4*>(&sm.v[4 * lane]);
+    const f2 bt = dup(sm.beta);
+    delta[0] = mul2(bt, add2(make_float2(v4.x, v4.y), make_float2(-ulo.x, -ulo.y)));
+    delta[1] = mul2(bt, add2(make_float2(v4.z, v4.w), make_float2(-uhi.x, -uhi.y)));
+  }
+  V2<2> o = tree<0, RPW, 2>([&](int rr) {
+    const f2 kk = dup(sm.k[r0 + rr]), qq = dup(sm.q[r0 + rr]);
+    s[rr][0] = add2(s[rr][0], mul2(kk, delta[0]));
+    s[rr][1] = add2(s[rr][1], mul2(kk, delta[1]));
+    V2<2> leaf;
+    leaf.x[0] = mul2(qq, s[rr][0]);
+    leaf.x[1] = mul2(qq, s[rr][1]);
+    return leaf;
+  });
+  put_partial(sm.red[1][0], w, lane, o.x[0], o.x[1]);
+#pragma unroll
+  for (int rr = 0; rr < RPW; ++rr)
+    *reinterpret_cast<uint2*>(hr.pivots + (r0 + rr) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
+  __syncthreads();
+  if (w == 0) {
+    f2 lo, hi;
+    warp_tree(sm.red[1][0], lane, lo, hi);
+    *reinterpret_cast<float4*>(o_out + 4 * lane) = make_float4(lo.x, lo.y, hi.x, hi.y);
+  }
+  if (tid < 2 * D) hr.scales[tid] = 0.0f;
 }
 
 // ---------------------------------------------------------------------------------
@@ -335,7 +632,7 @@ decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* 
   __shared__ HeadSmem sm;
   const int item = blockIdx.x;
   const int bq = item / P.H, h = item - bq * P.H;
-  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, lane = tid & 31;
   const int slot = slots[bq];
   if (slot < 0 || slot >= P.n_slots) {
     if (tid == 0) atomicOr(P.err, ERR_SLOT_RANGE);
@@ -357,121 +654,52 @@ decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* 
   if (tid == 0) sm.beta = beta[item];
   copy16(stage, hr.codes, hr.code_bytes);
   copy16(stage + hr.piv_stage_off, hr.pivots, hr.piv_count * D * 2);
-  float cin[4];
+  f2 cin[2];
   {
     const float4 c4 = *reinterpret_cast<const float4*>(hr.scales + D + 4 * lane);
-    cin[0] = c4.x; cin[1] = c4.y; cin[2] = c4.z; cin[3] = c4.w;
+    cin[0] = make_float2(c4.x, c4.y);
+    cin[1] = make_float2(c4.z, c4.w);
   }
   __syncthreads();
-
-  // ---- restore S' = D (r c Q) and the column sums u_j = sum_i k_i S'_ij ---------------
-  float s[RPW][4];
-#pragma unroll
-  for (int rr = 0; rr < RPW; ++rr) {
-    const int i = w * RPW + rr;
-    const uint32_t info = sm.info[i];
-    const int bits = row_bits(info);
-    if (bits == PIVOT) {
-      const uint2 hv = *reinterpret_cast<const uint2*>(stage + hr.piv_stage_off + row_off(info) * (D * 2) + 8 * lane);
-      const float dec = sm.dec[i];
-      s[rr][0] = fmul(dec, __half2float(__ushort_as_half(uint16_t(hv.x & 0xFFFFu))));
-      s[rr][1] = fmul(dec, __half2float(__ushort_as_half(uint16_t(hv.x >> 16))));
-      s[rr][2] = fmul(dec, __half2float(__ushort_as_half(uint16_t(hv.y & 0xFFFFu))));
-      s[rr][3] = fmul(dec, __half2float(__ushort_as_half(uint16_t(hv.y >> 16))));
-    } else {
-      const uint32_t f = lane_field(stage + row_off(info), bits, lane);
-      const uint32_t mask = (1u << bits) - 1u;
-      const float tb = TWO23 + float(1 << (bits - 1));
-      const float rd = sm.rd[i];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const float Q = code_value((f >> (bits * cc)) & mask, tb);
-        s[rr][cc] = fmul(fmul(Q, rd), cin[cc]);
-      }
-    }
+  float* o_out = out + vec;
+  switch (hr.bits) {
+    case 2: decode_head<2>(P, h, sm, stage, hr, cin, o_out); break;
+    case 4: decode_head<4>(P, h, sm, stage, hr, cin, o_out); break;
+    case 6: decode_head<6>(P, h, sm, stage, hr, cin, o_out); break;
+    case 8: decode_head<8>(P, h, sm, stage, hr, cin, o_out); break;
+    case PIVOT: decode_pivot_head(sm, stage, hr, o_out); break;
+    default: decode_head<MIXED>(P, h, sm, stage, hr, cin, o_out); break;
   }
-  {
-    Vec<4> u = tree<0, RPW, 4>([&](int rr) {
-      const float kk = sm.k[w * RPW + rr];
-      Vec<4> leaf;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) leaf.x[cc] = fmul(kk, s[rr][cc]);
-      return leaf;
-    });
-    *reinterpret_cast<float4*>(&sm.red[0][0][w][4 * lane]) = make_float4(u.x[0], u.x[1], u.x[2], u.x[3]);
-  }
-  __syncthreads();
-
-  // ---- delta_j = beta (v_j - u_j); S = S' + k delta^T; readout partials ----------------
-  float delta[4];
-  {
-    const float bt = sm.beta;
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      const int j = 4 * lane + cc;
-      float (*r0)[D] = sm.red[0][0];
-      const float u = fadd(fadd(fadd(r0[0][j], r0[1][j]), fadd(r0[2][j], r0[3][j])),
-                           fadd(fadd(r0[4][j], r0[5][j]), fadd(r0[6][j], r0[7][j])));
-      delta[cc] = fmul(bt, __fsub_rn(sm.v[j], u));
-    }
-  }
-#pragma unroll
-  for (int rr = 0; rr < RPW; ++rr) {
-    const float kk = sm.k[w * RPW + rr];
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) s[rr][cc] = fadd(s[rr][cc], fmul(kk, delta[cc]));
-  }
-  {
-    Vec<4> o = tree<0, RPW, 4>([&](int rr) {
-      const float qq = sm.q[w * RPW + rr];
-      Vec<4> leaf;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) leaf.x[cc] = fmul(qq, s[rr][cc]);
-      return leaf;
-    });
-    *reinterpret_cast<float4*>(&sm.red[1][0][w][4 * lane]) = make_float4(o.x[0], o.x[1], o.x[2], o.x[3]);
-  }
-  // pivot rows: store float16(S) now (they take no part in the refit)
-#pragma unroll
-  for (int rr = 0; rr < RPW; ++rr) {
-    const uint32_t info = sm.info[w * RPW + rr];
-    if (row_bits(info) == PIVOT) {
-      const uint32_t lo = uint32_t(__half_as_ushort(__float2half_rn(s[rr][0]))) |
-                          (uint32_t(__half_as_ushort(__float2half_rn(s[rr][1]))) << 16);
-      const uint32_t hi = uint32_t(__half_as_ushort(__float2half_rn(s[rr][2]))) |
-                          (uint32_t(__half_as_ushort(__float2half_rn(s[rr][3]))) << 16);
-      *reinterpret_cast<uint2*>(hr.pivots + row_off(info) * D + 4 * lane) = make_uint2(lo, hi);
-    }
-  }
-
-  // ---- refit + requantise (all-pivot heads keep r = c = 0) ---------------------------
-  float c[4];
-  if (hr.piv_count == D) {
-    __syncthreads();
-    if (w == 0) {
-      float o[4];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int j = 4 * lane + cc;
-        float (*r1)[D] = sm.red[1][0];
-        o[cc] = fadd(fadd(fadd(r1[0][j], r1[1][j]), fadd(r1[2][j], r1[3][j])),
-                     fadd(fadd(r1[4][j], r1[5][j]), fadd(r1[6][j], r1[7][j])));
-      }
-      *reinterpret_cast<float4*>(out + vec + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
-    }
-    if (tid < D) hr.scales[tid] = 0.0f;
-    c[0] = c[1] = c[2] = c[3] = 0.0f;
-  } else {
-    refit_pack(P, h, sm, stage, s, hr.scales, c, out + vec);
-  }
-  __syncthreads();
-  copy16_out(hr.codes, stage, hr.code_bytes);
-  if (w == 0) *reinterpret_cast<float4*>(hr.scales + D + 4 * lane) = make_float4(c[0], c[1], c[2], c[3]);
 }
 
 // ---------------------------------------------------------------------------------
 // stq_quantize_init: float32 states -> packed pool.
 // ---------------------------------------------------------------------------------
+template <int BITS>
+__device__ __forceinline__ void quantize_head(const PoolDev& P, int h, HeadSmem& sm, uint8_t* stage,
+                                              const HeadRef& hr, const float* src) {
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int r0 = w * RPW;
+  f2 s[RPW][2];
+#pragma unroll
+  for (int rr = 0; rr < RPW; ++rr) {
+    const int i = r0 + rr;
+    const float4 x = *reinterpret_cast<const float4*>(src + i * D + 4 * lane);
+    s[rr][0] = make_float2(x.x, x.y);
+    s[rr][1] = make_float2(x.z, x.w);
+    if constexpr (BITS == MIXED) {
+      const uint32_t info = sm.info[i];
+      if (row_bits(info) == PIVOT)
+        *reinterpret_cast<uint2*>(hr.pivots + row_off(info) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
+    }
+  }
+  f2 c[2];
+  refit_pack<BITS>(P, h, sm, stage, s, hr.scales, c, nullptr);
+  __syncthreads();
+  copy16(hr.codes, stage, hr.code_bytes);
+  if (w == 0) *reinterpret_cast<float4*>(hr.scales + D + 4 * lane) = make_float4(c[0].x, c[0].y, c[1].x, c[1].y);
+}
+
 __global__ void __launch_bounds__(NT, 2)
 quantize_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* __restrict__ S) {
   extern __shared__ __align__(16) uint8_t stage[];
@@ -487,37 +715,38 @@ quantize_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float
   const HeadRef hr = head_ref(P, slot, h);
   load_row_meta(P, h, sm);
   __syncthreads();
-  float s[RPW][4];
   const float* src = S + uint64_t(item) * D * D;
+  switch (hr.bits) {
+    case 2: quantize_head<2>(P, h, sm, stage, hr, src); break;
+    case 4: quantize_head<4>(P, h, sm, stage, hr, src); break;
+    case 6: quantize_head<6>(P, h, sm, stage, hr, src); break;
+    case 8: quantize_head<8>(P, h, sm, stage, hr, src); break;
+    case PIVOT:
 #pragma unroll
-  for (int rr = 0; rr < RPW; ++rr) {
-    const int i = w * RPW + rr;
-    const float4 x = *reinterpret_cast<const float4*>(src + i * D + 4 * lane);
-    s[rr][0] = x.x; s[rr][1] = x.y; s[rr][2] = x.z; s[rr][3] = x.w;
-    const uint32_t info = sm.info[i];
-    if (row_bits(info) == PIVOT) {
-      const uint32_t lo = uint32_t(__half_as_ushort(__float2half_rn(x.x))) |
-                          (uint32_t(__half_as_ushort(__float2half_rn(x.y))) << 16);
-      const uint32_t hi = uint32_t(__half_as_ushort(__float2half_rn(x.z))) |
-                          (uint32_t(__half_as_ushort(__float2half_rn(x.w))) << 16);
-      *reinterpret_cast<uint2*>(hr.pivots + row_off(info) * D + 4 * lane) = make_uint2(lo, hi);
-    }
+      for (int rr = 0; rr < RPW; ++rr) {
+        const int i = w * RPW + rr;
+        const float4 x = *reinterpret_cast<const float4*>(src + i * D + 4 * lane);
+        *reinterpret_cast<uint2*>(hr.pivots + i * D + 4 * lane) =
+            half4_bits(make_float2(x.x, x.y), make_float2(x.z, x.w));
+      }
+      if (tid < 2 * D) hr.scales[tid] = 0.0f;
+      break;
+    default: quantize_head<MIXED>(P, h, sm, stage, hr, src); break;
   }
-  float c[4];
-  if (hr.piv_count == D) {
-    if (tid < D) hr.scales[tid] = 0.0f;
-    c[0] = c[1] = c[2] = c[3] = 0.0f;
-  } else {
-    refit_pack(P, h, sm, stage, s, hr.scales, c, nullptr);
-  }
-  __syncthreads();
-  copy16_out(hr.codes, stage, hr.code_bytes);
-  if (w == 0) *reinterpret_cast<float4*>(hr.scales + D + 4 * lane) = make_float4(c[0], c[1], c[2], c[3]);
 }
 
 // ---------------------------------------------------------------------------------
 // stq_dequantize: packed pool -> float32 states, S_ij = (Q_ij r_i) c_j.
 // ---------------------------------------------------------------------------------
+template <int BITS>
+__device__ __forceinline__ void dequant_row(const uint8_t* row, int lane, float r, const f2 (&cin)[2],
+                                            float* dst) {
+  constexpr float TB = TWO23 + float(1 << (BITS - 1));
+  f2 a, b;
+  restore_row<BITS>(row, lane, r, TB, cin, a, b);
+  *reinterpret_cast<float4*>(dst) = make_float4(a.x, a.y, b.x, b.y);
+}
+
 __global__ void __launch_bounds__(NT)
 dequant_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, float* __restrict__ S_out) {
   extern __shared__ __align__(16) uint8_t stage[];
@@ -539,30 +768,27 @@ dequant_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, float* __res
   copy16(stage, hr.codes, hr.code_bytes);
   copy16(stage + hr.piv_stage_off, hr.pivots, hr.piv_count * D * 2);
   const float4 c4 = *reinterpret_cast<const float4*>(hr.scales + D + 4 * lane);
-  const float cin[4] = {c4.x, c4.y, c4.z, c4.w};
+  const f2 cin[2] = {make_float2(c4.x, c4.y), make_float2(c4.z, c4.w)};
   __syncthreads();
   float* dst = S_out + uint64_t(item) * D * D;
 #pragma unroll 4
   for (int rr = 0; rr < RPW; ++rr) {
     const int i = w * RPW + rr;
     const uint32_t info = info_s[i];
-    const int bits = row_bits(info);
-    float x[4];
-    if (bits == PIVOT) {
-      const uint2 hv = *reinterpret_cast<const uint2*>(stage + hr.piv_stage_off + row_off(info) * (D * 2) + 8 * lane);
-      x[0] = __half2float(__ushort_as_half(uint16_t(hv.x & 0xFFFFu)));
-      x[1] = __half2float(__ushort_as_half(uint16_t(hv.x >> 16)));
-      x[2] = __half2float(__ushort_as_half(uint16_t(hv.y & 0xFFFFu)));
-      x[3] = __half2float(__ushort_as_half(uint16_t(hv.y >> 16)));
-    } else {
-      const uint32_t f = lane_field(stage + row_off(info), bits, lane);
-      const uint32_t mask = (1u << bits) - 1u;
-      const float tb = TWO23 + float(1 << (bits - 1));
-      const float r = r_s[i];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) x[cc] = fmul(fmul(code_value((f >> (bits * cc)) & mask, tb), r), cin[cc]);
+    const uint8_t* row = stage + row_off(info);
+    float* o = dst + i * D + 4 * lane;
+    switch (row_bits(info)) {
+      case 2: dequant_row<2>(row, lane, r_s[i], cin, o); break;
+      case 4: dequant_row<4>(row, lane, r_s[i], cin, o); break;
+      case 6: dequant_row<6>(row, lane, r_s[i], cin, o); break;
+      case 8: dequant_row<8>(row, lane, r_s[i], cin, o); break;
+      default: {
+        const uint2 hv = *reinterpret_cast<const uint2*>(stage + hr.piv_stage_off + row_off(info) * (D * 2) + 8 * lane);
+        f2 a, b;
+        half4_floats(hv, a, b);
+        *reinterpret_cast<float4*>(o) = make_float4(a.x, a.y, b.x, b.y);
+      }
     }
-    *reinterpret_cast<float4*>(dst + i * D + 4 * lane) = make_float4(x[0], x[1], x[2], x[3]);
   }
 }
 
@@ -574,10 +800,11 @@ fp32_step_kernel(int kind, float* __restrict__ S, const float* __restrict__ q,
                  const float* __restrict__ k, const float* __restrict__ v,
                  const float* __restrict__ gate, const float* __restrict__ beta,
                  float* __restrict__ out) {
-  __shared__ float ks[D], qs[D], vs[D], ds[D];
-  __shared__ __align__(16) float red[2][NW][D];
+  __shared__ __align__(16) float ks[D], qs[D], vs[D], ds[D];
+  __shared__ float4 red[2][NW][D / 4];
   const int item = blockIdx.x;
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int r0 = w * RPW;
   const uint64_t vec = uint64_t(item) * D;
   if (tid < D) {
     ks[tid] = k[vec + tid];
@@ -588,57 +815,49 @@ fp32_step_kernel(int kind, float* __restrict__ S, const float* __restrict__ q,
   const float bt = beta[item];
   __syncthreads();
   float* base = S + vec * D;
-  float s[RPW][4];
+  f2 s[RPW][2];
 #pragma unroll
   for (int rr = 0; rr < RPW; ++rr) {
-    const int i = w * RPW + rr;
+    const int i = r0 + rr;
     const float4 x = *reinterpret_cast<const float4*>(base + i * D + 4 * lane);
-    const float dd = ds[i];
-    s[rr][0] = fmul(dd, x.x); s[rr][1] = fmul(dd, x.y); s[rr][2] = fmul(dd, x.z); s[rr][3] = fmul(dd, x.w);
+    const f2 dd = dup(ds[i]);
+    s[rr][0] = mul2(dd, make_float2(x.x, x.y));
+    s[rr][1] = mul2(dd, make_float2(x.z, x.w));
   }
-  Vec<4> u = tree<0, RPW, 4>([&](int rr) {
-    const float kk = ks[w * RPW + rr];
-    Vec<4> leaf;
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) leaf.x[cc] = fmul(kk, s[rr][cc]);
+  V2<2> u = tree<0, RPW, 2>([&](int rr) {
+    const f2 kk = dup(ks[r0 + rr]);
+    V2<2> leaf;
+    leaf.x[0] = mul2(kk, s[rr][0]);
+    leaf.x[1] = mul2(kk, s[rr][1]);
     return leaf;
   });
-  *reinterpret_cast<float4*>(&red[0][w][4 * lane]) = make_float4(u.x[0], u.x[1], u.x[2], u.x[3]);
+  put_partial(red[0], w, lane, u.x[0], u.x[1]);
   __syncthreads();
-  float delta[4];
-#pragma unroll
-  for (int cc = 0; cc < 4; ++cc) {
-    const int j = 4 * lane + cc;
-    const float uu = fadd(fadd(fadd(red[0][0][j], red[0][1][j]), fadd(red[0][2][j], red[0][3][j])),
-                          fadd(fadd(red[0][4][j], red[0][5][j]), fadd(red[0][6][j], red[0][7][j])));
-    delta[cc] = fmul(bt, __fsub_rn(vs[j], uu));
+  f2 delta[2];
+  {
+    f2 ulo, uhi;
+    warp_tree(red[0], lane, ulo, uhi);
+    const float4 v4 = *reinterpret_cast<const float4*>(&vs[4 * lane]);
+    delta[0] = mul2(dup(bt), add2(make_float2(v4.x, v4.y), make_float2(-ulo.x, -ulo.y)));
+    delta[1] = mul2(dup(bt), add2(make_float2(v4.z, v4.w), make_float2(-uhi.x, -uhi.y)));
   }
-#pragma unroll
-  for (int rr = 0; rr < RPW; ++rr) {
-    const int i = w * RPW + rr;
-    const float kk = ks[i];
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) s[rr][cc] = fadd(s[rr][cc], fmul(kk, delta[cc]));
-    *reinterpret_cast<float4*>(base + i * D + 4 * lane) = make_float4(s[rr][0], s[rr][1], s[rr][2], s[rr][3]);
-  }
-  Vec<4> o = tree<0, RPW, 4>([&](int rr) {
-    const float qq = qs[w * RPW + rr];
-    Vec<4> leaf;
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) leaf.x[cc] = fmul(qq, s[rr][cc]);
+  V2<2> o = tree<0, RPW, 2>([&](int rr) {
+    const int i = r0 + rr;
+    const f2 kk = dup(ks[i]), qq = dup(qs[i]);
+    s[rr][0] = add2(s[rr][0], mul2(kk, delta[0]));
+    s[rr][1] = add2(s[rr][1], mul2(kk, delta[1]));
+    *reinterpret_cast<float4*>(base + i * D + 4 * lane) = make_float4(s[rr][0].x, s[rr][0].y, s[rr][1].x, s[rr][1].y);
+    V2<2> leaf;
+    leaf.x[0] = mul2(qq, s[rr][0]);
+    leaf.x[1] = mul2(qq, s[rr][1]);
     return leaf;
   });
-  *reinterpret_cast<float4*>(&red[1][w][4 * lane]) = make_float4(o.x[0], o.x[1], o.x[2], o.x[3]);
+  put_partial(red[1], w, lane, o.x[0], o.x[1]);
   __syncthreads();
   if (w == 0) {
-    float oo[4];
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      const int j = 4 * lane + cc;
-      oo[cc] = fadd(fadd(fadd(red[1][0][j], red[1][1][j]), fadd(red[1][2][j], red[1][3][j])),
-                    fadd(fadd(red[1][4][j], red[1][5][j]), fadd(red[1][6][j], red[1][7][j])));
-    }
-    *reinterpret_cast<float4*>(out + vec + 4 * lane) = make_float4(oo[0], oo[1], oo[2], oo[3]);
+    f2 lo, hi;
+    warp_tree(red[1], lane, lo, hi);
+    *reinterpret_cast<float4*>(out + vec + 4 * lane) = make_float4(lo.x, lo.y, hi.x, hi.y);
   }
 }
 
