@@ -18,9 +18,11 @@ Readings taken where the pages are silent (each also listed in the design doc):
     S'_ij = (Q_ij * (d_i * r_i)) * c_j. D_t is diagonal over key rows, so this is the
     same matrix as D_t * (r c Q).
   * Every sum over the 128 entries of a row or a column is a balanced binary tree:
-    adjacent pairs first, then adjacent pairs of those, and so on (`tree_sum`).
-  * Products are rounded before they are added (no fused multiply-add), except the
-    quantiser's x = y * (1/c), which is taken exactly before rounding to an integer.
+    adjacent pairs first, then adjacent pairs of those, and so on (`tree_sum`). A sum
+    of products a_i b_i forms each adjacent pair with one fused multiply-add,
+    fma(a_2m, b_2m, a_2m+1 * b_2m+1) (`tree_dot`); the state update is the fused
+    S_ij = fma(k_i, delta_j, S'_ij). Every other product is rounded on its own. The
+    quantiser's x = y * (1/c) is taken exactly before rounding to an integer.
   * Row scale r_i = mean_j |S_ij| * (omega_i / mean omega)^(-1/2); the column scale
     starts at c_j = max_i |S_ij| / (r_i qmax_i) and takes exactly two omega-weighted
     least-squares steps; the stored codes are requantised with the final c.
@@ -71,6 +73,38 @@ def tree_sum(x, axis):
     while x.shape[-1] > 1:
         x = x[..., 0::2] + x[..., 1::2]
     return x[..., 0]
+
+
+def fma32(a, b, c):
+    """float32 fused multiply-add a*b + c with one rounding (nearest-even).
+
+    a*b is exact in float64; a + b in float64 is made "round to odd" (if the float64
+    sum is inexact and its last bit is even, step one float64 ulp towards the exact
+    value, found with the error-free two-sum), so that the final rounding to float32
+    equals the rounding of the exact value (round-to-odd with 53 >= 24 + 2 bits;
+    Boldo and Melquiond, "Emulation of FMA and correctly rounded sums: proved
+    algorithms using rounding to odd", IEEE TC 2008)."""
+    a = np.asarray(a, dtype=F32).astype(F64)
+    b = np.asarray(b, dtype=F32).astype(F64)
+    c = np.asarray(c, dtype=F32).astype(F64)
+    p = a * b
+    s = p + c
+    bp = s - p
+    err = (p - (s - bp)) + (c - bp)
+    even = (np.asarray(s).view(np.int64) & 1) == 0
+    fix = (err != 0) & even
+    s = np.where(fix, np.nextafter(s, np.where(err > 0, np.inf, -np.inf)), s)
+    return s.astype(F32)
+
+
+def tree_dot(a, b, axis):
+    """sum_i a_i b_i along `axis` (power-of-two length): adjacent products paired by
+    one fused multiply-add, fma(a_2m, b_2m, a_2m+1 * b_2m+1), then `tree_sum`."""
+    a = np.moveaxis(np.asarray(a, dtype=F32), axis, -1)
+    b = np.moveaxis(np.asarray(b, dtype=F32), axis, -1)
+    a, b = np.broadcast_arrays(a, b)
+    pairs = fma32(a[..., 0::2], b[..., 0::2], a[..., 1::2] * b[..., 1::2])
+    return tree_sum(pairs, axis=-1)
 
 
 def row_gain(omega):
@@ -229,9 +263,9 @@ def delta_update(Sp, k, v, beta):
     beta [...]."""
     Sp = np.asarray(Sp, dtype=F32)
     k = np.asarray(k, dtype=F32)
-    u = tree_sum(k[..., :, None] * Sp, axis=-2)
+    u = tree_dot(k[..., :, None], Sp, axis=-2)
     delta = np.asarray(beta, dtype=F32)[..., None] * (np.asarray(v, dtype=F32) - u)
-    return Sp + k[..., :, None] * delta[..., None, :]
+    return fma32(k[..., :, None], delta[..., None, :], Sp)
 
 
 def readout(S, q):
@@ -287,8 +321,8 @@ def refit(S, omega, row_bits, n_ls=2):
     for _ in range(n_ls):
         Q = _quantise(y, _recip(c), qm)
         p = b[..., :, None] * Q
-        num = tree_sum(p * y, axis=-2)
-        den = tree_sum(p * Q, axis=-2)
+        num = tree_dot(p, y, axis=-2)
+        den = tree_dot(p, Q, axis=-2)
         safe = np.where(den > 0, den, F32(1))
         c = np.where(den > 0, num / safe, c).astype(F32)
     Q = _quantise(y, _recip(c), qm)

@@ -184,11 +184,38 @@ def test_dequantize_hand_example():
 # to catch axis and broadcasting slips in the vectorised oracle
 # ---------------------------------------------------------------------------------
 
+def rn32(x: Fraction) -> np.float32:
+    """Exact rational -> nearest float32, ties to even (normal and subnormal range)."""
+    if x == 0:
+        return np.float32(0.0)
+    sign = -1 if x < 0 else 1
+    x = abs(x)
+    e = x.numerator.bit_length() - x.denominator.bit_length()
+    if Fraction(2) ** e > x:
+        e -= 1
+    e = max(e, -126)                       # subnormals share the 2^-149 step
+    scaled = x / Fraction(2) ** (e - 23)   # in [2^23, 2^24) for normal numbers
+    m = scaled.numerator // scaled.denominator
+    rem = scaled - m
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and m % 2 == 1):
+        m += 1
+    return np.float32(sign * float(Fraction(m) * Fraction(2) ** (e - 23)))
+
+
+def fma_exact(a, b, c):
+    return rn32(Fraction(float(a)) * Fraction(float(b)) + Fraction(float(c)))
+
+
 def _tsum(xs):
     xs = list(xs)
     while len(xs) > 1:
         xs = [xs[2 * i] + xs[2 * i + 1] for i in range(len(xs) // 2)]
     return xs[0]
+
+
+def _tdot(a, b):
+    a, b = list(a), list(b)
+    return _tsum([fma_exact(a[2 * m], b[2 * m], a[2 * m + 1] * b[2 * m + 1]) for m in range(len(a) // 2)])
 
 
 def _scalar_refit(S, omega, bits):
@@ -231,8 +258,8 @@ def _scalar_refit(S, omega, bits):
         Q = quant(c)
         for j in range(d):
             p = [b[i] * Q[i][j] for i in range(d)]
-            num = _tsum([p[i] * y[i][j] for i in range(d)])
-            den = _tsum([p[i] * Q[i][j] for i in range(d)])
+            num = _tdot(p, [y[i][j] for i in range(d)])
+            den = _tdot(p, [Q[i][j] for i in range(d)])
             if den > 0:
                 c[j] = num / den
     return r, c, quant(c)
@@ -253,3 +280,32 @@ def test_vectorised_refit_equals_scalar_twin(seed):
     for i in range(d):
         if bits[i] != 16:
             assert [int(x) for x in u[i] - bias[i]] == [int(x) for x in Qs[i]]
+
+
+def test_fma32_is_correctly_rounded():
+    # against exact rational arithmetic, on random operands and on products that land
+    # on or next to float32 rounding midpoints
+    rng = np.random.default_rng(13)
+    a = rng.standard_normal(3000).astype(F32)
+    b = (rng.standard_normal(3000) * np.exp2(rng.integers(-30, 30, 3000))).astype(F32)
+    c = rng.standard_normal(3000).astype(F32)
+    # c = -RN(a*b) + tiny makes the result depend on the low product bits
+    c[:1000] = (-(a[:1000] * b[:1000])).astype(F32)
+    c[1000:1500] = (a[1000:1500] * b[1000:1500] * F32(3)).astype(F32)
+    # midpoint cases: a*b exactly halfway between floats of c's binade
+    c[1500:1600] = F32(1.0)
+    a[1500:1600] = F32(2.0 ** -24)
+    b[1500:1600] = np.where(rng.random(100) < 0.5, 1.0, -1.0).astype(F32) * F32(1 + 2.0 ** -23)
+    got = O.fma32(a, b, c)
+    for i in range(3000):
+        assert got[i] == fma_exact(a[i], b[i], c[i]), i
+
+
+def test_tree_dot_pairs_products_by_fma():
+    rng = np.random.default_rng(14)
+    a = rng.standard_normal((5, 16)).astype(F32)
+    b = rng.standard_normal((5, 16)).astype(F32)
+    got = O.tree_dot(a, b, axis=1)
+    for r in range(5):
+        assert got[r] == _tdot(a[r], b[r])
+    assert np.allclose(got, (a.astype(np.float64) * b).sum(1), atol=1e-5)
