@@ -13,13 +13,13 @@
 // share one width run a code path specialised for it.
 //
 // Float32 evaluation order (the CPU oracle restates the same order):
-//   * every product is rounded before it is added (explicit _rn intrinsics, including
-//     the packed float2 forms __fmul2_rn/__fadd2_rn; the file is also built with
-//     --fmad=false);
 //   * sums over the 128 rows of a column or the 128 columns of a row are balanced
 //     binary trees, adjacent pairs first. Column sums: a thread's 16 rows form the
 //     lower 4 levels, the 8 warps (shared memory) the top 3. Row sums: a thread's 4
 //     columns form the lower 2 levels, butterfly shuffle steps xor 1,2,...,16 the top 5;
+//   * in a sum of products a_i b_i each adjacent pair is one fused multiply-add,
+//     fma(a_2m, b_2m, a_2m+1 * b_2m+1); the state update is S = fma(k, delta, S'); every
+//     other product is rounded on its own (explicit _rn forms, --fmad=false);
 //   * the quantiser's x = y * inv_c is taken exactly: fma(y, inv_c, 1.5*2^23) rounds the
 //     exact product to the nearest integer (ties to even) inside the 2^23 binade, and
 //     clamping is done in that binade, where the low bits are the (biased) code.
@@ -43,6 +43,9 @@ using f2 = float2;
 
 __device__ __forceinline__ float fmul(float a, float b) { return __fmul_rn(a, b); }
 __device__ __forceinline__ float fadd(float a, float b) { return __fadd_rn(a, b); }
+// Packed float2 arithmetic (one rounding per component, like the scalar _rn forms). The
+// code generator fuses a multiply that feeds an add, so every sum of products below is
+// written with explicit fused pairs and leaves no multiply-add pair to fuse.
 __device__ __forceinline__ f2 mul2(f2 a, f2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ f2 add2(f2 a, f2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) { return __ffma2_rn(a, b, c); }
@@ -365,32 +368,41 @@ __device__ __forceinline__ void refit_pack(const PoolDev& P, int h, HeadSmem& sm
     const f2 ic[2] = {make_float2(recip_scale(c[0].x), recip_scale(c[0].y)),
                       make_float2(recip_scale(c[1].x), recip_scale(c[1].y))};
     float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f), q4 = b4;
-    V2<4> nd = tree<0, RPW, 4>([&](int rr) {
-      if ((rr & 3) == 0) {
-        b4 = *reinterpret_cast<const float4*>(&sm.b[r0 + rr]);
-        if constexpr (BITS == MIXED) q4 = *reinterpret_cast<const float4*>(&sm.qm[r0 + rr]);
+    V2<4> nd = tree<0, RPW / 2, 4>([&](int m) {
+      // rows 2m and 2m+1 form one fused pair of each sum
+      if ((m & 1) == 0) {
+        b4 = *reinterpret_cast<const float4*>(&sm.b[r0 + 2 * m]);
+        if constexpr (BITS == MIXED) q4 = *reinterpret_cast<const float4*>(&sm.qm[r0 + 2 * m]);
       }
-      const f2 bb = dup(at4(b4, rr & 3));
-      float lo_b, hi_b;
-      if constexpr (BITS == MIXED) {
-        lo_b = MAGIC - at4(q4, rr & 3);
-        hi_b = MAGIC + at4(q4, rr & 3);
-      } else {
-        lo_b = MAGIC - float((1 << (BITS - 1)) - 1);
-        hi_b = MAGIC + float((1 << (BITS - 1)) - 1);
+      f2 Q[2][2], p[2][2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int rr = 2 * m + e;
+        const f2 bb = dup(at4(b4, rr & 3));
+        float lo_b, hi_b;
+        if constexpr (BITS == MIXED) {
+          lo_b = MAGIC - at4(q4, rr & 3);
+          hi_b = MAGIC + at4(q4, rr & 3);
+        } else {
+          lo_b = MAGIC - float((1 << (BITS - 1)) - 1);
+          hi_b = MAGIC + float((1 << (BITS - 1)) - 1);
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          f2 t = fma2(s[rr][hh], ic[hh], dup(MAGIC));
+          if (it > 0) {  // step one never clips: c0 is the column maximum
+            t.x = fminf(fmaxf(t.x, lo_b), hi_b);
+            t.y = fminf(fmaxf(t.y, lo_b), hi_b);
+          }
+          Q[e][hh] = add2(t, dup(-MAGIC));
+          p[e][hh] = mul2(bb, Q[e][hh]);
+        }
       }
       V2<4> leaf;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
-        f2 t = fma2(s[rr][hh], ic[hh], dup(MAGIC));
-        if (it > 0) {  // step one never clips: c0 is the column maximum
-          t.x = fminf(fmaxf(t.x, lo_b), hi_b);
-          t.y = fminf(fmaxf(t.y, lo_b), hi_b);
-        }
-        const f2 Q = add2(t, dup(-MAGIC));
-        const f2 p = mul2(bb, Q);
-        leaf.x[hh] = mul2(p, s[rr][hh]);
-        leaf.x[2 + hh] = mul2(p, Q);
+        leaf.x[hh] = fma2(p[0][hh], s[2 * m][hh], mul2(p[1][hh], s[2 * m + 1][hh]));
+        leaf.x[2 + hh] = fma2(p[0][hh], Q[0][hh], mul2(p[1][hh], Q[1][hh]));
       }
       return leaf;
     });
@@ -507,12 +519,12 @@ __device__ __forceinline__ void decode_head(const PoolDev& P, int h, HeadSmem& s
   }
   {
     float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    V2<2> u = tree<0, RPW, 2>([&](int rr) {
-      if ((rr & 3) == 0) k4 = *reinterpret_cast<const float4*>(&sm.k[r0 + rr]);
-      const f2 kk = dup(at4(k4, rr & 3));
+    V2<2> u = tree<0, RPW / 2, 2>([&](int m) {
+      if ((m & 1) == 0) k4 = *reinterpret_cast<const float4*>(&sm.k[r0 + 2 * m]);
+      const f2 ke = dup(at4(k4, (2 * m) & 3)), ko = dup(at4(k4, (2 * m + 1) & 3));
       V2<2> leaf;
-      leaf.x[0] = mul2(kk, s[rr][0]);
-      leaf.x[1] = mul2(kk, s[rr][1]);
+      leaf.x[0] = fma2(ke, s[2 * m][0], mul2(ko, s[2 * m + 1][0]));
+      leaf.x[1] = fma2(ke, s[2 * m][1], mul2(ko, s[2 * m + 1][1]));
       return leaf;
     });
     put_partial(sm.red[0][0], w, lane, u.x[0], u.x[1]);
@@ -531,17 +543,21 @@ __device__ __forceinline__ void decode_head(const PoolDev& P, int h, HeadSmem& s
   }
   {
     float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f), q4 = k4;
-    V2<2> o = tree<0, RPW, 2>([&](int rr) {
-      if ((rr & 3) == 0) {
-        k4 = *reinterpret_cast<const float4*>(&sm.k[r0 + rr]);
-        q4 = *reinterpret_cast<const float4*>(&sm.q[r0 + rr]);
+    V2<2> o = tree<0, RPW / 2, 2>([&](int m) {
+      if ((m & 1) == 0) {
+        k4 = *reinterpret_cast<const float4*>(&sm.k[r0 + 2 * m]);
+        q4 = *reinterpret_cast<const float4*>(&sm.q[r0 + 2 * m]);
       }
-      const f2 kk = dup(at4(k4, rr & 3)), qq = dup(at4(q4, rr & 3));
-      s[rr][0] = add2(s[rr][0], mul2(kk, delta[0]));
-      s[rr][1] = add2(s[rr][1], mul2(kk, delta[1]));
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const f2 kk = dup(at4(k4, (2 * m + e) & 3));
+        s[2 * m + e][0] = fma2(kk, delta[0], s[2 * m + e][0]);
+        s[2 * m + e][1] = fma2(kk, delta[1], s[2 * m + e][1]);
+      }
+      const f2 qe = dup(at4(q4, (2 * m) & 3)), qo = dup(at4(q4, (2 * m + 1) & 3));
       V2<2> leaf;
-      leaf.x[0] = mul2(qq, s[rr][0]);
-      leaf.x[1] = mul2(qq, s[rr][1]);
+      leaf.x[0] = fma2(qe, s[2 * m][0], mul2(qo, s[2 * m + 1][0]));
+      leaf.x[1] = fma2(qe, s[2 * m][1], mul2(qo, s[2 * m + 1][1]));
       return leaf;
     });
     put_partial(sm.red[1][0], w, lane, o.x[0], o.x[1]);
@@ -579,11 +595,11 @@ __device__ __forceinline__ void decode_pivot_head(HeadSmem& sm, uint8_t* stage, 
     s[rr][1] = mul2(dd, b);
   }
   {
-    V2<2> u = tree<0, RPW, 2>([&](int rr) {
-      const f2 kk = dup(sm.k[r0 + rr]);
+    V2<2> u = tree<0, RPW / 2, 2>([&](int m) {
+      const f2 ke = dup(sm.k[r0 + 2 * m]), ko = dup(sm.k[r0 + 2 * m + 1]);
       V2<2> leaf;
-      leaf.x[0] = mul2(kk, s[rr][0]);
-      leaf.x[1] = mul2(kk, s[rr][1]);
+      leaf.x[0] = fma2(ke, s[2 * m][0], mul2(ko, s[2 * m + 1][0]));
+      leaf.x[1] = fma2(ke, s[2 * m][1], mul2(ko, s[2 * m + 1][1]));
       return leaf;
     });
     put_partial(sm.red[0][0], w, lane, u.x[0], u.x[1]);
@@ -598,13 +614,17 @@ __device__ __forceinline__ void decode_pivot_head(HeadSmem& sm, uint8_t* stage, 
     delta[0] = mul2(bt, add2(make_float2(v4.x, v4.y), make_float2(-ulo.x, -ulo.y)));
     delta[1] = mul2(bt, add2(make_float2(v4.z, v4.w), make_float2(-uhi.x, -uhi.y)));
   }
-  V2<2> o = tree<0, RPW, 2>([&](int rr) {
-    const f2 kk = dup(sm.k[r0 + rr]), qq = dup(sm.q[r0 + rr]);
-    s[rr][0] = add2(s[rr][0], mul2(kk, delta[0]));
-    s[rr][1] = add2(s[rr][1], mul2(kk, delta[1]));
+  V2<2> o = tree<0, RPW / 2, 2>([&](int m) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const f2 kk = dup(sm.k[r0 + 2 * m + e]);
+      s[2 * m + e][0] = fma2(kk, delta[0], s[2 * m + e][0]);
+      s[2 * m + e][1] = fma2(kk, delta[1], s[2 * m + e][1]);
+    }
+    const f2 qe = dup(sm.q[r0 + 2 * m]), qo = dup(sm.q[r0 + 2 * m + 1]);
     V2<2> leaf;
-    leaf.x[0] = mul2(qq, s[rr][0]);
-    leaf.x[1] = mul2(qq, s[rr][1]);
+    leaf.x[0] = fma2(qe, s[2 * m][0], mul2(qo, s[2 * m + 1][0]));
+    leaf.x[1] = fma2(qe, s[2 * m][1], mul2(qo, s[2 * m + 1][1]));
     return leaf;
   });
   put_partial(sm.red[1][0], w, lane, o.x[0], o.x[1]);
@@ -824,11 +844,11 @@ fp32_step_kernel(int kind, float* __restrict__ S, const float* __restrict__ q,
     s[rr][0] = mul2(dd, make_float2(x.x, x.y));
     s[rr][1] = mul2(dd, make_float2(x.z, x.w));
   }
-  V2<2> u = tree<0, RPW, 2>([&](int rr) {
-    const f2 kk = dup(ks[r0 + rr]);
+  V2<2> u = tree<0, RPW / 2, 2>([&](int m) {
+    const f2 ke = dup(ks[r0 + 2 * m]), ko = dup(ks[r0 + 2 * m + 1]);
     V2<2> leaf;
-    leaf.x[0] = mul2(kk, s[rr][0]);
-    leaf.x[1] = mul2(kk, s[rr][1]);
+    leaf.x[0] = fma2(ke, s[2 * m][0], mul2(ko, s[2 * m + 1][0]));
+    leaf.x[1] = fma2(ke, s[2 * m][1], mul2(ko, s[2 * m + 1][1]));
     return leaf;
   });
   put_partial(red[0], w, lane, u.x[0], u.x[1]);
@@ -841,15 +861,19 @@ fp32_step_kernel(int kind, float* __restrict__ S, const float* __restrict__ q,
     delta[0] = mul2(dup(bt), add2(make_float2(v4.x, v4.y), make_float2(-ulo.x, -ulo.y)));
     delta[1] = mul2(dup(bt), add2(make_float2(v4.z, v4.w), make_float2(-uhi.x, -uhi.y)));
   }
-  V2<2> o = tree<0, RPW, 2>([&](int rr) {
-    const int i = r0 + rr;
-    const f2 kk = dup(ks[i]), qq = dup(qs[i]);
-    s[rr][0] = add2(s[rr][0], mul2(kk, delta[0]));
-    s[rr][1] = add2(s[rr][1], mul2(kk, delta[1]));
-    *reinterpret_cast<float4*>(base + i * D + 4 * lane) = make_float4(s[rr][0].x, s[rr][0].y, s[rr][1].x, s[rr][1].y);
+  V2<2> o = tree<0, RPW / 2, 2>([&](int m) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int rr = 2 * m + e, i = r0 + rr;
+      const f2 kk = dup(ks[i]);
+      s[rr][0] = fma2(kk, delta[0], s[rr][0]);
+      s[rr][1] = fma2(kk, delta[1], s[rr][1]);
+      *reinterpret_cast<float4*>(base + i * D + 4 * lane) = make_float4(s[rr][0].x, s[rr][0].y, s[rr][1].x, s[rr][1].y);
+    }
+    const f2 qe = dup(qs[r0 + 2 * m]), qo = dup(qs[r0 + 2 * m + 1]);
     V2<2> leaf;
-    leaf.x[0] = mul2(qq, s[rr][0]);
-    leaf.x[1] = mul2(qq, s[rr][1]);
+    leaf.x[0] = fma2(qe, s[2 * m][0], mul2(qo, s[2 * m + 1][0]));
+    leaf.x[1] = fma2(qe, s[2 * m][1], mul2(qo, s[2 * m + 1][1]));
     return leaf;
   });
   put_partial(red[1], w, lane, o.x[0], o.x[1]);
