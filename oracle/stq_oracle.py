@@ -88,13 +88,16 @@ def fma32(a, b, c):
     b = np.asarray(b, dtype=F32).astype(F64)
     c = np.asarray(c, dtype=F32).astype(F64)
     p = a * b
-    s = p + c
+    s = np.asarray(p + c)
     bp = s - p
     err = (p - (s - bp)) + (c - bp)
-    even = (np.asarray(s).view(np.int64) & 1) == 0
-    fix = (err != 0) & even
-    s = np.where(fix, np.nextafter(s, np.where(err > 0, np.inf, -np.inf)), s)
-    return s.astype(F32)
+    bits = s.view(np.int64)
+    fix = (err != 0) & ((bits & 1) == 0)
+    # one float64 ulp towards the exact value: +1 on the bit pattern when s and err
+    # have the same sign (away from zero), -1 otherwise (s == 0 implies err == 0)
+    step = np.where((s > 0) == (err > 0), 1, -1)
+    bits = bits + np.where(fix, step, 0)
+    return bits.view(F64).astype(F32)
 
 
 def tree_dot(a, b, axis):
