@@ -134,6 +134,35 @@ stq_status stq_decode_step_host(stq_pool* pool, const int32_t* d_slots, int B,
                                 const float* h_gate, const float* h_beta, float* h_out,
                                 void* d_staging, size_t staging_bytes, void* stream);
 
+/* Bytes of the library's own device staging array used by
+ * stq_decode_step_host_static (8 MiB). */
+#define STQ_STATIC_STAGING_BYTES (8u << 20)
+
+/* stq_decode_step_host without a caller-provided staging buffer. The paper has no
+ * counterpart: this is a service of this library for callers that cannot allocate
+ * device memory on their decode path -- a host application that was handed the state
+ * pool once and only has host buffers per step, or a serving loop that must not take
+ * the device-wide synchronisation a cudaMalloc implies. The per-step device staging
+ * (q, k, v, gate, beta and the readout) lives in a fixed array of
+ * STQ_STATIC_STAGING_BYTES that the library declares in device memory; every GPU that
+ * loads the library holds it until the process exits. Arguments are those of
+ * stq_decode_step_host minus d_staging/staging_bytes.
+ *   - Returns STQ_ERR_INVALID_ARG (with a message) when the step's staging for B
+ *     requests exceeds STQ_STATIC_STAGING_BYTES (about 3,200 KDA or 4,000 GDN
+ *     head-states per call); use stq_decode_step_host with your own buffer then.
+ *   - Calls no cudaMalloc/cudaFree and no allocating routine.
+ *   - The first call on each device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture on the device.
+ *   - All calls share the one array, which keeps the last call's contents (nothing in
+ *     it needs to start at zero: each call writes every byte it reads). Calls whose
+ *     work overlaps on the GPU (other streams, other host threads) race on it: order
+ *     them on one stream or synchronise between them. */
+stq_status stq_decode_step_host_static(stq_pool* pool, const int32_t* d_slots, int B,
+                                       const float* h_q, const float* h_k, const float* h_v,
+                                       const float* h_gate, const float* h_beta, float* h_out,
+                                       void* stream);
+
 /* Dequantise slots d_slots[0..B) into d_S_out [B, H, 128, 128] float32:
  * S_ij = (Q_ij * r_i) * c_j, pivot rows float32(h_ij). */
 stq_status stq_dequantize(stq_pool* pool, const int32_t* d_slots, int B, float* d_S_out,

@@ -149,6 +149,15 @@ struct stq_pool {
   void* meta = nullptr;
 };
 
+namespace stq {
+
+const PoolDev* pool_dev(const ::stq_pool* pool) { return pool ? &pool->dev : nullptr; }
+int pool_kind(const ::stq_pool* pool) { return pool ? pool->L.kind : -1; }
+void set_last_error(const char* msg) { g_last_error = msg; }
+void clear_last_error() { g_last_error.clear(); }
+
+}  // namespace stq
+
 extern "C" {
 
 const char* stq_last_error(void) { return g_last_error.c_str(); }

@@ -7,6 +7,8 @@
 
 #include <cuda_runtime.h>
 
+struct stq_pool;
+
 namespace stq {
 
 constexpr int D = 128;           // d_k = d_v
@@ -60,5 +62,11 @@ cudaError_t launch_dequantize(const PoolDev& P, const int32_t* slots, int B, flo
 cudaError_t launch_fp32_step(int kind, int B, int H, float* S, const float* q,
                              const float* k, const float* v, const float* gate,
                              const float* beta, float* out, cudaStream_t s);
+
+// Accessors for entry points that live outside stq_abi.cpp.
+const PoolDev* pool_dev(const struct ::stq_pool* pool);
+int pool_kind(const struct ::stq_pool* pool);
+void set_last_error(const char* msg);
+void clear_last_error();
 
 }  // namespace stq

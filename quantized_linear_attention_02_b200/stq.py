@@ -62,6 +62,7 @@ def lib():
         "stq_decode_step_host_staging_bytes": (ctypes.c_size_t, [_vp, _i]),
         "stq_decode_step_host": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                       ctypes.c_size_t, _vp]),
+        "stq_decode_step_host_static": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
         "stq_dequantize": (_i, [_vp, _vp, _i, _vp, _vp]),
         "stq_fp32_decode_step": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
         "stq_pool_check": (_i, [_vp, _vp]),
@@ -206,6 +207,20 @@ class Pool:
             ctypes.c_void_p(h_gate.data_ptr()), ctypes.c_void_p(h_beta.data_ptr()),
             ctypes.c_void_p(h_out.data_ptr()), _ptr(staging, torch.uint8, "staging"),
             ctypes.c_size_t(staging.numel()), _stream(stream)))
+
+    def decode_step_host_static(self, slots, h_q, h_k, h_v, h_gate, h_beta, h_out, stream=None):
+        """Decode step with host (pinned) tensors and the library's own static device
+        staging (no device buffer from the caller; see include/stq.h)."""
+        import torch
+        B = slots.numel()
+        for name, t in (("q", h_q), ("k", h_k), ("v", h_v), ("gate", h_gate), ("beta", h_beta), ("out", h_out)):
+            if t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+                raise ValueError(f"host {name} must be a contiguous float32 CPU tensor")
+        _check(lib().stq_decode_step_host_static(
+            self.handle, self._slots(slots), B, ctypes.c_void_p(h_q.data_ptr()),
+            ctypes.c_void_p(h_k.data_ptr()), ctypes.c_void_p(h_v.data_ptr()),
+            ctypes.c_void_p(h_gate.data_ptr()), ctypes.c_void_p(h_beta.data_ptr()),
+            ctypes.c_void_p(h_out.data_ptr()), _stream(stream)))
 
     def dequantize(self, slots, S_out, stream=None):
         import torch
