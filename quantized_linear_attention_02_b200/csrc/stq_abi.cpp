@@ -388,6 +388,8 @@ stq_status stq_pool_check(stq_pool* pool, void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "clear of device error word");
     if (bits[0] & stq::ERR_SLOT_RANGE)
       return fail(STQ_ERR_DEVICE_CHECK, "a slot index was outside [0, n_slots); those heads were skipped");
+    if (bits[0] & stq::ERR_TIMEOUT)
+      return fail(STQ_ERR_DEVICE_CHECK, "a kernel gave up waiting for its staged inputs; its outputs are incomplete");
     return fail(STQ_ERR_DEVICE_CHECK, "device error bits 0x%x", bits[0]);
   }
   return ok();

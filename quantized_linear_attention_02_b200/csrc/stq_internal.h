@@ -16,6 +16,7 @@ constexpr int PIVOT = 16;        // width marker of an FP16 pivot unit
 
 // Error bits written by kernels into the pool's device error word.
 constexpr uint32_t ERR_SLOT_RANGE = 1u;   // a slot index was outside [0, n_slots)
+constexpr uint32_t ERR_TIMEOUT = 2u;      // a wait for staged inputs gave up
 
 // Device view of a pool: caller-owned state buffers plus the metadata the library
 // uploaded into the caller-owned meta buffer. Passed to kernels by value.

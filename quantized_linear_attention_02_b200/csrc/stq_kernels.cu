@@ -252,9 +252,9 @@ __device__ __forceinline__ void put_partial(float4 (*red)[D / 4], int w, int lan
 // BITS is the head's uniform width, or MIXED for per-row widths.
 // ---------------------------------------------------------------------------------
 template <int BITS>
-__device__ __forceinline__ void refit_pack(const PoolDev& P, int h, HeadSmem& sm, uint8_t* stage,
-                                           f2 (&s)[RPW][2], float* r_global, f2 (&c_out)[2],
-                                           float* o_global) {
+__device__ __forceinline__ void refit_pack(const float* g_row, const float* om_row, HeadSmem& sm,
+                                           uint8_t* stage, f2 (&s)[RPW][2], float* r_global,
+                                           f2 (&c_out)[2], float* o_global) {
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r0 = w * RPW;
 
@@ -297,8 +297,8 @@ __device__ __forceinline__ void refit_pack(const PoolDev& P, int h, HeadSmem& sm
     const int R = ((lane & 1) << 3) | ((lane & 2) << 1) | ((lane & 4) >> 1) | ((lane & 8) >> 3);
     const int i = r0 + R;
     const bool pivot = (BITS == MIXED) ? (row_bits(sm.info[i]) == PIVOT) : false;
-    const float g = P.g[h * D + i];
-    const float om = P.omega[h * D + i];
+    const float g = g_row[i];
+    const float om = om_row[i];
     const float r = pivot ? 0.0f : fmul(fmul(a[0], 0.0078125f), g);
     if (lane < 16) {
       sm.inv_r[i] = recip_scale(r);
@@ -478,8 +478,9 @@ __device__ __forceinline__ void restore_row(const uint8_t* row, int lane, float 
 // One (request, head) of stq_decode_step.
 // ---------------------------------------------------------------------------------
 template <int BITS>
-__device__ __forceinline__ void decode_head(const PoolDev& P, int h, HeadSmem& sm, uint8_t* stage,
-                                            const HeadRef& hr, const f2 (&cin)[2], float* o_out) {
+__device__ __forceinline__ void decode_head(const float* g_row, const float* om_row, HeadSmem& sm,
+                                            uint8_t* stage, const HeadRef& hr, const f2 (&cin)[2],
+                                            float* o_out) {
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int r0 = w * RPW;
   f2 s[RPW][2];
@@ -572,7 +573,7 @@ __device__ __forceinline__ void decode_head(const PoolDev& P, int h, HeadSmem& s
     }
   }
   f2 c[2];
-  refit_pack<BITS>(P, h, sm, stage, s, hr.scales, c, o_out);
+  refit_pack<BITS>(g_row, om_row, sm, stage, s, hr.scales, c, o_out);
   __syncthreads();
   copy16(hr.codes, stage, hr.code_bytes);
   if (w == 0) *reinterpret_cast<float4*>(hr.scales + D + 4 * lane) = make_float4(c[0].x, c[0].y, c[1].x, c[1].y);
@@ -641,54 +642,241 @@ __device__ __forceinline__ void decode_pivot_head(HeadSmem& sm, uint8_t* stage, 
 }
 
 // ---------------------------------------------------------------------------------
-// stq_decode_step: one CTA per (request, head).
+// stq_decode_step: persistent CTAs, each walking (request, head) items with a stride of
+// the grid size. While one item is computed, the next one's inputs (packed codes, FP16
+// pivot rows, scales, q/k/v, gate, row metadata) stream into the other half of a
+// double buffer with 1-D bulk asynchronous copies that complete on an mbarrier.
 // ---------------------------------------------------------------------------------
+struct __align__(16) HeadIn {
+  float k[D], q[D], v[D];
+  float gate[D];        // KDA per-row retention (unused for GDN)
+  float r[D], c[D];     // input scales (adjacent in the pool)
+  float g[D], om[D];    // row gain and omega of the head
+  uint32_t info[D];     // row widths and offsets
+  HeadRef ref;          // where the item lives in the pool
+  float gate_s, beta_s; // GDN retention and beta (plain loads)
+  int valid;            // slot index in range
+  int pad[3];
+};
+constexpr int HEAD_IN_BYTES = int(sizeof(HeadIn));
+static_assert(HEAD_IN_BYTES % 16 == 0, "staging sections must stay 16-byte aligned");
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+// Global -> shared bulk copy (bytes and both addresses multiples of 16), completing on bar.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for a phase of bar, giving up after about two seconds.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > 2000000000ull) return false;
+  }
+}
+
+// Scalars of one item, loaded by thread 0 an iteration before they are used so that
+// their latency hides behind the current item's compute.
+struct ItemMeta {
+  int slot;
+  uint32_t code_off, code_bytes, piv_first, piv_count, bits;
+  float gate_s, beta_s;
+};
+
+__device__ __forceinline__ ItemMeta load_item_meta(const PoolDev& P, int item,
+                                                   const int32_t* __restrict__ slots,
+                                                   const float* __restrict__ gate,
+                                                   const float* __restrict__ beta) {
+  const int bq = item / P.H, h = item - bq * P.H;
+  ItemMeta m;
+  m.slot = slots[bq];
+  m.code_off = P.head_code_off[h];
+  m.code_bytes = P.head_code_bytes[h];
+  m.piv_first = P.head_piv_first[h];
+  m.piv_count = P.head_piv_count[h];
+  m.bits = P.head_bits[h];
+  m.gate_s = (P.kind == 0) ? gate[item] : 0.0f;
+  m.beta_s = beta[item];
+  return m;
+}
+
+// Thread 0: start loading item `item` into buffer `in` (+ its staging area).
+__device__ __forceinline__ void issue_prefetch(const PoolDev& P, int item, const ItemMeta& m,
+                                               HeadIn& in, uint8_t* stage, uint64_t* bar,
+                                               const float* __restrict__ q,
+                                               const float* __restrict__ k,
+                                               const float* __restrict__ v,
+                                               const float* __restrict__ gate) {
+  const int bq = item / P.H, h = item - bq * P.H;
+  in.gate_s = m.gate_s;
+  in.beta_s = m.beta_s;
+  if (m.slot < 0 || m.slot >= P.n_slots) {
+    atomicOr(P.err, ERR_SLOT_RANGE);
+    in.valid = 0;
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+    return;
+  }
+  in.valid = 1;
+  HeadRef hr;
+  hr.code_bytes = int(m.code_bytes);
+  hr.piv_count = int(m.piv_count);
+  hr.bits = int(m.bits);
+  hr.codes = P.codes + uint64_t(m.slot) * P.slot_code_bytes + m.code_off;
+  hr.pivots = P.pivots + (uint64_t(m.slot) * P.n_pivot_rows + m.piv_first) * D;
+  hr.scales = P.scales + (uint64_t(m.slot) * P.H + h) * 2 * D;
+  hr.piv_stage_off = hr.code_bytes;
+  in.ref = hr;
+  const uint64_t vec = uint64_t(item) * D;
+  uint32_t bytes = 3 * D * 4 + 2 * D * 4 + 3 * D * 4;
+  if (P.kind != 0) bytes += D * 4;
+  bytes += m.code_bytes + m.piv_count * D * 2;
+  mbar_expect_tx(bar, bytes);
+  bulk_load(in.k, k + vec, D * 4, bar);
+  bulk_load(in.q, q + vec, D * 4, bar);
+  bulk_load(in.v, v + vec, D * 4, bar);
+  if (P.kind != 0) bulk_load(in.gate, gate + vec, D * 4, bar);
+  bulk_load(in.r, hr.scales, 2 * D * 4, bar);
+  bulk_load(in.g, P.g + h * D, D * 4, bar);
+  bulk_load(in.om, P.omega + h * D, D * 4, bar);
+  bulk_load(in.info, P.row_info + h * D, D * 4, bar);
+  if (m.code_bytes) bulk_load(stage, hr.codes, m.code_bytes, bar);
+  if (m.piv_count) bulk_load(stage + m.code_bytes, hr.pivots, m.piv_count * D * 2, bar);
+}
+
 __global__ void __launch_bounds__(NT, 2)
 decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* __restrict__ q,
               const float* __restrict__ k, const float* __restrict__ v,
               const float* __restrict__ gate, const float* __restrict__ beta,
-              float* __restrict__ out) {
-  extern __shared__ __align__(16) uint8_t stage[];
+              float* __restrict__ out, int stage_stride) {
+  extern __shared__ __align__(16) uint8_t dyn[];
   __shared__ HeadSmem sm;
-  const int item = blockIdx.x;
-  const int bq = item / P.H, h = item - bq * P.H;
+  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ int abort_flag;
+  HeadIn* ins[2] = {reinterpret_cast<HeadIn*>(dyn), reinterpret_cast<HeadIn*>(dyn + stage_stride)};
+  uint8_t* stages[2] = {dyn + HEAD_IN_BYTES, dyn + stage_stride + HEAD_IN_BYTES};
   const int tid = threadIdx.x, lane = tid & 31;
-  const int slot = slots[bq];
-  if (slot < 0 || slot >= P.n_slots) {
-    if (tid == 0) atomicOr(P.err, ERR_SLOT_RANGE);
-    return;
-  }
-  const HeadRef hr = head_ref(P, slot, h);
-  const uint64_t vec = uint64_t(item) * D;
-
-  // ---- load: per-row vectors, the head's packed codes and pivot rows ----------------
-  load_row_meta(P, h, sm);
-  if (tid < D) {
-    sm.k[tid] = k[vec + tid];
-    sm.q[tid] = q[vec + tid];
-    sm.v[tid] = v[vec + tid];
-    const float dec = (P.kind == 0) ? gate[item] : gate[vec + tid];
-    sm.dec[tid] = dec;
-    sm.rd[tid] = fmul(dec, hr.scales[tid]);
-  }
-  if (tid == 0) sm.beta = beta[item];
-  copy16(stage, hr.codes, hr.code_bytes);
-  copy16(stage + hr.piv_stage_off, hr.pivots, hr.piv_count * D * 2);
-  f2 cin[2];
-  {
-    const float4 c4 = *reinterpret_cast<const float4*>(hr.scales + D + 4 * lane);
-    cin[0] = make_float2(c4.x, c4.y);
-    cin[1] = make_float2(c4.z, c4.w);
+  const int total = B * P.H;
+  int item = blockIdx.x;
+  ItemMeta next_meta;
+  int stuck_n = -1;       // thread 0: iteration whose wait gave up
+  bool stuck_next = false;
+  if (tid == 0) {
+    mbar_init(&bars[0]);
+    mbar_init(&bars[1]);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    abort_flag = 0;
+    if (item < total) {
+      const ItemMeta m0 = load_item_meta(P, item, slots, gate, beta);
+      issue_prefetch(P, item, m0, *ins[0], stages[0], &bars[0], q, k, v, gate);
+    }
+    if (item + int(gridDim.x) < total) next_meta = load_item_meta(P, item + gridDim.x, slots, gate, beta);
   }
   __syncthreads();
-  float* o_out = out + vec;
-  switch (hr.bits) {
-    case 2: decode_head<2>(P, h, sm, stage, hr, cin, o_out); break;
-    case 4: decode_head<4>(P, h, sm, stage, hr, cin, o_out); break;
-    case 6: decode_head<6>(P, h, sm, stage, hr, cin, o_out); break;
-    case 8: decode_head<8>(P, h, sm, stage, hr, cin, o_out); break;
-    case PIVOT: decode_pivot_head(sm, stage, hr, o_out); break;
-    default: decode_head<MIXED>(P, h, sm, stage, hr, cin, o_out); break;
+  for (int n = 0; item < total; ++n, item += gridDim.x) {
+    const int b = n & 1;
+    const int next = item + gridDim.x;
+    HeadIn& in = *ins[b];
+    uint8_t* stage = stages[b];
+    if (tid == 0) {
+      if (next < total) {
+        // the other buffer was last read in iteration n-1, which ended with a barrier;
+        // order those generic-proxy accesses before the asynchronous writes
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue_prefetch(P, next, next_meta, *ins[b ^ 1], stages[b ^ 1], &bars[b ^ 1], q, k, v, gate);
+        if (next + int(gridDim.x) < total) next_meta = load_item_meta(P, next + gridDim.x, slots, gate, beta);
+      }
+      if (!mbar_wait_bounded(&bars[b], uint32_t(n >> 1) & 1u)) {
+        atomicOr(P.err, ERR_TIMEOUT);
+        abort_flag = 1;
+        stuck_n = n;
+        stuck_next = next < total;
+      }
+    }
+    __syncthreads();
+    if (abort_flag) break;
+    if (in.valid) {
+      const HeadRef hr = in.ref;
+      const uint64_t vec = uint64_t(item) * D;
+      if (tid < D) {
+        const uint32_t info = in.info[tid];
+        const int bits = row_bits(info);
+        sm.info[tid] = info;
+        if (bits == PIVOT) {
+          sm.qm[tid] = 0.0f;
+          sm.iq[tid] = 0.0f;
+          sm.mb[tid] = MAGIC;
+          sm.tb[tid] = TWO23;
+        } else {
+          const int bias = 1 << (bits - 1);
+          sm.qm[tid] = float(bias - 1);
+          sm.iq[tid] = __frcp_rn(float(bias - 1));
+          sm.mb[tid] = MAGIC + float(bias);
+          sm.tb[tid] = TWO23 + float(bias);
+        }
+        sm.k[tid] = in.k[tid];
+        sm.q[tid] = in.q[tid];
+        sm.v[tid] = in.v[tid];
+        const float dec = (P.kind == 0) ? in.gate_s : in.gate[tid];
+        sm.dec[tid] = dec;
+        sm.rd[tid] = fmul(dec, in.r[tid]);
+      }
+      if (tid == 0) sm.beta = in.beta_s;
+      const float4 c4 = *reinterpret_cast<const float4*>(&in.c[4 * lane]);
+      const f2 cin[2] = {make_float2(c4.x, c4.y), make_float2(c4.z, c4.w)};
+      __syncthreads();
+      float* o_out = out + vec;
+      switch (hr.bits) {
+        case 2: decode_head<2>(in.g, in.om, sm, stage, hr, cin, o_out); break;
+        case 4: decode_head<4>(in.g, in.om, sm, stage, hr, cin, o_out); break;
+        case 6: decode_head<6>(in.g, in.om, sm, stage, hr, cin, o_out); break;
+        case 8: decode_head<8>(in.g, in.om, sm, stage, hr, cin, o_out); break;
+        case PIVOT: decode_pivot_head(sm, stage, hr, o_out); break;
+        default: decode_head<MIXED>(in.g, in.om, sm, stage, hr, cin, o_out); break;
+      }
+    }
+    __syncthreads();
+  }
+  if (tid == 0 && stuck_n >= 0) {
+    // give the loads this CTA started a bounded chance to land before its shared
+    // memory goes away: the phase that timed out and the prefetch issued after it
+    mbar_wait_bounded(&bars[stuck_n & 1], uint32_t(stuck_n >> 1) & 1u);
+    if (stuck_next) mbar_wait_bounded(&bars[(stuck_n + 1) & 1], uint32_t((stuck_n + 1) >> 1) & 1u);
   }
 }
 
@@ -714,7 +902,7 @@ __device__ __forceinline__ void quantize_head(const PoolDev& P, int h, HeadSmem&
     }
   }
   f2 c[2];
-  refit_pack<BITS>(P, h, sm, stage, s, hr.scales, c, nullptr);
+  refit_pack<BITS>(P.g + h * D, P.omega + h * D, sm, stage, s, hr.scales, c, nullptr);
   __syncthreads();
   copy16(hr.codes, stage, hr.code_bytes);
   if (w == 0) *reinterpret_cast<float4*>(hr.scales + D + 4 * lane) = make_float4(c[0].x, c[0].y, c[1].x, c[1].y);
@@ -909,10 +1097,18 @@ cudaError_t launch_decode(const PoolDev& P, const int32_t* slots, int B, const f
                           const float* k, const float* v, const float* gate,
                           const float* beta, float* out, cudaStream_t s) {
   if (B == 0) return cudaSuccess;
-  const int dyn = stage_bytes(P);
-  cudaError_t e = prepare(decode_kernel, dyn, int(sizeof(HeadSmem)), g_decode_dyn);
+  const int stride = HEAD_IN_BYTES + stage_bytes(P);
+  const int dyn = 2 * stride;
+  cudaError_t e = prepare(decode_kernel, dyn, int(sizeof(HeadSmem)) + 64, g_decode_dyn);
   if (e != cudaSuccess) return e;
-  decode_kernel<<<B * P.H, NT, dyn, s>>>(P, slots, B, q, k, v, gate, beta, out);
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const long long items = (long long)B * P.H;
+  const int grid = int(items < 2LL * sms ? items : 2LL * sms);
+  decode_kernel<<<grid, NT, dyn, s>>>(P, slots, B, q, k, v, gate, beta, out, stride);
   return cudaGetLastError();
 }
 
