@@ -80,18 +80,29 @@ __device__ __forceinline__ V2<M> tree(F&& f) {
 }
 
 struct __align__(16) HeadSmem {
-  float k[D], q[D], v[D], dec[D];
-  float rd[D];       // decayed input row scale dec_i * r_i
   float inv_r[D];    // 1/r_i of the refit
   float b[D];        // omega_i * r_i^2
-  float qm[D];       // qmax_i (0 for pivot rows)
-  float iq[D];       // 1/qmax_i (0 for pivot rows)
-  float mb[D];       // 1.5*2^23 + 2^(b-1): magic that yields the biased code
-  float tb[D];       // 2^23 + 2^(b-1): magic that turns a code into its value
-  uint32_t info[D];  // bits | offset << 8
+  uint32_t info[D];  // bits | offset << 8 (quantiser path)
+  // per-width constants, indexed by the width (2/4/6/8; 16 = pivot row, others unused)
+  float tqm[32];     // qmax = 2^(b-1) - 1 (0 for pivots)
+  float tiq[32];     // 1/qmax (0 for pivots)
+  float tmb[32];     // 1.5*2^23 + 2^(b-1): magic that yields the biased code
+  float ttb[32];     // 2^23 + 2^(b-1): magic that turns a code into its value
   float4 red[2][2][NW][D / 4];  // ping-pong partials: [buffer][quantity][warp][col/4]
-  float beta;
 };
+
+// Fill the per-width tables (threads 0..31).
+__device__ __forceinline__ void init_width_tables(HeadSmem& sm) {
+  const int bits = threadIdx.x;
+  if (bits < 32) {
+    const bool q = bits == 2 || bits == 4 || bits == 6 || bits == 8;
+    const int bias = q ? (1 << (bits - 1)) : 0;
+    sm.tqm[bits] = q ? float(bias - 1) : 0.0f;
+    sm.tiq[bits] = q ? __frcp_rn(float(bias - 1)) : 0.0f;
+    sm.tmb[bits] = MAGIC + float(bias);
+    sm.ttb[bits] = TWO23 + float(bias);
+  }
+}
 
 __device__ __forceinline__ int row_bits(uint32_t info) { return int(info & 0xFFu); }
 __device__ __forceinline__ int row_off(uint32_t info) { return int(info >> 8); }
@@ -188,26 +199,10 @@ __device__ __forceinline__ HeadRef head_ref(const PoolDev& P, int slot, int h) {
   return r;
 }
 
-// Per-row static data of head h into shared memory (threads 0..127, one row each).
+// Row widths and offsets of head h into shared memory (threads 0..127, one row each).
 __device__ __forceinline__ void load_row_meta(const PoolDev& P, int h, HeadSmem& sm) {
   const int i = threadIdx.x;
-  if (i < D) {
-    const uint32_t info = P.row_info[h * D + i];
-    const int bits = row_bits(info);
-    sm.info[i] = info;
-    if (bits == PIVOT) {
-      sm.qm[i] = 0.0f;
-      sm.iq[i] = 0.0f;
-      sm.mb[i] = MAGIC;
-      sm.tb[i] = TWO23;
-    } else {
-      const int bias = 1 << (bits - 1);
-      sm.qm[i] = float(bias - 1);
-      sm.iq[i] = __frcp_rn(float(bias - 1));
-      sm.mb[i] = MAGIC + float(bias);
-      sm.tb[i] = TWO23 + float(bias);
-    }
-  }
+  if (i < D) sm.info[i] = P.row_info[h * D + i];
 }
 
 __device__ __forceinline__ uint2 half4_bits(f2 a, f2 b) {
@@ -252,7 +247,8 @@ __device__ __forceinline__ void put_partial(float4 (*red)[D / 4], int w, int lan
 // BITS is the head's uniform width, or MIXED for per-row widths.
 // ---------------------------------------------------------------------------------
 template <int BITS>
-__device__ __forceinline__ void refit_pack(const float* g_row, const float* om_row, HeadSmem& sm,
+__device__ __forceinline__ void refit_pack(const float* g_row, const float* om_row,
+                                           const uint32_t* info_row, HeadSmem& sm,
                                            uint8_t* stage, f2 (&s)[RPW][2], float* r_global,
                                            f2 (&c_out)[2], float* o_global) {
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -296,7 +292,7 @@ __device__ __forceinline__ void refit_pack(const float* g_row, const float* om_r
     // lane l now holds the sum of row R(l): bits 0..3 of l chose halves 8, 4, 2, 1
     const int R = ((lane & 1) << 3) | ((lane & 2) << 1) | ((lane & 4) >> 1) | ((lane & 8) >> 3);
     const int i = r0 + R;
-    const bool pivot = (BITS == MIXED) ? (row_bits(sm.info[i]) == PIVOT) : false;
+    const bool pivot = (BITS == MIXED) ? (row_bits(info_row[i]) == PIVOT) : false;
     const float g = g_row[i];
     const float om = om_row[i];
     const float r = pivot ? 0.0f : fmul(fmul(a[0], 0.0078125f), g);
@@ -314,7 +310,11 @@ __device__ __forceinline__ void refit_pack(const float* g_row, const float* om_r
   for (int g4 = 0; g4 < RPW / 4; ++g4) {
     const float4 ir4 = *reinterpret_cast<const float4*>(&sm.inv_r[r0 + 4 * g4]);
     float4 iq4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    if constexpr (BITS == MIXED) iq4 = *reinterpret_cast<const float4*>(&sm.iq[r0 + 4 * g4]);
+    if constexpr (BITS == MIXED) {
+      const uint4 in4 = *reinterpret_cast<const uint4*>(&info_row[r0 + 4 * g4]);
+      iq4 = make_float4(sm.tiq[row_bits(in4.x)], sm.tiq[row_bits(in4.y)], sm.tiq[row_bits(in4.z)],
+                        sm.tiq[row_bits(in4.w)]);
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int rr = 4 * g4 + j;
@@ -372,7 +372,11 @@ __device__ __forceinline__ void refit_pack(const float* g_row, const float* om_r
       // rows 2m and 2m+1 form one fused pair of each sum
       if ((m & 1) == 0) {
         b4 = *reinterpret_cast<const float4*>(&sm.b[r0 + 2 * m]);
-        if constexpr (BITS == MIXED) q4 = *reinterpret_cast<const float4*>(&sm.qm[r0 + 2 * m]);
+        if constexpr (BITS == MIXED) {
+          const uint4 in4 = *reinterpret_cast<const uint4*>(&info_row[r0 + 2 * m]);
+          q4 = make_float4(sm.tqm[row_bits(in4.x)], sm.tqm[row_bits(in4.y)], sm.tqm[row_bits(in4.z)],
+                           sm.tqm[row_bits(in4.w)]);
+        }
       }
       f2 Q[2][2], p[2][2];
 #pragma unroll
@@ -427,10 +431,10 @@ __device__ __forceinline__ void refit_pack(const float* g_row, const float* om_r
   for (int rr = 0; rr < RPW; ++rr) {
     const int i = r0 + rr;
     if constexpr (BITS == MIXED) {
-      const uint32_t info = sm.info[i];
+      const uint32_t info = info_row[i];
       const int bits = row_bits(info);
       if (bits == PIVOT) continue;
-      const float mb = sm.mb[i], q = sm.qm[i];
+      const float mb = sm.tmb[bits], q = sm.tqm[bits];
       const f2 t01 = fma2(s[rr][0], ic[0], dup(mb));
       const f2 t23 = fma2(s[rr][1], ic[1], dup(mb));
       const float lo_b = mb - q, hi_b = mb + q;
@@ -475,177 +479,7 @@ __device__ __forceinline__ void restore_row(const uint8_t* row, int lane, float 
 }
 
 // ---------------------------------------------------------------------------------
-// One (request, head) of stq_decode_step.
-// ---------------------------------------------------------------------------------
-template <int BITS>
-__device__ __forceinline__ void decode_head(const float* g_row, const float* om_row, HeadSmem& sm,
-                                            uint8_t* stage, const HeadRef& hr, const f2 (&cin)[2],
-                                            float* o_out) {
-  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  const int r0 = w * RPW;
-  f2 s[RPW][2];
-
-  // ---- restore S' and the column sums u_j = sum_i k_i S'_ij ---------------------------
-#pragma unroll
-  for (int g4 = 0; g4 < RPW / 4; ++g4) {
-    const float4 rd4 = *reinterpret_cast<const float4*>(&sm.rd[r0 + 4 * g4]);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int rr = 4 * g4 + j, i = r0 + rr;
-      if constexpr (BITS == MIXED) {
-        const uint32_t info = sm.info[i];
-        const int bits = row_bits(info);
-        const uint8_t* row = stage + row_off(info);
-        const float tb = sm.tb[i];
-        switch (bits) {
-          case 2: restore_row<2>(row, lane, at4(rd4, j), tb, cin, s[rr][0], s[rr][1]); break;
-          case 4: restore_row<4>(row, lane, at4(rd4, j), tb, cin, s[rr][0], s[rr][1]); break;
-          case 6: restore_row<6>(row, lane, at4(rd4, j), tb, cin, s[rr][0], s[rr][1]); break;
-          case 8: restore_row<8>(row, lane, at4(rd4, j), tb, cin, s[rr][0], s[rr][1]); break;
-          default: {
-            const uint2 hv = *reinterpret_cast<const uint2*>(stage + hr.piv_stage_off +
-                                                              row_off(info) * (D * 2) + 8 * lane);
-            f2 a, b;
-            half4_floats(hv, a, b);
-            const f2 dd = dup(sm.dec[i]);
-            s[rr][0] = mul2(dd, a);
-            s[rr][1] = mul2(dd, b);
-          }
-        }
-      } else {
-        constexpr float TB = TWO23 + float(1 << (BITS - 1));
-        restore_row<BITS>(stage + i * (D * BITS / 8), lane, at4(rd4, j), TB, cin, s[rr][0], s[rr][1]);
-      }
-    }
-  }
-  {
-    float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    V2<2> u = tree<0, RPW / 2, 2>([&](int m) {
-      if ((m & 1) == 0) k4 = *reinterpret_cast<const float4*>(&sm.k[r0 + 2 * m]);
-      const f2 ke = dup(at4(k4, (2 * m) & 3)), ko = dup(at4(k4, (2 * m + 1) & 3));
-      V2<2> leaf;
-      leaf.x[0] = fma2(ke, s[2 * m][0], mul2(ko, s[2 * m + 1][0]));
-      leaf.x[1] = fma2(ke, s[2 * m][1], mul2(ko, s[2 * m + 1][1]));
-      return leaf;
-    });
-    put_partial(sm.red[0][0], w, lane, u.x[0], u.x[1]);
-  }
-  __syncthreads();
-
-  // ---- delta_j = beta (v_j - u_j); S = S' + k delta^T; readout partials ----------------
-  f2 delta[2];
-  {
-    f2 ulo, uhi;
-    warp_tree(sm.red[0][0], lane, ulo, uhi);
-    const float4 v4 = *reinterpret_cast<const float4*>(&sm.v[4 * lane]);
-    const f2 bt = dup(sm.beta);
-    delta[0] = mul2(bt, add2(make_float2(v4.x, v4.y), make_float2(-ulo.x, -ulo.y)));
-    delta[1] = mul2(bt, add2(make_float2(v4.z, v4.w), make_float2(-uhi.x, -uhi.y)));
-  }
-  {
-    float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f), q4 = k4;
-    V2<2> o = tree<0, RPW / 2, 2>([&](int m) {
-      if ((m & 1) == 0) {
-        k4 = *reinterpret_cast<const float4*>(&sm.k[r0 + 2 * m]);
-        q4 = *reinterpret_cast<const float4*>(&sm.q[r0 + 2 * m]);
-      }
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const f2 kk = dup(at4(k4, (2 * m + e) & 3));
-        s[2 * m + e][0] = fma2(kk, delta[0], s[2 * m + e][0]);
-        s[2 * m + e][1] = fma2(kk, delta[1], s[2 * m + e][1]);
-      }
-      const f2 qe = dup(at4(q4, (2 * m) & 3)), qo = dup(at4(q4, (2 * m + 1) & 3));
-      V2<2> leaf;
-      leaf.x[0] = fma2(qe, s[2 * m][0], mul2(qo, s[2 * m + 1][0]));
-      leaf.x[1] = fma2(qe, s[2 * m][1], mul2(qo, s[2 * m + 1][1]));
-      return leaf;
-    });
-    put_partial(sm.red[1][0], w, lane, o.x[0], o.x[1]);
-  }
-  if constexpr (BITS == MIXED) {
-    // pivot rows: store float16(S) now (they take no part in the refit)
-#pragma unroll
-    for (int rr = 0; rr < RPW; ++rr) {
-      const uint32_t info = sm.info[r0 + rr];
-      if (row_bits(info) == PIVOT)
-        *reinterpret_cast<uint2*>(hr.pivots + row_off(info) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
-    }
-  }
-  f2 c[2];
-  refit_pack<BITS>(g_row, om_row, sm, stage, s, hr.scales, c, o_out);
-  __syncthreads();
-  copy16(hr.codes, stage, hr.code_bytes);
-  if (w == 0) *reinterpret_cast<float4*>(hr.scales + D + 4 * lane) = make_float4(c[0].x, c[0].y, c[1].x, c[1].y);
-}
-
-// A head whose rows are all FP16 pivots: decay, update, readout, store float16; r = c = 0.
-__device__ __forceinline__ void decode_pivot_head(HeadSmem& sm, uint8_t* stage, const HeadRef& hr,
-                                                  float* o_out) {
-  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  const int r0 = w * RPW;
-  f2 s[RPW][2];
-#pragma unroll
-  for (int rr = 0; rr < RPW; ++rr) {
-    const int i = r0 + rr;
-    const uint2 hv = *reinterpret_cast<const uint2*>(stage + i * (D * 2) + 8 * lane);
-    f2 a, b;
-    half4_floats(hv, a, b);
-    const f2 dd = dup(sm.dec[i]);
-    s[rr][0] = mul2(dd, a);
-    s[rr][1] = mul2(dd, b);
-  }
-  {
-    V2<2> u = tree<0, RPW / 2, 2>([&](int m) {
-      const f2 ke = dup(sm.k[r0 + 2 * m]), ko = dup(sm.k[r0 + 2 * m + 1]);
-      V2<2> leaf;
-      leaf.x[0] = fma2(ke, s[2 * m][0], mul2(ko, s[2 * m + 1][0]));
-      leaf.x[1] = fma2(ke, s[2 * m][1], mul2(ko, s[2 * m + 1][1]));
-      return leaf;
-    });
-    put_partial(sm.red[0][0], w, lane, u.x[0], u.x[1]);
-  }
-  __syncthreads();
-  f2 delta[2];
-  {
-    f2 ulo, uhi;
-    warp_tree(sm.red[0][0], lane, ulo, uhi);
-    const float4 v4 = *reinterpret_cast<const float4*>(&sm.v[4 * lane]);
-    const f2 bt = dup(sm.beta);
-    delta[0] = mul2(bt, add2(make_float2(v4.x, v4.y), make_float2(-ulo.x, -ulo.y)));
-    delta[1] = mul2(bt, add2(make_float2(v4.z, v4.w), make_float2(-uhi.x, -uhi.y)));
-  }
-  V2<2> o = tree<0, RPW / 2, 2>([&](int m) {
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const f2 kk = dup(sm.k[r0 + 2 * m + e]);
-      s[2 * m + e][0] = fma2(kk, delta[0], s[2 * m + e][0]);
-      s[2 * m + e][1] = fma2(kk, delta[1], s[2 * m + e][1]);
-    }
-    const f2 qe = dup(sm.q[r0 + 2 * m]), qo = dup(sm.q[r0 + 2 * m + 1]);
-    V2<2> leaf;
-    leaf.x[0] = fma2(qe, s[2 * m][0], mul2(qo, s[2 * m + 1][0]));
-    leaf.x[1] = fma2(qe, s[2 * m][1], mul2(qo, s[2 * m + 1][1]));
-    return leaf;
-  });
-  put_partial(sm.red[1][0], w, lane, o.x[0], o.x[1]);
-#pragma unroll
-  for (int rr = 0; rr < RPW; ++rr)
-    *reinterpret_cast<uint2*>(hr.pivots + (r0 + rr) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
-  __syncthreads();
-  if (w == 0) {
-    f2 lo, hi;
-    warp_tree(sm.red[1][0], lane, lo, hi);
-    *reinterpret_cast<float4*>(o_out + 4 * lane) = make_float4(lo.x, lo.y, hi.x, hi.y);
-  }
-  if (tid < 2 * D) hr.scales[tid] = 0.0f;
-}
-
-// ---------------------------------------------------------------------------------
-// stq_decode_step: persistent CTAs, each walking (request, head) items with a stride of
-// the grid size. While one item is computed, the next one's inputs (packed codes, FP16
-// pivot rows, scales, q/k/v, gate, row metadata) stream into the other half of a
-// double buffer with 1-D bulk asynchronous copies that complete on an mbarrier.
+// Staged inputs of one (request, head) and the asynchronous-copy helpers.
 // ---------------------------------------------------------------------------------
 struct __align__(16) HeadIn {
   float k[D], q[D], v[D];
@@ -711,48 +545,66 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
-// Scalars of one item, loaded by thread 0 an iteration before they are used so that
-// their latency hides behind the current item's compute.
+// Scalars of one item (slot index, head record, GDN gate, beta). Lanes 0..7 of warp 0
+// fetch them into shared memory with 4-byte asynchronous copies an iteration before
+// they are needed, so that no register holds them across an item's compute.
 struct ItemMeta {
   int slot;
   uint32_t code_off, code_bytes, piv_first, piv_count, bits;
   float gate_s, beta_s;
 };
 
-__device__ __forceinline__ ItemMeta load_item_meta(const PoolDev& P, int item,
-                                                   const int32_t* __restrict__ slots,
-                                                   const float* __restrict__ gate,
-                                                   const float* __restrict__ beta) {
-  const int bq = item / P.H, h = item - bq * P.H;
-  ItemMeta m;
-  m.slot = slots[bq];
-  m.code_off = P.head_code_off[h];
-  m.code_bytes = P.head_code_bytes[h];
-  m.piv_first = P.head_piv_first[h];
-  m.piv_count = P.head_piv_count[h];
-  m.bits = P.head_bits[h];
-  m.gate_s = (P.kind == 0) ? gate[item] : 0.0f;
-  m.beta_s = beta[item];
-  return m;
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
 }
 
-// Thread 0: start loading item `item` into buffer `in` (+ its staging area).
-__device__ __forceinline__ void issue_prefetch(const PoolDev& P, int item, const ItemMeta& m,
+__device__ __forceinline__ void start_item_meta(const PoolDev& P, int item, int B,
+                                                const int32_t* __restrict__ slots,
+                                                const float* __restrict__ gate,
+                                                const float* __restrict__ beta, ItemMeta& m,
+                                                int lane) {
+  const int h = item / B, bq = item - h * B;   // items run head-major: same width in a row
+  const int vi = bq * P.H + h;
+  switch (lane) {
+    case 0: cp_async4(&m.slot, slots + bq); break;
+    case 1: cp_async4(&m.code_off, P.head_code_off + h); break;
+    case 2: cp_async4(&m.code_bytes, P.head_code_bytes + h); break;
+    case 3: cp_async4(&m.piv_first, P.head_piv_first + h); break;
+    case 4: cp_async4(&m.piv_count, P.head_piv_count + h); break;
+    case 5: cp_async4(&m.bits, P.head_bits + h); break;
+    case 6: if (P.kind == 0) cp_async4(&m.gate_s, gate + vi); break;
+    case 7: cp_async4(&m.beta_s, beta + vi); break;
+    default: break;
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// Wait for this warp's outstanding 4-byte copies, then make them visible warp-wide.
+__device__ __forceinline__ void finish_item_meta() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncwarp();
+}
+
+// Warp 0: start loading item `item` into buffer `in` (+ its staging area). Lane 0 sets
+// the expected byte count, then the lanes issue the copies side by side.
+__device__ __forceinline__ void issue_prefetch(const PoolDev& P, int item, int B, const ItemMeta m,
                                                HeadIn& in, uint8_t* stage, uint64_t* bar,
                                                const float* __restrict__ q,
                                                const float* __restrict__ k,
                                                const float* __restrict__ v,
-                                               const float* __restrict__ gate) {
-  const int bq = item / P.H, h = item - bq * P.H;
-  in.gate_s = m.gate_s;
-  in.beta_s = m.beta_s;
-  if (m.slot < 0 || m.slot >= P.n_slots) {
-    atomicOr(P.err, ERR_SLOT_RANGE);
-    in.valid = 0;
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+                                               const float* __restrict__ gate, int lane) {
+  const int h = item / B, bq = item - h * B;
+  const bool ok = m.slot >= 0 && m.slot < P.n_slots;
+  if (!ok) {
+    if (lane == 0) {
+      atomicOr(P.err, ERR_SLOT_RANGE);
+      in.valid = 0;
+      in.gate_s = m.gate_s;
+      in.beta_s = m.beta_s;
+      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+    }
     return;
   }
-  in.valid = 1;
   HeadRef hr;
   hr.code_bytes = int(m.code_bytes);
   hr.piv_count = int(m.piv_count);
@@ -761,24 +613,217 @@ __device__ __forceinline__ void issue_prefetch(const PoolDev& P, int item, const
   hr.pivots = P.pivots + (uint64_t(m.slot) * P.n_pivot_rows + m.piv_first) * D;
   hr.scales = P.scales + (uint64_t(m.slot) * P.H + h) * 2 * D;
   hr.piv_stage_off = hr.code_bytes;
-  in.ref = hr;
-  const uint64_t vec = uint64_t(item) * D;
-  uint32_t bytes = 3 * D * 4 + 2 * D * 4 + 3 * D * 4;
-  if (P.kind != 0) bytes += D * 4;
-  bytes += m.code_bytes + m.piv_count * D * 2;
-  mbar_expect_tx(bar, bytes);
-  bulk_load(in.k, k + vec, D * 4, bar);
-  bulk_load(in.q, q + vec, D * 4, bar);
-  bulk_load(in.v, v + vec, D * 4, bar);
-  if (P.kind != 0) bulk_load(in.gate, gate + vec, D * 4, bar);
-  bulk_load(in.r, hr.scales, 2 * D * 4, bar);
-  bulk_load(in.g, P.g + h * D, D * 4, bar);
-  bulk_load(in.om, P.omega + h * D, D * 4, bar);
-  bulk_load(in.info, P.row_info + h * D, D * 4, bar);
-  if (m.code_bytes) bulk_load(stage, hr.codes, m.code_bytes, bar);
-  if (m.piv_count) bulk_load(stage + m.code_bytes, hr.pivots, m.piv_count * D * 2, bar);
+  const uint64_t vec = (uint64_t(bq) * P.H + h) * D;
+  if (lane == 0) {
+    in.valid = 1;
+    in.ref = hr;
+    in.gate_s = m.gate_s;
+    in.beta_s = m.beta_s;
+    uint32_t bytes = 3 * D * 4 + 2 * D * 4 + 3 * D * 4;
+    if (P.kind != 0) bytes += D * 4;
+    bytes += m.code_bytes + m.piv_count * D * 2;
+    mbar_expect_tx(bar, bytes);
+  }
+  __syncwarp();
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  switch (lane) {
+    case 0: bulk_load(in.k, k + vec, D * 4, bar); break;
+    case 1: bulk_load(in.q, q + vec, D * 4, bar); break;
+    case 2: bulk_load(in.v, v + vec, D * 4, bar); break;
+    case 3: if (P.kind != 0) bulk_load(in.gate, gate + vec, D * 4, bar); break;
+    case 4: bulk_load(in.r, hr.scales, 2 * D * 4, bar); break;
+    case 5: bulk_load(in.g, P.g + h * D, D * 4, bar); break;
+    case 6: bulk_load(in.om, P.omega + h * D, D * 4, bar); break;
+    case 7: bulk_load(in.info, P.row_info + h * D, D * 4, bar); break;
+    case 8: if (m.code_bytes) bulk_load(stage, hr.codes, m.code_bytes, bar); break;
+    case 9: if (m.piv_count) bulk_load(stage + m.code_bytes, hr.pivots, m.piv_count * D * 2, bar); break;
+    default: break;
+  }
 }
 
+// ---------------------------------------------------------------------------------
+// One (request, head) of stq_decode_step, reading its staged inputs `in`.
+// ---------------------------------------------------------------------------------
+template <int BITS>
+__device__ __forceinline__ void decode_head(const HeadIn& in, int kind, HeadSmem& sm, uint8_t* stage,
+                                            float* o_out) {
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int r0 = w * RPW;
+  const HeadRef& hr = in.ref;
+  f2 s[RPW][2];
+  f2 cin[2];
+  {
+    const float4 c4 = *reinterpret_cast<const float4*>(&in.c[4 * lane]);
+    cin[0] = make_float2(c4.x, c4.y);
+    cin[1] = make_float2(c4.z, c4.w);
+  }
+
+  // ---- restore S' = D (r c Q) and the column sums u_j = sum_i k_i S'_ij ---------------
+#pragma unroll
+  for (int g4 = 0; g4 < RPW / 4; ++g4) {
+    const float4 r4 = *reinterpret_cast<const float4*>(&in.r[r0 + 4 * g4]);
+    float4 d4 = make_float4(in.gate_s, in.gate_s, in.gate_s, in.gate_s);
+    if (kind != 0) d4 = *reinterpret_cast<const float4*>(&in.gate[r0 + 4 * g4]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int rr = 4 * g4 + j, i = r0 + rr;
+      const float dec = at4(d4, j);
+      const float rd = fmul(dec, at4(r4, j));
+      if constexpr (BITS == MIXED) {
+        const uint32_t info = in.info[i];
+        const int bits = row_bits(info);
+        const uint8_t* row = stage + row_off(info);
+        const float tb = sm.ttb[bits];
+        switch (bits) {
+          case 2: restore_row<2>(row, lane, rd, tb, cin, s[rr][0], s[rr][1]); break;
+          case 4: restore_row<4>(row, lane, rd, tb, cin, s[rr][0], s[rr][1]); break;
+          case 6: restore_row<6>(row, lane, rd, tb, cin, s[rr][0], s[rr][1]); break;
+          case 8: restore_row<8>(row, lane, rd, tb, cin, s[rr][0], s[rr][1]); break;
+          default: {
+            const uint2 hv = *reinterpret_cast<const uint2*>(stage + hr.piv_stage_off +
+                                                              row_off(info) * (D * 2) + 8 * lane);
+            f2 a, b;
+            half4_floats(hv, a, b);
+            s[rr][0] = mul2(dup(dec), a);
+            s[rr][1] = mul2(dup(dec), b);
+          }
+        }
+      } else {
+        constexpr float TB = TWO23 + float(1 << (BITS - 1));
+        restore_row<BITS>(stage + i * (D * BITS / 8), lane, rd, TB, cin, s[rr][0], s[rr][1]);
+      }
+    }
+  }
+  {
+    float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    V2<2> u = tree<0, RPW / 2, 2>([&](int m) {
+      if ((m & 1) == 0) k4 = *reinterpret_cast<const float4*>(&in.k[r0 + 2 * m]);
+      const f2 ke = dup(at4(k4, (2 * m) & 3)), ko = dup(at4(k4, (2 * m + 1) & 3));
+      V2<2> leaf;
+      leaf.x[0] = fma2(ke, s[2 * m][0], mul2(ko, s[2 * m + 1][0]));
+      leaf.x[1] = fma2(ke, s[2 * m][1], mul2(ko, s[2 * m + 1][1]));
+      return leaf;
+    });
+    put_partial(sm.red[0][0], w, lane, u.x[0], u.x[1]);
+  }
+  __syncthreads();
+
+  // ---- delta_j = beta (v_j - u_j); S = S' + k delta^T; readout partials ----------------
+  f2 delta[2];
+  {
+    f2 ulo, uhi;
+    warp_tree(sm.red[0][0], lane, ulo, uhi);
+    const float4 v4 = *reinterpret_cast<const float4*>(&in.v[4 * lane]);
+    const f2 bt = dup(in.beta_s);
+    delta[0] = mul2(bt, add2(make_float2(v4.x, v4.y), make_float2(-ulo.x, -ulo.y)));
+    delta[1] = mul2(bt, add2(make_float2(v4.z, v4.w), make_float2(-uhi.x, -uhi.y)));
+  }
+  {
+    float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f), q4 = k4;
+    V2<2> o = tree<0, RPW / 2, 2>([&](int m) {
+      if ((m & 1) == 0) {
+        k4 = *reinterpret_cast<const float4*>(&in.k[r0 + 2 * m]);
+        q4 = *reinterpret_cast<const float4*>(&in.q[r0 + 2 * m]);
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const f2 kk = dup(at4(k4, (2 * m + e) & 3));
+        s[2 * m + e][0] = fma2(kk, delta[0], s[2 * m + e][0]);
+        s[2 * m + e][1] = fma2(kk, delta[1], s[2 * m + e][1]);
+      }
+      const f2 qe = dup(at4(q4, (2 * m) & 3)), qo = dup(at4(q4, (2 * m + 1) & 3));
+      V2<2> leaf;
+      leaf.x[0] = fma2(qe, s[2 * m][0], mul2(qo, s[2 * m + 1][0]));
+      leaf.x[1] = fma2(qe, s[2 * m][1], mul2(qo, s[2 * m + 1][1]));
+      return leaf;
+    });
+    put_partial(sm.red[1][0], w, lane, o.x[0], o.x[1]);
+  }
+  if constexpr (BITS == MIXED) {
+    // pivot rows: store float16(S) now (they take no part in the refit)
+#pragma unroll
+    for (int rr = 0; rr < RPW; ++rr) {
+      const uint32_t info = in.info[r0 + rr];
+      if (row_bits(info) == PIVOT)
+        *reinterpret_cast<uint2*>(hr.pivots + row_off(info) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
+    }
+  }
+  f2 c[2];
+  refit_pack<BITS>(in.g, in.om, in.info, sm, stage, s, hr.scales, c, o_out);
+  __syncthreads();
+  copy16(hr.codes, stage, hr.code_bytes);
+  if (w == 0) *reinterpret_cast<float4*>(hr.scales + D + 4 * lane) = make_float4(c[0].x, c[0].y, c[1].x, c[1].y);
+}
+
+// A head whose rows are all FP16 pivots: decay, update, readout, store float16; r = c = 0.
+__device__ __forceinline__ void decode_pivot_head(const HeadIn& in, int kind, HeadSmem& sm,
+                                                  const uint8_t* stage, float* o_out) {
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int r0 = w * RPW;
+  const HeadRef& hr = in.ref;
+  f2 s[RPW][2];
+#pragma unroll
+  for (int rr = 0; rr < RPW; ++rr) {
+    const int i = r0 + rr;
+    const uint2 hv = *reinterpret_cast<const uint2*>(stage + i * (D * 2) + 8 * lane);
+    f2 a, b;
+    half4_floats(hv, a, b);
+    const f2 dd = dup(kind != 0 ? in.gate[i] : in.gate_s);
+    s[rr][0] = mul2(dd, a);
+    s[rr][1] = mul2(dd, b);
+  }
+  {
+    V2<2> u = tree<0, RPW / 2, 2>([&](int m) {
+      const f2 ke = dup(in.k[r0 + 2 * m]), ko = dup(in.k[r0 + 2 * m + 1]);
+      V2<2> leaf;
+      leaf.x[0] = fma2(ke, s[2 * m][0], mul2(ko, s[2 * m + 1][0]));
+      leaf.x[1] = fma2(ke, s[2 * m][1], mul2(ko, s[2 * m + 1][1]));
+      return leaf;
+    });
+    put_partial(sm.red[0][0], w, lane, u.x[0], u.x[1]);
+  }
+  __syncthreads();
+  f2 delta[2];
+  {
+    f2 ulo, uhi;
+    warp_tree(sm.red[0][0], lane, ulo, uhi);
+    const float4 v4 = *reinterpret_cast<const float4*>(&in.v[4 * lane]);
+    const f2 bt = dup(in.beta_s);
+    delta[0] = mul2(bt, add2(make_float2(v4.x, v4.y), make_float2(-ulo.x, -ulo.y)));
+    delta[1] = mul2(bt, add2(make_float2(v4.z, v4.w), make_float2(-uhi.x, -uhi.y)));
+  }
+  V2<2> o = tree<0, RPW / 2, 2>([&](int m) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const f2 kk = dup(in.k[r0 + 2 * m + e]);
+      s[2 * m + e][0] = fma2(kk, delta[0], s[2 * m + e][0]);
+      s[2 * m + e][1] = fma2(kk, delta[1], s[2 * m + e][1]);
+    }
+    const f2 qe = dup(in.q[r0 + 2 * m]), qo = dup(in.q[r0 + 2 * m + 1]);
+    V2<2> leaf;
+    leaf.x[0] = fma2(qe, s[2 * m][0], mul2(qo, s[2 * m + 1][0]));
+    leaf.x[1] = fma2(qe, s[2 * m][1], mul2(qo, s[2 * m + 1][1]));
+    return leaf;
+  });
+  put_partial(sm.red[1][0], w, lane, o.x[0], o.x[1]);
+#pragma unroll
+  for (int rr = 0; rr < RPW; ++rr)
+    *reinterpret_cast<uint2*>(hr.pivots + (r0 + rr) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
+  __syncthreads();
+  if (w == 0) {
+    f2 lo, hi;
+    warp_tree(sm.red[1][0], lane, lo, hi);
+    *reinterpret_cast<float4*>(o_out + 4 * lane) = make_float4(lo.x, lo.y, hi.x, hi.y);
+  }
+  if (tid < 2 * D) hr.scales[tid] = 0.0f;
+}
+
+// ---------------------------------------------------------------------------------
+// stq_decode_step: persistent CTAs walking (head, request) items head-major with a
+// grid stride. Item n+1's inputs (packed codes, FP16 pivot rows, scales, q/k/v, gate,
+// row metadata) stream into the other half of a shared-memory double buffer with 1-D
+// bulk asynchronous copies completing on an mbarrier while item n is computed.
+// ---------------------------------------------------------------------------------
 __global__ void __launch_bounds__(NT, 2)
 decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* __restrict__ q,
               const float* __restrict__ k, const float* __restrict__ v,
@@ -790,93 +835,61 @@ decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* 
   __shared__ int abort_flag;
   HeadIn* ins[2] = {reinterpret_cast<HeadIn*>(dyn), reinterpret_cast<HeadIn*>(dyn + stage_stride)};
   uint8_t* stages[2] = {dyn + HEAD_IN_BYTES, dyn + stage_stride + HEAD_IN_BYTES};
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int total = B * P.H;
+  const int stride = gridDim.x;
   int item = blockIdx.x;
-  ItemMeta next_meta;
-  int stuck_n = -1;       // thread 0: iteration whose wait gave up
-  bool stuck_next = false;
+  __shared__ ItemMeta meta;   // scalars of the next item to prefetch
+  int stuck_n = -1;          // thread 0: iteration whose wait gave up
+  init_width_tables(sm);
   if (tid == 0) {
     mbar_init(&bars[0]);
     mbar_init(&bars[1]);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     abort_flag = 0;
-    if (item < total) {
-      const ItemMeta m0 = load_item_meta(P, item, slots, gate, beta);
-      issue_prefetch(P, item, m0, *ins[0], stages[0], &bars[0], q, k, v, gate);
-    }
-    if (item + int(gridDim.x) < total) next_meta = load_item_meta(P, item + gridDim.x, slots, gate, beta);
   }
   __syncthreads();
-  for (int n = 0; item < total; ++n, item += gridDim.x) {
+  if (w == 0 && item < total) {
+    start_item_meta(P, item, B, slots, gate, beta, meta, lane);
+    finish_item_meta();
+    issue_prefetch(P, item, B, meta, *ins[0], stages[0], &bars[0], q, k, v, gate, lane);
+    __syncwarp();
+    if (item + stride < total) start_item_meta(P, item + stride, B, slots, gate, beta, meta, lane);
+  }
+  for (int n = 0; item < total; ++n, item += stride) {
     const int b = n & 1;
-    const int next = item + gridDim.x;
-    HeadIn& in = *ins[b];
-    uint8_t* stage = stages[b];
-    if (tid == 0) {
-      if (next < total) {
-        // the other buffer was last read in iteration n-1, which ended with a barrier;
-        // order those generic-proxy accesses before the asynchronous writes
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        issue_prefetch(P, next, next_meta, *ins[b ^ 1], stages[b ^ 1], &bars[b ^ 1], q, k, v, gate);
-        if (next + int(gridDim.x) < total) next_meta = load_item_meta(P, next + gridDim.x, slots, gate, beta);
-      }
-      if (!mbar_wait_bounded(&bars[b], uint32_t(n >> 1) & 1u)) {
-        atomicOr(P.err, ERR_TIMEOUT);
-        abort_flag = 1;
-        stuck_n = n;
-        stuck_next = next < total;
-      }
+    const int next = item + stride;
+    if (tid == 0 && !mbar_wait_bounded(&bars[b], uint32_t(n >> 1) & 1u)) {
+      atomicOr(P.err, ERR_TIMEOUT);
+      abort_flag = 1;
+      stuck_n = n;
     }
-    __syncthreads();
+    __syncthreads();   // item n is staged; every thread is done with item n-1
     if (abort_flag) break;
+    if (w == 0 && next < total) {
+      finish_item_meta();
+      issue_prefetch(P, next, B, meta, *ins[b ^ 1], stages[b ^ 1], &bars[b ^ 1], q, k, v, gate, lane);
+      __syncwarp();
+      if (next + stride < total) start_item_meta(P, next + stride, B, slots, gate, beta, meta, lane);
+    }
+    const HeadIn& in = *ins[b];
     if (in.valid) {
-      const HeadRef hr = in.ref;
-      const uint64_t vec = uint64_t(item) * D;
-      if (tid < D) {
-        const uint32_t info = in.info[tid];
-        const int bits = row_bits(info);
-        sm.info[tid] = info;
-        if (bits == PIVOT) {
-          sm.qm[tid] = 0.0f;
-          sm.iq[tid] = 0.0f;
-          sm.mb[tid] = MAGIC;
-          sm.tb[tid] = TWO23;
-        } else {
-          const int bias = 1 << (bits - 1);
-          sm.qm[tid] = float(bias - 1);
-          sm.iq[tid] = __frcp_rn(float(bias - 1));
-          sm.mb[tid] = MAGIC + float(bias);
-          sm.tb[tid] = TWO23 + float(bias);
-        }
-        sm.k[tid] = in.k[tid];
-        sm.q[tid] = in.q[tid];
-        sm.v[tid] = in.v[tid];
-        const float dec = (P.kind == 0) ? in.gate_s : in.gate[tid];
-        sm.dec[tid] = dec;
-        sm.rd[tid] = fmul(dec, in.r[tid]);
-      }
-      if (tid == 0) sm.beta = in.beta_s;
-      const float4 c4 = *reinterpret_cast<const float4*>(&in.c[4 * lane]);
-      const f2 cin[2] = {make_float2(c4.x, c4.y), make_float2(c4.z, c4.w)};
-      __syncthreads();
-      float* o_out = out + vec;
-      switch (hr.bits) {
-        case 2: decode_head<2>(in.g, in.om, sm, stage, hr, cin, o_out); break;
-        case 4: decode_head<4>(in.g, in.om, sm, stage, hr, cin, o_out); break;
-        case 6: decode_head<6>(in.g, in.om, sm, stage, hr, cin, o_out); break;
-        case 8: decode_head<8>(in.g, in.om, sm, stage, hr, cin, o_out); break;
-        case PIVOT: decode_pivot_head(sm, stage, hr, o_out); break;
-        default: decode_head<MIXED>(in.g, in.om, sm, stage, hr, cin, o_out); break;
+      const int h = item / B, bq = item - h * B;
+      float* o_out = out + (uint64_t(bq) * P.H + h) * D;
+      switch (in.ref.bits) {
+        case 2: decode_head<2>(in, P.kind, sm, stages[b], o_out); break;
+        case 4: decode_head<4>(in, P.kind, sm, stages[b], o_out); break;
+        case 6: decode_head<6>(in, P.kind, sm, stages[b], o_out); break;
+        case 8: decode_head<8>(in, P.kind, sm, stages[b], o_out); break;
+        case PIVOT: decode_pivot_head(in, P.kind, sm, stages[b], o_out); break;
+        default: decode_head<MIXED>(in, P.kind, sm, stages[b], o_out); break;
       }
     }
-    __syncthreads();
   }
   if (tid == 0 && stuck_n >= 0) {
-    // give the loads this CTA started a bounded chance to land before its shared
-    // memory goes away: the phase that timed out and the prefetch issued after it
+    // give the loads of the phase that timed out a bounded chance to land before the
+    // CTA's shared memory goes away (no later prefetch was issued)
     mbar_wait_bounded(&bars[stuck_n & 1], uint32_t(stuck_n >> 1) & 1u);
-    if (stuck_next) mbar_wait_bounded(&bars[(stuck_n + 1) & 1], uint32_t((stuck_n + 1) >> 1) & 1u);
   }
 }
 
@@ -902,7 +915,7 @@ __device__ __forceinline__ void quantize_head(const PoolDev& P, int h, HeadSmem&
     }
   }
   f2 c[2];
-  refit_pack<BITS>(P.g + h * D, P.omega + h * D, sm, stage, s, hr.scales, c, nullptr);
+  refit_pack<BITS>(P.g + h * D, P.omega + h * D, sm.info, sm, stage, s, hr.scales, c, nullptr);
   __syncthreads();
   copy16(hr.codes, stage, hr.code_bytes);
   if (w == 0) *reinterpret_cast<float4*>(hr.scales + D + 4 * lane) = make_float4(c[0].x, c[0].y, c[1].x, c[1].y);
@@ -922,6 +935,7 @@ quantize_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float
   }
   const HeadRef hr = head_ref(P, slot, h);
   load_row_meta(P, h, sm);
+  init_width_tables(sm);
   __syncthreads();
   const float* src = S + uint64_t(item) * D * D;
   switch (hr.bits) {
