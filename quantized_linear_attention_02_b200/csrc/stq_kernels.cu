@@ -479,7 +479,7 @@ __device__ __forceinline__ void restore_row(const uint8_t* row, int lane, float 
 }
 
 // ---------------------------------------------------------------------------------
-// Staged inputs of one (request, head) and the asynchronous-copy helpers.
+// Staged inputs of one (request, head) in shared memory.
 // ---------------------------------------------------------------------------------
 struct __align__(16) HeadIn {
   float k[D], q[D], v[D];
@@ -494,152 +494,6 @@ struct __align__(16) HeadIn {
 };
 constexpr int HEAD_IN_BYTES = int(sizeof(HeadIn));
 static_assert(HEAD_IN_BYTES % 16 == 0, "staging sections must stay 16-byte aligned");
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
-               : "memory");
-}
-
-// Global -> shared bulk copy (bytes and both addresses multiples of 16), completing on bar.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-// Wait for a phase of bar, giving up after about two seconds.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  for (;;) {
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > 2000000000ull) return false;
-  }
-}
-
-// Scalars of one item (slot index, head record, GDN gate, beta). Lanes 0..7 of warp 0
-// fetch them into shared memory with 4-byte asynchronous copies an iteration before
-// they are needed, so that no register holds them across an item's compute.
-struct ItemMeta {
-  int slot;
-  uint32_t code_off, code_bytes, piv_first, piv_count, bits;
-  float gate_s, beta_s;
-};
-
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
-}
-
-__device__ __forceinline__ void start_item_meta(const PoolDev& P, int item, int B,
-                                                const int32_t* __restrict__ slots,
-                                                const float* __restrict__ gate,
-                                                const float* __restrict__ beta, ItemMeta& m,
-                                                int lane) {
-  const int h = item / B, bq = item - h * B;   // items run head-major: same width in a row
-  const int vi = bq * P.H + h;
-  switch (lane) {
-    case 0: cp_async4(&m.slot, slots + bq); break;
-    case 1: cp_async4(&m.code_off, P.head_code_off + h); break;
-    case 2: cp_async4(&m.code_bytes, P.head_code_bytes + h); break;
-    case 3: cp_async4(&m.piv_first, P.head_piv_first + h); break;
-    case 4: cp_async4(&m.piv_count, P.head_piv_count + h); break;
-    case 5: cp_async4(&m.bits, P.head_bits + h); break;
-    case 6: if (P.kind == 0) cp_async4(&m.gate_s, gate + vi); break;
-    case 7: cp_async4(&m.beta_s, beta + vi); break;
-    default: break;
-  }
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-// Wait for this warp's outstanding 4-byte copies, then make them visible warp-wide.
-__device__ __forceinline__ void finish_item_meta() {
-  asm volatile("cp.async.wait_all;" ::: "memory");
-  __syncwarp();
-}
-
-// Warp 0: start loading item `item` into buffer `in` (+ its staging area). Lane 0 sets
-// the expected byte count, then the lanes issue the copies side by side.
-__device__ __forceinline__ void issue_prefetch(const PoolDev& P, int item, int B, const ItemMeta m,
-                                               HeadIn& in, uint8_t* stage, uint64_t* bar,
-                                               const float* __restrict__ q,
-                                               const float* __restrict__ k,
-                                               const float* __restrict__ v,
-                                               const float* __restrict__ gate, int lane) {
-  const int h = item / B, bq = item - h * B;
-  const bool ok = m.slot >= 0 && m.slot < P.n_slots;
-  if (!ok) {
-    if (lane == 0) {
-      atomicOr(P.err, ERR_SLOT_RANGE);
-      in.valid = 0;
-      in.gate_s = m.gate_s;
-      in.beta_s = m.beta_s;
-      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-    }
-    return;
-  }
-  HeadRef hr;
-  hr.code_bytes = int(m.code_bytes);
-  hr.piv_count = int(m.piv_count);
-  hr.bits = int(m.bits);
-  hr.codes = P.codes + uint64_t(m.slot) * P.slot_code_bytes + m.code_off;
-  hr.pivots = P.pivots + (uint64_t(m.slot) * P.n_pivot_rows + m.piv_first) * D;
-  hr.scales = P.scales + (uint64_t(m.slot) * P.H + h) * 2 * D;
-  hr.piv_stage_off = hr.code_bytes;
-  const uint64_t vec = (uint64_t(bq) * P.H + h) * D;
-  if (lane == 0) {
-    in.valid = 1;
-    in.ref = hr;
-    in.gate_s = m.gate_s;
-    in.beta_s = m.beta_s;
-    uint32_t bytes = 3 * D * 4 + 2 * D * 4 + 3 * D * 4;
-    if (P.kind != 0) bytes += D * 4;
-    bytes += m.code_bytes + m.piv_count * D * 2;
-    mbar_expect_tx(bar, bytes);
-  }
-  __syncwarp();
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  switch (lane) {
-    case 0: bulk_load(in.k, k + vec, D * 4, bar); break;
-    case 1: bulk_load(in.q, q + vec, D * 4, bar); break;
-    case 2: bulk_load(in.v, v + vec, D * 4, bar); break;
-    case 3: if (P.kind != 0) bulk_load(in.gate, gate + vec, D * 4, bar); break;
-    case 4: bulk_load(in.r, hr.scales, 2 * D * 4, bar); break;
-    case 5: bulk_load(in.g, P.g + h * D, D * 4, bar); break;
-    case 6: bulk_load(in.om, P.omega + h * D, D * 4, bar); break;
-    case 7: bulk_load(in.info, P.row_info + h * D, D * 4, bar); break;
-    case 8: if (m.code_bytes) bulk_load(stage, hr.codes, m.code_bytes, bar); break;
-    case 9: if (m.piv_count) bulk_load(stage + m.code_bytes, hr.pivots, m.piv_count * D * 2, bar); break;
-    default: break;
-  }
-}
 
 // ---------------------------------------------------------------------------------
 // One (request, head) of stq_decode_step, reading its staged inputs `in`.
@@ -819,77 +673,57 @@ __device__ __forceinline__ void decode_pivot_head(const HeadIn& in, int kind, He
 }
 
 // ---------------------------------------------------------------------------------
-// stq_decode_step: persistent CTAs walking (head, request) items head-major with a
-// grid stride. Item n+1's inputs (packed codes, FP16 pivot rows, scales, q/k/v, gate,
-// row metadata) stream into the other half of a shared-memory double buffer with 1-D
-// bulk asynchronous copies completing on an mbarrier while item n is computed.
+// stq_decode_step: one CTA per (head, request) item, items numbered head-major so that
+// the CTAs resident on an SM at the same time mostly run the same width's code path.
 // ---------------------------------------------------------------------------------
 __global__ void __launch_bounds__(NT, 2)
 decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* __restrict__ q,
               const float* __restrict__ k, const float* __restrict__ v,
               const float* __restrict__ gate, const float* __restrict__ beta,
-              float* __restrict__ out, int stage_stride) {
+              float* __restrict__ out) {
   extern __shared__ __align__(16) uint8_t dyn[];
   __shared__ HeadSmem sm;
-  __shared__ __align__(8) uint64_t bars[2];
-  __shared__ int abort_flag;
-  HeadIn* ins[2] = {reinterpret_cast<HeadIn*>(dyn), reinterpret_cast<HeadIn*>(dyn + stage_stride)};
-  uint8_t* stages[2] = {dyn + HEAD_IN_BYTES, dyn + stage_stride + HEAD_IN_BYTES};
-  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  const int total = B * P.H;
-  const int stride = gridDim.x;
-  int item = blockIdx.x;
-  __shared__ ItemMeta meta;   // scalars of the next item to prefetch
-  int stuck_n = -1;          // thread 0: iteration whose wait gave up
+  HeadIn& in = *reinterpret_cast<HeadIn*>(dyn);
+  uint8_t* stage = dyn + HEAD_IN_BYTES;
+  const int tid = threadIdx.x;
+  const int h = blockIdx.x / B, bq = blockIdx.x - h * B;
+  const int slot = slots[bq];
+  if (slot < 0 || slot >= P.n_slots) {
+    if (tid == 0) atomicOr(P.err, ERR_SLOT_RANGE);
+    return;
+  }
+  const HeadRef hr = head_ref(P, slot, h);
+  const int vi = bq * P.H + h;
+  const uint64_t vec = uint64_t(vi) * D;
   init_width_tables(sm);
+  if (tid < D) {
+    in.k[tid] = k[vec + tid];
+    in.q[tid] = q[vec + tid];
+    in.v[tid] = v[vec + tid];
+    if (P.kind != 0) in.gate[tid] = gate[vec + tid];
+    in.r[tid] = hr.scales[tid];
+    in.c[tid] = hr.scales[D + tid];
+    in.g[tid] = P.g[h * D + tid];
+    in.om[tid] = P.omega[h * D + tid];
+    in.info[tid] = P.row_info[h * D + tid];
+  }
   if (tid == 0) {
-    mbar_init(&bars[0]);
-    mbar_init(&bars[1]);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    abort_flag = 0;
+    in.ref = hr;
+    in.gate_s = (P.kind == 0) ? gate[vi] : 0.0f;
+    in.beta_s = beta[vi];
+    in.valid = 1;
   }
+  copy16(stage, hr.codes, hr.code_bytes);
+  copy16(stage + hr.piv_stage_off, hr.pivots, hr.piv_count * D * 2);
   __syncthreads();
-  if (w == 0 && item < total) {
-    start_item_meta(P, item, B, slots, gate, beta, meta, lane);
-    finish_item_meta();
-    issue_prefetch(P, item, B, meta, *ins[0], stages[0], &bars[0], q, k, v, gate, lane);
-    __syncwarp();
-    if (item + stride < total) start_item_meta(P, item + stride, B, slots, gate, beta, meta, lane);
-  }
-  for (int n = 0; item < total; ++n, item += stride) {
-    const int b = n & 1;
-    const int next = item + stride;
-    if (tid == 0 && !mbar_wait_bounded(&bars[b], uint32_t(n >> 1) & 1u)) {
-      atomicOr(P.err, ERR_TIMEOUT);
-      abort_flag = 1;
-      stuck_n = n;
-    }
-    __syncthreads();   // item n is staged; every thread is done with item n-1
-    if (abort_flag) break;
-    if (w == 0 && next < total) {
-      finish_item_meta();
-      issue_prefetch(P, next, B, meta, *ins[b ^ 1], stages[b ^ 1], &bars[b ^ 1], q, k, v, gate, lane);
-      __syncwarp();
-      if (next + stride < total) start_item_meta(P, next + stride, B, slots, gate, beta, meta, lane);
-    }
-    const HeadIn& in = *ins[b];
-    if (in.valid) {
-      const int h = item / B, bq = item - h * B;
-      float* o_out = out + (uint64_t(bq) * P.H + h) * D;
-      switch (in.ref.bits) {
-        case 2: decode_head<2>(in, P.kind, sm, stages[b], o_out); break;
-        case 4: decode_head<4>(in, P.kind, sm, stages[b], o_out); break;
-        case 6: decode_head<6>(in, P.kind, sm, stages[b], o_out); break;
-        case 8: decode_head<8>(in, P.kind, sm, stages[b], o_out); break;
-        case PIVOT: decode_pivot_head(in, P.kind, sm, stages[b], o_out); break;
-        default: decode_head<MIXED>(in, P.kind, sm, stages[b], o_out); break;
-      }
-    }
-  }
-  if (tid == 0 && stuck_n >= 0) {
-    // give the loads of the phase that timed out a bounded chance to land before the
-    // CTA's shared memory goes away (no later prefetch was issued)
-    mbar_wait_bounded(&bars[stuck_n & 1], uint32_t(stuck_n >> 1) & 1u);
+  float* o_out = out + vec;
+  switch (hr.bits) {
+    case 2: decode_head<2>(in, P.kind, sm, stage, o_out); break;
+    case 4: decode_head<4>(in, P.kind, sm, stage, o_out); break;
+    case 6: decode_head<6>(in, P.kind, sm, stage, o_out); break;
+    case 8: decode_head<8>(in, P.kind, sm, stage, o_out); break;
+    case PIVOT: decode_pivot_head(in, P.kind, sm, stage, o_out); break;
+    default: decode_head<MIXED>(in, P.kind, sm, stage, o_out); break;
   }
 }
 
@@ -1111,18 +945,10 @@ cudaError_t launch_decode(const PoolDev& P, const int32_t* slots, int B, const f
                           const float* k, const float* v, const float* gate,
                           const float* beta, float* out, cudaStream_t s) {
   if (B == 0) return cudaSuccess;
-  const int stride = HEAD_IN_BYTES + stage_bytes(P);
-  const int dyn = 2 * stride;
-  cudaError_t e = prepare(decode_kernel, dyn, int(sizeof(HeadSmem)) + 64, g_decode_dyn);
+  const int dyn = HEAD_IN_BYTES + stage_bytes(P);
+  cudaError_t e = prepare(decode_kernel, dyn, int(sizeof(HeadSmem)), g_decode_dyn);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 0;
-  e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
-  const long long items = (long long)B * P.H;
-  const int grid = int(items < 2LL * sms ? items : 2LL * sms);
-  decode_kernel<<<grid, NT, dyn, s>>>(P, slots, B, q, k, v, gate, beta, out, stride);
+  decode_kernel<<<B * P.H, NT, dyn, s>>>(P, slots, B, q, k, v, gate, beta, out);
   return cudaGetLastError();
 }
 
