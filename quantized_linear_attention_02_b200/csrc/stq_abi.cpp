@@ -45,6 +45,7 @@ size_t up16(size_t x) { return (x + 15) & ~size_t(15); }
 struct HostLayout {
   int kind = 0, n_slots = 0, H = 0;
   std::vector<uint32_t> head_code_off, head_code_bytes, head_piv_first, head_piv_count, head_bits;
+  std::vector<uint32_t> warp_code_off;
   std::vector<uint32_t> row_info;
   std::vector<float> g, omega;
   uint64_t slot_code_bytes = 0;
@@ -71,6 +72,7 @@ stq_status build_layout(const stq_pool_desc* desc, HostLayout& L) {
   L.head_piv_count.assign(H, 0);
   L.head_bits.assign(H, 0);
   L.row_info.assign(size_t(H) * D, 0);
+  L.warp_code_off.assign(size_t(H) * 8, 0);
   L.g.assign(size_t(H) * D, 0.0f);
   L.omega.assign(size_t(H) * D, 0.0f);
   uint64_t off = 0;
@@ -97,6 +99,7 @@ stq_status build_layout(const stq_pool_desc* desc, HostLayout& L) {
       const int b = (desc->kind == STQ_GDN) ? desc->unit_bits[h] : desc->unit_bits[size_t(h) * D + i];
       if (b != 2 && b != 4 && b != 6 && b != 8 && b != STQ_PIVOT_BITS)
         return fail(STQ_ERR_INVALID_ARG, "unit width %d (head %d row %d) not in {2,4,6,8,16}", b, h, i);
+      if (i % 16 == 0) L.warp_code_off[size_t(h) * 8 + i / 16] = in_head;
       if (b == STQ_PIVOT_BITS) {
         L.row_info[size_t(h) * D + i] = uint32_t(b) | (piv_in_head << 8);
         ++piv_in_head;
@@ -133,6 +136,7 @@ MetaLayout meta_layout(int H) {
   m.head_piv_first = o;  o = up16(o + size_t(H) * 4);
   m.head_piv_count = o;  o = up16(o + size_t(H) * 4);
   m.head_bits = o;       o = up16(o + size_t(H) * 4);
+  m.warp_code_off = o;   o = up16(o + size_t(H) * 8 * 4);
   m.row_info = o;        o = up16(o + size_t(H) * D * 4);
   m.g = o;               o = up16(o + size_t(H) * D * 4);
   m.omega = o;           o = up16(o + size_t(H) * D * 4);
@@ -207,6 +211,7 @@ stq_status stq_pool_create(const stq_pool_desc* desc, void* d_codes, void* d_sca
   put(m.head_piv_first, L.head_piv_first.data(), L.H * 4);
   put(m.head_piv_count, L.head_piv_count.data(), L.H * 4);
   put(m.head_bits, L.head_bits.data(), L.H * 4);
+  put(m.warp_code_off, L.warp_code_off.data(), L.warp_code_off.size() * 4);
   put(m.row_info, L.row_info.data(), L.row_info.size() * 4);
   put(m.g, L.g.data(), L.g.size() * 4);
   put(m.omega, L.omega.data(), L.omega.size() * 4);
@@ -228,6 +233,7 @@ stq_status stq_pool_create(const stq_pool_desc* desc, void* d_codes, void* d_sca
   dv.head_piv_first = reinterpret_cast<const uint32_t*>(mb + m.head_piv_first);
   dv.head_piv_count = reinterpret_cast<const uint32_t*>(mb + m.head_piv_count);
   dv.head_bits = reinterpret_cast<const uint32_t*>(mb + m.head_bits);
+  dv.warp_code_off = reinterpret_cast<const uint32_t*>(mb + m.warp_code_off);
   dv.row_info = reinterpret_cast<const uint32_t*>(mb + m.row_info);
   dv.g = reinterpret_cast<const float*>(mb + m.g);
   dv.omega = reinterpret_cast<const float*>(mb + m.omega);

@@ -37,6 +37,7 @@ struct PoolDev {
   const uint32_t* head_piv_count;   // [H]
   const uint32_t* head_bits;        // [H] the width shared by all rows of head h
                                     //   (2/4/6/8, or 16 if all rows are pivots), 0 if mixed
+  const uint32_t* warp_code_off;    // [H*8] byte offset in head h where rows 16w.. start
   const uint32_t* row_info;         // [H*D] bits (low 8) | byte offset in head << 8
                                     //   (pivot rows: index in head's pivot block << 8)
   const float* g;                   // [H*D] row gain (omega_i / mean omega)^(-1/2)
@@ -47,7 +48,7 @@ struct PoolDev {
 // Byte layout of the meta buffer, computed on the host.
 struct MetaLayout {
   size_t head_code_off, head_code_bytes, head_piv_first, head_piv_count, head_bits;
-  size_t row_info, g, omega, err, total;
+  size_t warp_code_off, row_info, g, omega, err, total;
 };
 
 MetaLayout meta_layout(int H);

@@ -25,6 +25,7 @@
 //     clamping is done in that binade, where the low bits are the (biased) code.
 #include <cuda_fp16.h>
 
+#include "stq_fastdiv.cuh"
 #include "stq_internal.h"
 
 namespace stq {
@@ -50,13 +51,10 @@ __device__ __forceinline__ f2 mul2(f2 a, f2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ f2 add2(f2 a, f2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ f2 dup(float x) { return make_float2(x, x); }
-__device__ __forceinline__ float at4(const float4& v, int i) {
-  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
-}
 
 // 1/a correctly rounded for a >= 2^-126; 0 for a smaller (or zero) scale.
 __device__ __forceinline__ float recip_scale(float a) {
-  return a >= SMALLEST_NORMAL ? __frcp_rn(a) : 0.0f;
+  return a >= SMALLEST_NORMAL ? rcp_rn(a) : 0.0f;
 }
 
 template <int N>
@@ -76,31 +74,6 @@ __device__ __forceinline__ V2<M> tree(F&& f) {
 #pragma unroll
     for (int m = 0; m < M; ++m) a.x[m] = add2(a.x[m], b.x[m]);
     return a;
-  }
-}
-
-struct __align__(16) HeadSmem {
-  float inv_r[D];    // 1/r_i of the refit
-  float b[D];        // omega_i * r_i^2
-  uint32_t info[D];  // bits | offset << 8 (quantiser path)
-  // per-width constants, indexed by the width (2/4/6/8; 16 = pivot row, others unused)
-  float tqm[32];     // qmax = 2^(b-1) - 1 (0 for pivots)
-  float tiq[32];     // 1/qmax (0 for pivots)
-  float tmb[32];     // 1.5*2^23 + 2^(b-1): magic that yields the biased code
-  float ttb[32];     // 2^23 + 2^(b-1): magic that turns a code into its value
-  float4 red[2][2][NW][D / 4];  // ping-pong partials: [buffer][quantity][warp][col/4]
-};
-
-// Fill the per-width tables (threads 0..31).
-__device__ __forceinline__ void init_width_tables(HeadSmem& sm) {
-  const int bits = threadIdx.x;
-  if (bits < 32) {
-    const bool q = bits == 2 || bits == 4 || bits == 6 || bits == 8;
-    const int bias = q ? (1 << (bits - 1)) : 0;
-    sm.tqm[bits] = q ? float(bias - 1) : 0.0f;
-    sm.tiq[bits] = q ? __frcp_rn(float(bias - 1)) : 0.0f;
-    sm.tmb[bits] = MAGIC + float(bias);
-    sm.ttb[bits] = TWO23 + float(bias);
   }
 }
 
@@ -199,12 +172,6 @@ __device__ __forceinline__ HeadRef head_ref(const PoolDev& P, int slot, int h) {
   return r;
 }
 
-// Row widths and offsets of head h into shared memory (threads 0..127, one row each).
-__device__ __forceinline__ void load_row_meta(const PoolDev& P, int h, HeadSmem& sm) {
-  const int i = threadIdx.x;
-  if (i < D) sm.info[i] = P.row_info[h * D + i];
-}
-
 __device__ __forceinline__ uint2 half4_bits(f2 a, f2 b) {
   const uint32_t lo = uint32_t(__half_as_ushort(__float2half_rn(a.x))) |
                       (uint32_t(__half_as_ushort(__float2half_rn(a.y))) << 16);
@@ -238,19 +205,94 @@ __device__ __forceinline__ void put_partial(float4 (*red)[D / 4], int w, int lan
   red[w][lane] = make_float4(lo.x, lo.y, hi.x, hi.y);
 }
 
+// Restore one row of S' = D (r c Q) for this lane's 4 columns.
+template <int BITS>
+__device__ __forceinline__ void restore_row(const uint8_t* row, int lane, float rd, float tb,
+                                            const f2 (&cin)[2], f2& s01, f2& s23) {
+  uint32_t cd[4];
+  load_codes<BITS>(row, lane, cd);
+  const f2 ntb = dup(-tb);
+  const f2 q01 = add2(make_float2(__uint_as_float(cd[0]), __uint_as_float(cd[1])), ntb);
+  const f2 q23 = add2(make_float2(__uint_as_float(cd[2]), __uint_as_float(cd[3])), ntb);
+  s01 = mul2(mul2(q01, dup(rd)), cin[0]);
+  s23 = mul2(mul2(q23, dup(rd)), cin[1]);
+}
+
 // ---------------------------------------------------------------------------------
-// Refit: row scale, column scale start, two omega-weighted least-squares steps, final
-// codes (bloombook section 4; singularity-lens dual-axis paragraph). On entry s[][]
-// holds the float32 state (pivot rows already stored) and the caller may have put
-// readout partials into red[1][0]. On exit the head's packed codes are in `stage`,
-// r has been written to global, and c is returned in c_out (this lane's columns).
-// BITS is the head's uniform width, or MIXED for per-row widths.
+// Shared memory. Each warp stages and uses only its own 16 key rows (WarpRows), so the
+// only CTA-wide synchronisation is the exchange of column partial sums (red).
+// ---------------------------------------------------------------------------------
+struct __align__(16) WarpRows {
+  f2 kk[RPW], qq[RPW], rdd[RPW];   // (k_i, k_i), (q_i, q_i), (dec_i r_i, dec_i r_i)
+  f2 irr[RPW], bb[RPW];            // refit: (1/r_i, 1/r_i), (omega_i r_i^2, same)
+  float dec[RPW];                  // row retention
+  float g[RPW], om[RPW];           // row gain and omega
+  float qm[RPW], iq[RPW], mb[RPW], tb[RPW];   // per-row width constants (mixed heads)
+  uint32_t info[RPW];              // bits | offset << 8
+  uint8_t codes[RPW * D];          // this warp's rows of packed codes
+};
+
+struct __align__(16) CtaSmem {
+  float4 red[2][2][NW][D / 4];     // ping-pong partials: [buffer][quantity][warp][col/4]
+  WarpRows wr[NW];
+};
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+
+// Per-row constants of a width (2/4/6/8, 16 = pivot).
+__device__ __forceinline__ void width_consts(int bits, float& qm, float& iq, float& mb, float& tb) {
+  if (bits == PIVOT) {
+    qm = 0.0f; iq = 0.0f; mb = MAGIC; tb = TWO23;
+  } else {
+    const int bias = 1 << (bits - 1);
+    qm = float(bias - 1);
+    iq = __frcp_rn(qm);
+    mb = MAGIC + float(bias);
+    tb = TWO23 + float(bias);
+  }
+}
+
+// Lanes 0..15 of warp w: the per-row data of rows 16w..16w+15 of head h.
+__device__ __forceinline__ void load_warp_rows(const PoolDev& P, int h, WarpRows& wr, int lane, int r0,
+                                               const float* k_vec, const float* q_vec, const float* r_in,
+                                               const float* gate_rows, float gate_s) {
+  if (lane < RPW) {
+    const int i = r0 + lane;
+    const uint32_t info = P.row_info[h * D + i];
+    wr.info[lane] = info;
+    wr.g[lane] = P.g[h * D + i];
+    wr.om[lane] = P.omega[h * D + i];
+    float qm, iq, mb, tb;
+    width_consts(row_bits(info), qm, iq, mb, tb);
+    wr.qm[lane] = qm; wr.iq[lane] = iq; wr.mb[lane] = mb; wr.tb[lane] = tb;
+    if (k_vec != nullptr) {
+      const float dec = gate_rows != nullptr ? gate_rows[i] : gate_s;
+      const float kv = k_vec[i], qv = q_vec[i];
+      const float rd = fmul(dec, r_in[i]);
+      wr.dec[lane] = dec;
+      wr.kk[lane] = make_float2(kv, kv);
+      wr.qq[lane] = make_float2(qv, qv);
+      wr.rdd[lane] = make_float2(rd, rd);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// Refit of this warp's rows: row scale, column scale start, two omega-weighted
+// least-squares steps, final codes (bloombook section 4; singularity-lens dual-axis
+// paragraph). On entry s[][] holds the float32 state (pivot rows already stored) and the
+// caller may have put readout partials into red[1][0]. The codes go straight to the
+// pool; r of this warp's rows is written; c (this lane's columns) is returned.
+// Four CTA barriers: column maximum, step one, step two (and the caller's u exchange).
 // ---------------------------------------------------------------------------------
 template <int BITS>
-__device__ __forceinline__ void refit_pack(const float* g_row, const float* om_row,
-                                           const uint32_t* info_row, HeadSmem& sm,
-                                           uint8_t* stage, f2 (&s)[RPW][2], float* r_global,
-                                           f2 (&c_out)[2], float* o_global) {
+__device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], float* r_global,
+                                            uint8_t* codes_global, int warp_code_start, f2 (&c_out)[2],
+                                            float* o_global) {
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r0 = w * RPW;
 
@@ -291,15 +333,13 @@ __device__ __forceinline__ void refit_pack(const float* g_row, const float* om_r
   {
     // lane l now holds the sum of row R(l): bits 0..3 of l chose halves 8, 4, 2, 1
     const int R = ((lane & 1) << 3) | ((lane & 2) << 1) | ((lane & 4) >> 1) | ((lane & 8) >> 3);
-    const int i = r0 + R;
-    const bool pivot = (BITS == MIXED) ? (row_bits(info_row[i]) == PIVOT) : false;
-    const float g = g_row[i];
-    const float om = om_row[i];
-    const float r = pivot ? 0.0f : fmul(fmul(a[0], 0.0078125f), g);
+    const bool pivot = (BITS == MIXED) ? (row_bits(wr.info[R]) == PIVOT) : false;
+    const float r = pivot ? 0.0f : fmul(fmul(a[0], 0.0078125f), wr.g[R]);
     if (lane < 16) {
-      sm.inv_r[i] = recip_scale(r);
-      sm.b[i] = fmul(om, fmul(r, r));
-      r_global[i] = r;
+      const float ir = recip_scale(r), bv = fmul(wr.om[R], fmul(r, r));
+      wr.irr[R] = make_float2(ir, ir);
+      wr.bb[R] = make_float2(bv, bv);
+      r_global[r0 + R] = r;
     }
   }
   __syncwarp();
@@ -307,40 +347,29 @@ __device__ __forceinline__ void refit_pack(const float* g_row, const float* om_r
   // --- y = S * inv_r; column start c0_j = max_i |y_ij| / qmax_i -----------------------
   float mx[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-  for (int g4 = 0; g4 < RPW / 4; ++g4) {
-    const float4 ir4 = *reinterpret_cast<const float4*>(&sm.inv_r[r0 + 4 * g4]);
-    float4 iq4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int rr = 0; rr < RPW; ++rr) {
+    const f2 ir = wr.irr[rr];
+    s[rr][0] = mul2(s[rr][0], ir);
+    s[rr][1] = mul2(s[rr][1], ir);
     if constexpr (BITS == MIXED) {
-      const uint4 in4 = *reinterpret_cast<const uint4*>(&info_row[r0 + 4 * g4]);
-      iq4 = make_float4(sm.tiq[row_bits(in4.x)], sm.tiq[row_bits(in4.y)], sm.tiq[row_bits(in4.z)],
-                        sm.tiq[row_bits(in4.w)]);
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int rr = 4 * g4 + j;
-      const f2 ir = dup(at4(ir4, j));
-      s[rr][0] = mul2(s[rr][0], ir);
-      s[rr][1] = mul2(s[rr][1], ir);
-      if constexpr (BITS == MIXED) {
-        const float iq = at4(iq4, j);
-        mx[0] = fmaxf(mx[0], fmul(fabsf(s[rr][0].x), iq));
-        mx[1] = fmaxf(mx[1], fmul(fabsf(s[rr][0].y), iq));
-        mx[2] = fmaxf(mx[2], fmul(fabsf(s[rr][1].x), iq));
-        mx[3] = fmaxf(mx[3], fmul(fabsf(s[rr][1].y), iq));
-      } else {
-        mx[0] = fmaxf(mx[0], fabsf(s[rr][0].x));
-        mx[1] = fmaxf(mx[1], fabsf(s[rr][0].y));
-        mx[2] = fmaxf(mx[2], fabsf(s[rr][1].x));
-        mx[3] = fmaxf(mx[3], fabsf(s[rr][1].y));
-      }
+      const float iq = wr.iq[rr];
+      mx[0] = fmaxf(mx[0], fmul(fabsf(s[rr][0].x), iq));
+      mx[1] = fmaxf(mx[1], fmul(fabsf(s[rr][0].y), iq));
+      mx[2] = fmaxf(mx[2], fmul(fabsf(s[rr][1].x), iq));
+      mx[3] = fmaxf(mx[3], fmul(fabsf(s[rr][1].y), iq));
+    } else {
+      mx[0] = fmaxf(mx[0], fabsf(s[rr][0].x));
+      mx[1] = fmaxf(mx[1], fabsf(s[rr][0].y));
+      mx[2] = fmaxf(mx[2], fabsf(s[rr][1].x));
+      mx[3] = fmaxf(mx[3], fabsf(s[rr][1].y));
     }
   }
-  sm.red[1][1][w][lane] = make_float4(mx[0], mx[1], mx[2], mx[3]);
+  cs.red[1][1][w][lane] = make_float4(mx[0], mx[1], mx[2], mx[3]);
   __syncthreads();
 
   if (o_global != nullptr && w == 0) {
     f2 lo, hi;
-    warp_tree(sm.red[1][0], lane, lo, hi);
+    warp_tree(cs.red[1][0], lane, lo, hi);
     *reinterpret_cast<float4*>(o_global + 4 * lane) = make_float4(lo.x, lo.y, hi.x, hi.y);
   }
   f2 c[2];
@@ -348,7 +377,7 @@ __device__ __forceinline__ void refit_pack(const float* g_row, const float* om_r
     float m[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
     for (int ww = 0; ww < NW; ++ww) {
-      const float4 v = sm.red[1][1][ww][lane];
+      const float4 v = cs.red[1][1][ww][lane];
       m[0] = fmaxf(m[0], v.x); m[1] = fmaxf(m[1], v.y); m[2] = fmaxf(m[2], v.z); m[3] = fmaxf(m[3], v.w);
     }
     if constexpr (BITS != MIXED) {
@@ -367,26 +396,17 @@ __device__ __forceinline__ void refit_pack(const float* g_row, const float* om_r
   for (int it = 0; it < 2; ++it) {
     const f2 ic[2] = {make_float2(recip_scale(c[0].x), recip_scale(c[0].y)),
                       make_float2(recip_scale(c[1].x), recip_scale(c[1].y))};
-    float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f), q4 = b4;
     V2<4> nd = tree<0, RPW / 2, 4>([&](int m) {
       // rows 2m and 2m+1 form one fused pair of each sum
-      if ((m & 1) == 0) {
-        b4 = *reinterpret_cast<const float4*>(&sm.b[r0 + 2 * m]);
-        if constexpr (BITS == MIXED) {
-          const uint4 in4 = *reinterpret_cast<const uint4*>(&info_row[r0 + 2 * m]);
-          q4 = make_float4(sm.tqm[row_bits(in4.x)], sm.tqm[row_bits(in4.y)], sm.tqm[row_bits(in4.z)],
-                           sm.tqm[row_bits(in4.w)]);
-        }
-      }
       f2 Q[2][2], p[2][2];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int rr = 2 * m + e;
-        const f2 bb = dup(at4(b4, rr & 3));
+        const f2 bb = wr.bb[rr];
         float lo_b, hi_b;
         if constexpr (BITS == MIXED) {
-          lo_b = MAGIC - at4(q4, rr & 3);
-          hi_b = MAGIC + at4(q4, rr & 3);
+          lo_b = MAGIC - wr.qm[rr];
+          hi_b = MAGIC + wr.qm[rr];
         } else {
           lo_b = MAGIC - float((1 << (BITS - 1)) - 1);
           hi_b = MAGIC + float((1 << (BITS - 1)) - 1);
@@ -410,31 +430,30 @@ __device__ __forceinline__ void refit_pack(const float* g_row, const float* om_r
       }
       return leaf;
     });
-    float4 (*const num)[D / 4] = sm.red[it][0];
-    float4 (*const den)[D / 4] = sm.red[it][1];
+    float4 (*const num)[D / 4] = cs.red[it][0];
+    float4 (*const den)[D / 4] = cs.red[it][1];
     put_partial(num, w, lane, nd.x[0], nd.x[1]);
     put_partial(den, w, lane, nd.x[2], nd.x[3]);
     __syncthreads();
     f2 nlo, nhi, dlo, dhi;
     warp_tree(num, lane, nlo, nhi);
     warp_tree(den, lane, dlo, dhi);
-    if (dlo.x > 0.0f) c[0].x = __fdiv_rn(nlo.x, dlo.x);
-    if (dlo.y > 0.0f) c[0].y = __fdiv_rn(nlo.y, dlo.y);
-    if (dhi.x > 0.0f) c[1].x = __fdiv_rn(nhi.x, dhi.x);
-    if (dhi.y > 0.0f) c[1].y = __fdiv_rn(nhi.y, dhi.y);
+    if (dlo.x > 0.0f) c[0].x = div_rn(nlo.x, dlo.x);
+    if (dlo.y > 0.0f) c[0].y = div_rn(nlo.y, dlo.y);
+    if (dhi.x > 0.0f) c[1].x = div_rn(nhi.x, dhi.x);
+    if (dhi.y > 0.0f) c[1].y = div_rn(nhi.y, dhi.y);
   }
 
-  // --- final codes with the final c, packed into the staging buffer --------------------
+  // --- final codes with the final c, stored straight into the pool -------------------
   const f2 ic[2] = {make_float2(recip_scale(c[0].x), recip_scale(c[0].y)),
                     make_float2(recip_scale(c[1].x), recip_scale(c[1].y))};
 #pragma unroll
   for (int rr = 0; rr < RPW; ++rr) {
-    const int i = r0 + rr;
     if constexpr (BITS == MIXED) {
-      const uint32_t info = info_row[i];
+      const uint32_t info = wr.info[rr];
       const int bits = row_bits(info);
       if (bits == PIVOT) continue;
-      const float mb = sm.tmb[bits], q = sm.tqm[bits];
+      const float mb = wr.mb[rr], q = wr.qm[rr];
       const f2 t01 = fma2(s[rr][0], ic[0], dup(mb));
       const f2 t23 = fma2(s[rr][1], ic[1], dup(mb));
       const float lo_b = mb - q, hi_b = mb + q;
@@ -442,7 +461,7 @@ __device__ __forceinline__ void refit_pack(const float* g_row, const float* om_r
                              __float_as_uint(fminf(fmaxf(t01.y, lo_b), hi_b)),
                              __float_as_uint(fminf(fmaxf(t23.x, lo_b), hi_b)),
                              __float_as_uint(fminf(fmaxf(t23.y, lo_b), hi_b))};
-      uint8_t* row = stage + row_off(info);
+      uint8_t* row = codes_global + row_off(info);
       switch (bits) {
         case 2: store_codes<2>(row, lane, t); break;
         case 4: store_codes<4>(row, lane, t); break;
@@ -458,107 +477,65 @@ __device__ __forceinline__ void refit_pack(const float* g_row, const float* om_r
                              __float_as_uint(fminf(fmaxf(t01.y, MB - QM), MB + QM)),
                              __float_as_uint(fminf(fmaxf(t23.x, MB - QM), MB + QM)),
                              __float_as_uint(fminf(fmaxf(t23.y, MB - QM), MB + QM))};
-      store_codes<BITS>(stage + rr * (D * BITS / 8) + r0 * (D * BITS / 8), lane, t);
+      store_codes<BITS>(codes_global + warp_code_start + rr * (D * BITS / 8), lane, t);
     }
   }
   c_out[0] = c[0];
   c_out[1] = c[1];
 }
 
-// Restore one row of S' = D (r c Q) for this lane's 4 columns.
-template <int BITS>
-__device__ __forceinline__ void restore_row(const uint8_t* row, int lane, float rd, float tb,
-                                            const f2 (&cin)[2], f2& s01, f2& s23) {
-  uint32_t cd[4];
-  load_codes<BITS>(row, lane, cd);
-  const f2 ntb = dup(-tb);
-  const f2 q01 = add2(make_float2(__uint_as_float(cd[0]), __uint_as_float(cd[1])), ntb);
-  const f2 q23 = add2(make_float2(__uint_as_float(cd[2]), __uint_as_float(cd[3])), ntb);
-  s01 = mul2(mul2(q01, dup(rd)), cin[0]);
-  s23 = mul2(mul2(q23, dup(rd)), cin[1]);
-}
-
 // ---------------------------------------------------------------------------------
-// Staged inputs of one (request, head) in shared memory.
-// ---------------------------------------------------------------------------------
-struct __align__(16) HeadIn {
-  float k[D], q[D], v[D];
-  float gate[D];        // KDA per-row retention (unused for GDN)
-  float r[D], c[D];     // input scales (adjacent in the pool)
-  float g[D], om[D];    // row gain and omega of the head
-  uint32_t info[D];     // row widths and offsets
-  HeadRef ref;          // where the item lives in the pool
-  float gate_s, beta_s; // GDN retention and beta (plain loads)
-  int valid;            // slot index in range
-  int pad[3];
-};
-constexpr int HEAD_IN_BYTES = int(sizeof(HeadIn));
-static_assert(HEAD_IN_BYTES % 16 == 0, "staging sections must stay 16-byte aligned");
-
-// ---------------------------------------------------------------------------------
-// One (request, head) of stq_decode_step, reading its staged inputs `in`.
+// One (request, head) of stq_decode_step, from this warp's staged rows.
 // ---------------------------------------------------------------------------------
 template <int BITS>
-__device__ __forceinline__ void decode_head(const HeadIn& in, int kind, HeadSmem& sm, uint8_t* stage,
+__device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const HeadRef& hr, int warp_code_start,
+                                            const f2 (&cin)[2], const float4& v4, float beta_s,
                                             float* o_out) {
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  const int r0 = w * RPW;
-  const HeadRef& hr = in.ref;
   f2 s[RPW][2];
-  f2 cin[2];
-  {
-    const float4 c4 = *reinterpret_cast<const float4*>(&in.c[4 * lane]);
-    cin[0] = make_float2(c4.x, c4.y);
-    cin[1] = make_float2(c4.z, c4.w);
-  }
 
   // ---- restore S' = D (r c Q) and the column sums u_j = sum_i k_i S'_ij ---------------
 #pragma unroll
-  for (int g4 = 0; g4 < RPW / 4; ++g4) {
-    const float4 r4 = *reinterpret_cast<const float4*>(&in.r[r0 + 4 * g4]);
-    float4 d4 = make_float4(in.gate_s, in.gate_s, in.gate_s, in.gate_s);
-    if (kind != 0) d4 = *reinterpret_cast<const float4*>(&in.gate[r0 + 4 * g4]);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int rr = 4 * g4 + j, i = r0 + rr;
-      const float dec = at4(d4, j);
-      const float rd = fmul(dec, at4(r4, j));
-      if constexpr (BITS == MIXED) {
-        const uint32_t info = in.info[i];
-        const int bits = row_bits(info);
-        const uint8_t* row = stage + row_off(info);
-        const float tb = sm.ttb[bits];
-        switch (bits) {
-          case 2: restore_row<2>(row, lane, rd, tb, cin, s[rr][0], s[rr][1]); break;
-          case 4: restore_row<4>(row, lane, rd, tb, cin, s[rr][0], s[rr][1]); break;
-          case 6: restore_row<6>(row, lane, rd, tb, cin, s[rr][0], s[rr][1]); break;
-          case 8: restore_row<8>(row, lane, rd, tb, cin, s[rr][0], s[rr][1]); break;
-          default: {
-            const uint2 hv = *reinterpret_cast<const uint2*>(stage + hr.piv_stage_off +
-                                                              row_off(info) * (D * 2) + 8 * lane);
-            f2 a, b;
-            half4_floats(hv, a, b);
-            s[rr][0] = mul2(dup(dec), a);
-            s[rr][1] = mul2(dup(dec), b);
-          }
+  for (int rr = 0; rr < RPW; ++rr) {
+    if constexpr (BITS == MIXED) {
+      const uint32_t info = wr.info[rr];
+      const int bits = row_bits(info);
+      const uint8_t* row = wr.codes + (row_off(info) - warp_code_start);
+      const float rd = wr.rdd[rr].x, tb = wr.tb[rr];
+      switch (bits) {
+        case 2: restore_row<2>(row, lane, rd, tb, cin, s[rr][0], s[rr][1]); break;
+        case 4: restore_row<4>(row, lane, rd, tb, cin, s[rr][0], s[rr][1]); break;
+        case 6: restore_row<6>(row, lane, rd, tb, cin, s[rr][0], s[rr][1]); break;
+        case 8: restore_row<8>(row, lane, rd, tb, cin, s[rr][0], s[rr][1]); break;
+        default: {
+          const uint2 hv = *reinterpret_cast<const uint2*>(hr.pivots + row_off(info) * D + 4 * lane);
+          f2 x, y;
+          half4_floats(hv, x, y);
+          const f2 dd = dup(wr.dec[rr]);
+          s[rr][0] = mul2(dd, x);
+          s[rr][1] = mul2(dd, y);
         }
-      } else {
-        constexpr float TB = TWO23 + float(1 << (BITS - 1));
-        restore_row<BITS>(stage + i * (D * BITS / 8), lane, rd, TB, cin, s[rr][0], s[rr][1]);
       }
+    } else {
+      constexpr float TB = TWO23 + float(1 << (BITS - 1));
+      uint32_t cd[4];
+      load_codes<BITS>(wr.codes + rr * (D * BITS / 8), lane, cd);
+      const f2 rd = wr.rdd[rr];
+      const f2 q01 = add2(make_float2(__uint_as_float(cd[0]), __uint_as_float(cd[1])), dup(-TB));
+      const f2 q23 = add2(make_float2(__uint_as_float(cd[2]), __uint_as_float(cd[3])), dup(-TB));
+      s[rr][0] = mul2(mul2(q01, rd), cin[0]);
+      s[rr][1] = mul2(mul2(q23, rd), cin[1]);
     }
   }
   {
-    float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f);
     V2<2> u = tree<0, RPW / 2, 2>([&](int m) {
-      if ((m & 1) == 0) k4 = *reinterpret_cast<const float4*>(&in.k[r0 + 2 * m]);
-      const f2 ke = dup(at4(k4, (2 * m) & 3)), ko = dup(at4(k4, (2 * m + 1) & 3));
+      const f2 ke = wr.kk[2 * m], ko = wr.kk[2 * m + 1];
       V2<2> leaf;
       leaf.x[0] = fma2(ke, s[2 * m][0], mul2(ko, s[2 * m + 1][0]));
       leaf.x[1] = fma2(ke, s[2 * m][1], mul2(ko, s[2 * m + 1][1]));
       return leaf;
     });
-    put_partial(sm.red[0][0], w, lane, u.x[0], u.x[1]);
+    put_partial(cs.red[0][0], w, lane, u.x[0], u.x[1]);
   }
   __syncthreads();
 
@@ -566,126 +543,115 @@ __device__ __forceinline__ void decode_head(const HeadIn& in, int kind, HeadSmem
   f2 delta[2];
   {
     f2 ulo, uhi;
-    warp_tree(sm.red[0][0], lane, ulo, uhi);
-    const float4 v4 = *reinterpret_cast<const float4*>(&in.v[4 * lane]);
-    const f2 bt = dup(in.beta_s);
+    warp_tree(cs.red[0][0], lane, ulo, uhi);
+    const f2 bt = dup(beta_s);
     delta[0] = mul2(bt, add2(make_float2(v4.x, v4.y), make_float2(-ulo.x, -ulo.y)));
     delta[1] = mul2(bt, add2(make_float2(v4.z, v4.w), make_float2(-uhi.x, -uhi.y)));
   }
   {
-    float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f), q4 = k4;
     V2<2> o = tree<0, RPW / 2, 2>([&](int m) {
-      if ((m & 1) == 0) {
-        k4 = *reinterpret_cast<const float4*>(&in.k[r0 + 2 * m]);
-        q4 = *reinterpret_cast<const float4*>(&in.q[r0 + 2 * m]);
-      }
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const f2 kk = dup(at4(k4, (2 * m + e) & 3));
+        const f2 kk = wr.kk[2 * m + e];
         s[2 * m + e][0] = fma2(kk, delta[0], s[2 * m + e][0]);
         s[2 * m + e][1] = fma2(kk, delta[1], s[2 * m + e][1]);
       }
-      const f2 qe = dup(at4(q4, (2 * m) & 3)), qo = dup(at4(q4, (2 * m + 1) & 3));
+      const f2 qe = wr.qq[2 * m], qo = wr.qq[2 * m + 1];
       V2<2> leaf;
       leaf.x[0] = fma2(qe, s[2 * m][0], mul2(qo, s[2 * m + 1][0]));
       leaf.x[1] = fma2(qe, s[2 * m][1], mul2(qo, s[2 * m + 1][1]));
       return leaf;
     });
-    put_partial(sm.red[1][0], w, lane, o.x[0], o.x[1]);
+    put_partial(cs.red[1][0], w, lane, o.x[0], o.x[1]);
   }
   if constexpr (BITS == MIXED) {
     // pivot rows: store float16(S) now (they take no part in the refit)
 #pragma unroll
     for (int rr = 0; rr < RPW; ++rr) {
-      const uint32_t info = in.info[r0 + rr];
+      const uint32_t info = wr.info[rr];
       if (row_bits(info) == PIVOT)
         *reinterpret_cast<uint2*>(hr.pivots + row_off(info) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
     }
   }
   f2 c[2];
-  refit_pack<BITS>(in.g, in.om, in.info, sm, stage, s, hr.scales, c, o_out);
-  __syncthreads();
-  copy16(hr.codes, stage, hr.code_bytes);
+  refit_store<BITS>(cs, wr, s, hr.scales, hr.codes, warp_code_start, c, o_out);
   if (w == 0) *reinterpret_cast<float4*>(hr.scales + D + 4 * lane) = make_float4(c[0].x, c[0].y, c[1].x, c[1].y);
 }
 
 // A head whose rows are all FP16 pivots: decay, update, readout, store float16; r = c = 0.
-__device__ __forceinline__ void decode_pivot_head(const HeadIn& in, int kind, HeadSmem& sm,
-                                                  const uint8_t* stage, float* o_out) {
+__device__ __forceinline__ void decode_pivot_warp(CtaSmem& cs, WarpRows& wr, const HeadRef& hr,
+                                                  const float4& v4, float beta_s, float* o_out) {
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int r0 = w * RPW;
-  const HeadRef& hr = in.ref;
   f2 s[RPW][2];
 #pragma unroll
   for (int rr = 0; rr < RPW; ++rr) {
-    const int i = r0 + rr;
-    const uint2 hv = *reinterpret_cast<const uint2*>(stage + i * (D * 2) + 8 * lane);
-    f2 a, b;
-    half4_floats(hv, a, b);
-    const f2 dd = dup(kind != 0 ? in.gate[i] : in.gate_s);
-    s[rr][0] = mul2(dd, a);
-    s[rr][1] = mul2(dd, b);
+    const uint2 hv = *reinterpret_cast<const uint2*>(hr.pivots + (r0 + rr) * D + 4 * lane);
+    f2 x, y;
+    half4_floats(hv, x, y);
+    const f2 dd = dup(wr.dec[rr]);
+    s[rr][0] = mul2(dd, x);
+    s[rr][1] = mul2(dd, y);
   }
   {
     V2<2> u = tree<0, RPW / 2, 2>([&](int m) {
-      const f2 ke = dup(in.k[r0 + 2 * m]), ko = dup(in.k[r0 + 2 * m + 1]);
+      const f2 ke = wr.kk[2 * m], ko = wr.kk[2 * m + 1];
       V2<2> leaf;
       leaf.x[0] = fma2(ke, s[2 * m][0], mul2(ko, s[2 * m + 1][0]));
       leaf.x[1] = fma2(ke, s[2 * m][1], mul2(ko, s[2 * m + 1][1]));
       return leaf;
     });
-    put_partial(sm.red[0][0], w, lane, u.x[0], u.x[1]);
+    put_partial(cs.red[0][0], w, lane, u.x[0], u.x[1]);
   }
   __syncthreads();
   f2 delta[2];
   {
     f2 ulo, uhi;
-    warp_tree(sm.red[0][0], lane, ulo, uhi);
-    const float4 v4 = *reinterpret_cast<const float4*>(&in.v[4 * lane]);
-    const f2 bt = dup(in.beta_s);
+    warp_tree(cs.red[0][0], lane, ulo, uhi);
+    const f2 bt = dup(beta_s);
     delta[0] = mul2(bt, add2(make_float2(v4.x, v4.y), make_float2(-ulo.x, -ulo.y)));
     delta[1] = mul2(bt, add2(make_float2(v4.z, v4.w), make_float2(-uhi.x, -uhi.y)));
   }
   V2<2> o = tree<0, RPW / 2, 2>([&](int m) {
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      const f2 kk = dup(in.k[r0 + 2 * m + e]);
+      const f2 kk = wr.kk[2 * m + e];
       s[2 * m + e][0] = fma2(kk, delta[0], s[2 * m + e][0]);
       s[2 * m + e][1] = fma2(kk, delta[1], s[2 * m + e][1]);
     }
-    const f2 qe = dup(in.q[r0 + 2 * m]), qo = dup(in.q[r0 + 2 * m + 1]);
+    const f2 qe = wr.qq[2 * m], qo = wr.qq[2 * m + 1];
     V2<2> leaf;
     leaf.x[0] = fma2(qe, s[2 * m][0], mul2(qo, s[2 * m + 1][0]));
     leaf.x[1] = fma2(qe, s[2 * m][1], mul2(qo, s[2 * m + 1][1]));
     return leaf;
   });
-  put_partial(sm.red[1][0], w, lane, o.x[0], o.x[1]);
+  put_partial(cs.red[1][0], w, lane, o.x[0], o.x[1]);
 #pragma unroll
   for (int rr = 0; rr < RPW; ++rr)
     *reinterpret_cast<uint2*>(hr.pivots + (r0 + rr) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
   __syncthreads();
   if (w == 0) {
     f2 lo, hi;
-    warp_tree(sm.red[1][0], lane, lo, hi);
+    warp_tree(cs.red[1][0], lane, lo, hi);
     *reinterpret_cast<float4*>(o_out + 4 * lane) = make_float4(lo.x, lo.y, hi.x, hi.y);
   }
   if (tid < 2 * D) hr.scales[tid] = 0.0f;
 }
 
 // ---------------------------------------------------------------------------------
-// stq_decode_step: one CTA per (head, request) item, items numbered head-major so that
-// the CTAs resident on an SM at the same time mostly run the same width's code path.
+// stq_decode_step: one CTA per (head, request) item, numbered head-major so that the
+// CTAs resident on an SM at the same time mostly run the same width's code path. Each
+// warp stages its own 16 rows (asynchronous 16-byte copies) and writes its own codes
+// back, so the CTA synchronises only for the four column exchanges.
 // ---------------------------------------------------------------------------------
 __global__ void __launch_bounds__(NT, 2)
 decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* __restrict__ q,
               const float* __restrict__ k, const float* __restrict__ v,
               const float* __restrict__ gate, const float* __restrict__ beta,
               float* __restrict__ out) {
-  extern __shared__ __align__(16) uint8_t dyn[];
-  __shared__ HeadSmem sm;
-  HeadIn& in = *reinterpret_cast<HeadIn*>(dyn);
-  uint8_t* stage = dyn + HEAD_IN_BYTES;
-  const int tid = threadIdx.x;
+  __shared__ CtaSmem cs;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int r0 = w * RPW;
   const int h = blockIdx.x / B, bq = blockIdx.x - h * B;
   const int slot = slots[bq];
   if (slot < 0 || slot >= P.n_slots) {
@@ -695,35 +661,28 @@ decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* 
   const HeadRef hr = head_ref(P, slot, h);
   const int vi = bq * P.H + h;
   const uint64_t vec = uint64_t(vi) * D;
-  init_width_tables(sm);
-  if (tid < D) {
-    in.k[tid] = k[vec + tid];
-    in.q[tid] = q[vec + tid];
-    in.v[tid] = v[vec + tid];
-    if (P.kind != 0) in.gate[tid] = gate[vec + tid];
-    in.r[tid] = hr.scales[tid];
-    in.c[tid] = hr.scales[D + tid];
-    in.g[tid] = P.g[h * D + tid];
-    in.om[tid] = P.omega[h * D + tid];
-    in.info[tid] = P.row_info[h * D + tid];
-  }
-  if (tid == 0) {
-    in.ref = hr;
-    in.gate_s = (P.kind == 0) ? gate[vi] : 0.0f;
-    in.beta_s = beta[vi];
-    in.valid = 1;
-  }
-  copy16(stage, hr.codes, hr.code_bytes);
-  copy16(stage + hr.piv_stage_off, hr.pivots, hr.piv_count * D * 2);
-  __syncthreads();
+  WarpRows& wr = cs.wr[w];
+  // this warp's packed rows -> shared memory (16-byte asynchronous copies)
+  const int wstart = int(P.warp_code_off[h * NW + w]);
+  const int wend = (w + 1 < NW) ? int(P.warp_code_off[h * NW + w + 1]) : hr.code_bytes;
+  for (int o = 16 * lane; o < wend - wstart; o += 16 * 32) cp_async16(wr.codes + o, hr.codes + wstart + o);
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  const float gate_s = (P.kind == 0) ? gate[vi] : 0.0f;
+  load_warp_rows(P, h, wr, lane, r0, k + vec, q + vec, hr.scales, P.kind == 0 ? nullptr : gate + vec, gate_s);
+  const float beta_s = beta[vi];
+  const float4 c4 = *reinterpret_cast<const float4*>(hr.scales + D + 4 * lane);
+  const f2 cin[2] = {make_float2(c4.x, c4.y), make_float2(c4.z, c4.w)};
+  const float4 v4 = *reinterpret_cast<const float4*>(v + vec + 4 * lane);
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncwarp();
   float* o_out = out + vec;
   switch (hr.bits) {
-    case 2: decode_head<2>(in, P.kind, sm, stage, o_out); break;
-    case 4: decode_head<4>(in, P.kind, sm, stage, o_out); break;
-    case 6: decode_head<6>(in, P.kind, sm, stage, o_out); break;
-    case 8: decode_head<8>(in, P.kind, sm, stage, o_out); break;
-    case PIVOT: decode_pivot_head(in, P.kind, sm, stage, o_out); break;
-    default: decode_head<MIXED>(in, P.kind, sm, stage, o_out); break;
+    case 2: decode_warp<2>(cs, wr, hr, wstart, cin, v4, beta_s, o_out); break;
+    case 4: decode_warp<4>(cs, wr, hr, wstart, cin, v4, beta_s, o_out); break;
+    case 6: decode_warp<6>(cs, wr, hr, wstart, cin, v4, beta_s, o_out); break;
+    case 8: decode_warp<8>(cs, wr, hr, wstart, cin, v4, beta_s, o_out); break;
+    case PIVOT: decode_pivot_warp(cs, wr, hr, v4, beta_s, o_out); break;
+    default: decode_warp<MIXED>(cs, wr, hr, wstart, cin, v4, beta_s, o_out); break;
   }
 }
 
@@ -731,63 +690,61 @@ decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* 
 // stq_quantize_init: float32 states -> packed pool.
 // ---------------------------------------------------------------------------------
 template <int BITS>
-__device__ __forceinline__ void quantize_head(const PoolDev& P, int h, HeadSmem& sm, uint8_t* stage,
-                                              const HeadRef& hr, const float* src) {
+__device__ __forceinline__ void quantize_warp(CtaSmem& cs, WarpRows& wr, const HeadRef& hr, int warp_code_start,
+                                              const float* src) {
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int r0 = w * RPW;
   f2 s[RPW][2];
 #pragma unroll
   for (int rr = 0; rr < RPW; ++rr) {
-    const int i = r0 + rr;
-    const float4 x = *reinterpret_cast<const float4*>(src + i * D + 4 * lane);
+    const float4 x = *reinterpret_cast<const float4*>(src + (r0 + rr) * D + 4 * lane);
     s[rr][0] = make_float2(x.x, x.y);
     s[rr][1] = make_float2(x.z, x.w);
     if constexpr (BITS == MIXED) {
-      const uint32_t info = sm.info[i];
+      const uint32_t info = wr.info[rr];
       if (row_bits(info) == PIVOT)
         *reinterpret_cast<uint2*>(hr.pivots + row_off(info) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
     }
   }
   f2 c[2];
-  refit_pack<BITS>(P.g + h * D, P.omega + h * D, sm.info, sm, stage, s, hr.scales, c, nullptr);
-  __syncthreads();
-  copy16(hr.codes, stage, hr.code_bytes);
+  refit_store<BITS>(cs, wr, s, hr.scales, hr.codes, warp_code_start, c, nullptr);
   if (w == 0) *reinterpret_cast<float4*>(hr.scales + D + 4 * lane) = make_float4(c[0].x, c[0].y, c[1].x, c[1].y);
 }
 
 __global__ void __launch_bounds__(NT, 2)
 quantize_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* __restrict__ S) {
-  extern __shared__ __align__(16) uint8_t stage[];
-  __shared__ HeadSmem sm;
+  __shared__ CtaSmem cs;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int r0 = w * RPW;
   const int item = blockIdx.x;
   const int bq = item / P.H, h = item - bq * P.H;
-  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int slot = slots[bq];
   if (slot < 0 || slot >= P.n_slots) {
     if (tid == 0) atomicOr(P.err, ERR_SLOT_RANGE);
     return;
   }
   const HeadRef hr = head_ref(P, slot, h);
-  load_row_meta(P, h, sm);
-  init_width_tables(sm);
-  __syncthreads();
+  WarpRows& wr = cs.wr[w];
+  load_warp_rows(P, h, wr, lane, r0, nullptr, nullptr, nullptr, nullptr, 0.0f);
+  __syncwarp();
+  const int wstart = int(P.warp_code_off[h * NW + w]);
   const float* src = S + uint64_t(item) * D * D;
   switch (hr.bits) {
-    case 2: quantize_head<2>(P, h, sm, stage, hr, src); break;
-    case 4: quantize_head<4>(P, h, sm, stage, hr, src); break;
-    case 6: quantize_head<6>(P, h, sm, stage, hr, src); break;
-    case 8: quantize_head<8>(P, h, sm, stage, hr, src); break;
+    case 2: quantize_warp<2>(cs, wr, hr, wstart, src); break;
+    case 4: quantize_warp<4>(cs, wr, hr, wstart, src); break;
+    case 6: quantize_warp<6>(cs, wr, hr, wstart, src); break;
+    case 8: quantize_warp<8>(cs, wr, hr, wstart, src); break;
     case PIVOT:
 #pragma unroll
       for (int rr = 0; rr < RPW; ++rr) {
-        const int i = w * RPW + rr;
+        const int i = r0 + rr;
         const float4 x = *reinterpret_cast<const float4*>(src + i * D + 4 * lane);
         *reinterpret_cast<uint2*>(hr.pivots + i * D + 4 * lane) =
             half4_bits(make_float2(x.x, x.y), make_float2(x.z, x.w));
       }
       if (tid < 2 * D) hr.scales[tid] = 0.0f;
       break;
-    default: quantize_head<MIXED>(P, h, sm, stage, hr, src); break;
+    default: quantize_warp<MIXED>(cs, wr, hr, wstart, src); break;
   }
 }
 
@@ -937,7 +894,7 @@ cudaError_t prepare(K kernel, int dyn, int static_bytes, int* done_per_device) {
   return cudaSuccess;
 }
 
-int g_decode_dyn[64], g_quant_dyn[64], g_dequant_dyn[64];
+int g_dequant_dyn[64];
 
 }  // namespace
 
@@ -945,20 +902,14 @@ cudaError_t launch_decode(const PoolDev& P, const int32_t* slots, int B, const f
                           const float* k, const float* v, const float* gate,
                           const float* beta, float* out, cudaStream_t s) {
   if (B == 0) return cudaSuccess;
-  const int dyn = HEAD_IN_BYTES + stage_bytes(P);
-  cudaError_t e = prepare(decode_kernel, dyn, int(sizeof(HeadSmem)), g_decode_dyn);
-  if (e != cudaSuccess) return e;
-  decode_kernel<<<B * P.H, NT, dyn, s>>>(P, slots, B, q, k, v, gate, beta, out);
+  decode_kernel<<<B * P.H, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
   return cudaGetLastError();
 }
 
 cudaError_t launch_quantize(const PoolDev& P, const int32_t* slots, int B, const float* S,
                             cudaStream_t s) {
   if (B == 0) return cudaSuccess;
-  const int dyn = stage_bytes(P);
-  cudaError_t e = prepare(quantize_kernel, dyn, int(sizeof(HeadSmem)), g_quant_dyn);
-  if (e != cudaSuccess) return e;
-  quantize_kernel<<<B * P.H, NT, dyn, s>>>(P, slots, B, S);
+  quantize_kernel<<<B * P.H, NT, 0, s>>>(P, slots, B, S);
   return cudaGetLastError();
 }
 
