@@ -25,7 +25,6 @@
 //     clamping is done in that binade, where the low bits are the (biased) code.
 #include <cuda_fp16.h>
 
-#include "stq_fastdiv.cuh"
 #include "stq_internal.h"
 
 namespace stq {
@@ -54,7 +53,7 @@ __device__ __forceinline__ f2 dup(float x) { return make_float2(x, x); }
 
 // 1/a correctly rounded for a >= 2^-126; 0 for a smaller (or zero) scale.
 __device__ __forceinline__ float recip_scale(float a) {
-  return a >= SMALLEST_NORMAL ? rcp_rn(a) : 0.0f;
+  return a >= SMALLEST_NORMAL ? __frcp_rn(a) : 0.0f;
 }
 
 template <int N>
@@ -438,10 +437,10 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
     f2 nlo, nhi, dlo, dhi;
     warp_tree(num, lane, nlo, nhi);
     warp_tree(den, lane, dlo, dhi);
-    if (dlo.x > 0.0f) c[0].x = div_rn(nlo.x, dlo.x);
-    if (dlo.y > 0.0f) c[0].y = div_rn(nlo.y, dlo.y);
-    if (dhi.x > 0.0f) c[1].x = div_rn(nhi.x, dhi.x);
-    if (dhi.y > 0.0f) c[1].y = div_rn(nhi.y, dhi.y);
+    if (dlo.x > 0.0f) c[0].x = __fdiv_rn(nlo.x, dlo.x);
+    if (dlo.y > 0.0f) c[0].y = __fdiv_rn(nlo.y, dlo.y);
+    if (dhi.x > 0.0f) c[1].x = __fdiv_rn(nhi.x, dhi.x);
+    if (dhi.y > 0.0f) c[1].y = __fdiv_rn(nhi.y, dhi.y);
   }
 
   // --- final codes with the final c, stored straight into the pool -------------------
