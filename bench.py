@@ -91,6 +91,24 @@ def algorithmic_flops(w, B):
 
 
 # ---------------------------------------------------------------------------------
+# multi-rank timing: every rank times its own work; the job's time is the slowest rank
+# ---------------------------------------------------------------------------------
+def max_over_ranks(ms, world, device):
+    """Largest of the ranks' times (ms); a no-op for one rank."""
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step, world, ms_per_step):
+    """Units all ranks process per second (weak scaling: every rank does the same work)."""
+    return units_per_rank_step * world / (ms_per_step * 1e-3)
+
+
+# ---------------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------------
 class ClockSampler:
@@ -171,6 +189,31 @@ def oracle_rate(w, budget_s=10.0, reqs=1):
     return heads / el, {"kind": "oracle", "cores": 1,
                         "sample": f"{calls} oracle decode steps of {reqs} request(s) x {w.H} heads "
                                   f"of {w.name} in {el:.1f} s, one thread"}
+
+
+def measure_drift(pool, slots, S_fp32, w, B, gen, dev, steps):
+    """Chain `steps` decode steps on a copy of the packed state and on the FP32 state
+    with the same inputs; report the relative L2 distance of the dequantised packed
+    state from the FP32 state, and of the readouts, at the end (reported, not gated)."""
+    import torch
+    from quantized_linear_attention_02_b200 import stq
+    sub = min(B, 64)                       # a sub-batch keeps the FP32 copy small
+    idx = slots[:sub].contiguous()
+    S = S_fp32[:sub].clone()
+    pool.quantize_init(idx, S)
+    o_q = torch.empty((sub, w.H, D), device=dev)
+    o_f = torch.empty_like(o_q)
+    g2 = torch.Generator(device=dev).manual_seed(4242)
+    for _ in range(steps):
+        q, k, v, g, b = W.torch_step_inputs(w, sub, g2, dev)
+        pool.decode_step(idx, q, k, v, g, b, o_q)
+        stq.fp32_decode_step(w.kind, S, q, k, v, g, b, o_f)
+    Sq = torch.empty_like(S)
+    pool.dequantize(idx, Sq)
+    pool.check()
+    rel_s = float(torch.linalg.vector_norm(Sq - S) / torch.linalg.vector_norm(S))
+    rel_o = float(torch.linalg.vector_norm(o_q - o_f) / torch.linalg.vector_norm(o_f))
+    return {"steps": steps, "requests": sub, "state_rel_l2_vs_fp32": rel_s, "readout_rel_l2_vs_fp32": rel_o}
 
 
 def reference_arm(args, rank, world):
@@ -258,6 +301,9 @@ def stq_arm(args, rank, world, local_rank):
     W.torch_scale_outlier_rows(S, w)
     pool.quantize_init(slots, S)
     pool.check()
+    drift = None
+    if args.drift_steps > 0:
+        drift = measure_drift(pool, slots, S, w, B, gen, dev, args.drift_steps)
     del S
     torch.cuda.empty_cache()
 
@@ -294,13 +340,10 @@ def stq_arm(args, rank, world, local_rank):
     clk = clocks.stop()
     pool.check()
 
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, world, dev)
     ms_step = ms_max / args.steps
     heads_per_step = B * H * world
-    value = heads_per_step / (ms_step * 1e-3)
+    value = whole_job_rate(B * H, world, ms_step)
 
     # end to end through the host-buffer entry point: pinned inputs in, readout out
     e2e = None
@@ -321,12 +364,11 @@ def stq_arm(args, rank, world, local_rank):
             pool.decode_step_host(slots, *pin[i % 2], h_out, staging, stream)
         f1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)
         if world > 1:
             dist.barrier()
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        te = max_over_ranks(f0.elapsed_time(f1), world, dev)
         h2d = sum(x.numel() * 4 for x in pin[0])
-        e2e = {"value": heads_per_step / (float(te.item()) / n_e * 1e-3), "unit": UNIT,
+        e2e = {"value": whole_job_rate(B * H, world, te / n_e), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": B * H * D * 4, "steps": n_e}
 
     if rank != 0:
@@ -361,6 +403,8 @@ def stq_arm(args, rank, world, local_rank):
         "roofline": roofline, "roofline_other": other,
         "clocks": clk, "e2e": e2e, "gpu_launches": args.steps,
     }
+    if drift is not None:
+        line["drift"] = drift
     if world == 1 and not args.no_cpu_baseline:
         rate, info = oracle_rate(w, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, **info}
@@ -378,6 +422,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-budget", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--drift-steps", type=int, default=0,
+                    help="after timing, chain this many steps on 64 requests against the FP32 state")
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling captures only)")
     ap.add_argument("--compact-slots", action="store_true", help="B slots instead of 5B+1 (profiling captures only)")
     ap.add_argument("--warm-steps", type=int, default=-1, help="override the FP32 warm-up length (profiling only)")

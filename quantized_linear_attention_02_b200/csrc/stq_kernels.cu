@@ -347,7 +347,8 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
   float mx[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
   for (int rr = 0; rr < RPW; ++rr) {
-    const f2 ir = wr.irr[rr];
+    const float4 i2 = *reinterpret_cast<const float4*>(&wr.irr[rr & ~1]);
+    const f2 ir = (rr & 1) ? make_float2(i2.z, i2.w) : make_float2(i2.x, i2.y);
     s[rr][0] = mul2(s[rr][0], ir);
     s[rr][1] = mul2(s[rr][1], ir);
     if constexpr (BITS == MIXED) {
@@ -398,10 +399,11 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
     V2<4> nd = tree<0, RPW / 2, 4>([&](int m) {
       // rows 2m and 2m+1 form one fused pair of each sum
       f2 Q[2][2], p[2][2];
+      const float4 b2 = *reinterpret_cast<const float4*>(&wr.bb[2 * m]);
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int rr = 2 * m + e;
-        const f2 bb = wr.bb[rr];
+        const f2 bb = e == 0 ? make_float2(b2.x, b2.y) : make_float2(b2.z, b2.w);
         float lo_b, hi_b;
         if constexpr (BITS == MIXED) {
           lo_b = MAGIC - wr.qm[rr];
@@ -519,7 +521,8 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
       constexpr float TB = TWO23 + float(1 << (BITS - 1));
       uint32_t cd[4];
       load_codes<BITS>(wr.codes + rr * (D * BITS / 8), lane, cd);
-      const f2 rd = wr.rdd[rr];
+      const float4 r2 = *reinterpret_cast<const float4*>(&wr.rdd[rr & ~1]);
+      const f2 rd = (rr & 1) ? make_float2(r2.z, r2.w) : make_float2(r2.x, r2.y);
       const f2 q01 = add2(make_float2(__uint_as_float(cd[0]), __uint_as_float(cd[1])), dup(-TB));
       const f2 q23 = add2(make_float2(__uint_as_float(cd[2]), __uint_as_float(cd[3])), dup(-TB));
       s[rr][0] = mul2(mul2(q01, rd), cin[0]);
@@ -528,7 +531,8 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
   }
   {
     V2<2> u = tree<0, RPW / 2, 2>([&](int m) {
-      const f2 ke = wr.kk[2 * m], ko = wr.kk[2 * m + 1];
+      const float4 k2 = *reinterpret_cast<const float4*>(&wr.kk[2 * m]);
+      const f2 ke = make_float2(k2.x, k2.y), ko = make_float2(k2.z, k2.w);
       V2<2> leaf;
       leaf.x[0] = fma2(ke, s[2 * m][0], mul2(ko, s[2 * m + 1][0]));
       leaf.x[1] = fma2(ke, s[2 * m][1], mul2(ko, s[2 * m + 1][1]));
@@ -549,13 +553,15 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
   }
   {
     V2<2> o = tree<0, RPW / 2, 2>([&](int m) {
+      const float4 k2 = *reinterpret_cast<const float4*>(&wr.kk[2 * m]);
+      const float4 q2 = *reinterpret_cast<const float4*>(&wr.qq[2 * m]);
+      const f2 kp[2] = {make_float2(k2.x, k2.y), make_float2(k2.z, k2.w)};
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const f2 kk = wr.kk[2 * m + e];
-        s[2 * m + e][0] = fma2(kk, delta[0], s[2 * m + e][0]);
-        s[2 * m + e][1] = fma2(kk, delta[1], s[2 * m + e][1]);
+        s[2 * m + e][0] = fma2(kp[e], delta[0], s[2 * m + e][0]);
+        s[2 * m + e][1] = fma2(kp[e], delta[1], s[2 * m + e][1]);
       }
-      const f2 qe = wr.qq[2 * m], qo = wr.qq[2 * m + 1];
+      const f2 qe = make_float2(q2.x, q2.y), qo = make_float2(q2.z, q2.w);
       V2<2> leaf;
       leaf.x[0] = fma2(qe, s[2 * m][0], mul2(qo, s[2 * m + 1][0]));
       leaf.x[1] = fma2(qe, s[2 * m][1], mul2(qo, s[2 * m + 1][1]));
@@ -594,7 +600,8 @@ __device__ __forceinline__ void decode_pivot_warp(CtaSmem& cs, WarpRows& wr, con
   }
   {
     V2<2> u = tree<0, RPW / 2, 2>([&](int m) {
-      const f2 ke = wr.kk[2 * m], ko = wr.kk[2 * m + 1];
+      const float4 k2 = *reinterpret_cast<const float4*>(&wr.kk[2 * m]);
+      const f2 ke = make_float2(k2.x, k2.y), ko = make_float2(k2.z, k2.w);
       V2<2> leaf;
       leaf.x[0] = fma2(ke, s[2 * m][0], mul2(ko, s[2 * m + 1][0]));
       leaf.x[1] = fma2(ke, s[2 * m][1], mul2(ko, s[2 * m + 1][1]));
@@ -612,13 +619,15 @@ __device__ __forceinline__ void decode_pivot_warp(CtaSmem& cs, WarpRows& wr, con
     delta[1] = mul2(bt, add2(make_float2(v4.z, v4.w), make_float2(-uhi.x, -uhi.y)));
   }
   V2<2> o = tree<0, RPW / 2, 2>([&](int m) {
+    const float4 k2 = *reinterpret_cast<const float4*>(&wr.kk[2 * m]);
+    const float4 q2 = *reinterpret_cast<const float4*>(&wr.qq[2 * m]);
+    const f2 kp[2] = {make_float2(k2.x, k2.y), make_float2(k2.z, k2.w)};
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      const f2 kk = wr.kk[2 * m + e];
-      s[2 * m + e][0] = fma2(kk, delta[0], s[2 * m + e][0]);
-      s[2 * m + e][1] = fma2(kk, delta[1], s[2 * m + e][1]);
+      s[2 * m + e][0] = fma2(kp[e], delta[0], s[2 * m + e][0]);
+      s[2 * m + e][1] = fma2(kp[e], delta[1], s[2 * m + e][1]);
     }
-    const f2 qe = wr.qq[2 * m], qo = wr.qq[2 * m + 1];
+    const f2 qe = make_float2(q2.x, q2.y), qo = make_float2(q2.z, q2.w);
     V2<2> leaf;
     leaf.x[0] = fma2(qe, s[2 * m][0], mul2(qo, s[2 * m + 1][0]));
     leaf.x[1] = fma2(qe, s[2 * m][1], mul2(qo, s[2 * m + 1][1]));
