@@ -233,6 +233,7 @@ struct __align__(16) WarpRows {
 
 struct __align__(16) CtaSmem {
   float4 red[2][2][NW][D / 4];     // ping-pong partials: [buffer][quantity][warp][col/4]
+  float col_ic[D];                 // 1/c_j of the current column scale, from its owner
   WarpRows wr[NW];
 };
 
@@ -290,7 +291,7 @@ __device__ __forceinline__ void load_warp_rows(const PoolDev& P, int h, WarpRows
 // ---------------------------------------------------------------------------------
 template <int BITS>
 __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], float* r_global,
-                                            uint8_t* codes_global, int warp_code_start, f2 (&c_out)[2],
+                                            float* c_global, uint8_t* codes_global, int warp_code_start,
                                             float* o_global) {
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r0 = w * RPW;
@@ -372,30 +373,34 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
     warp_tree(cs.red[1][0], lane, lo, hi);
     *reinterpret_cast<float4*>(o_global + 4 * lane) = make_float4(lo.x, lo.y, hi.x, hi.y);
   }
-  f2 c[2];
+  // Column scales are owned: lane l of warp w (l < 16) owns column 16w + l, keeps its c
+  // in a register and publishes 1/c for everyone through shared memory; the other 16
+  // lanes help reduce the least-squares denominators.
+  const int jown = 16 * w + (lane & 15);
+  float c_own;
   {
-    float m[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float m = 0.0f;
 #pragma unroll
-    for (int ww = 0; ww < NW; ++ww) {
-      const float4 v = cs.red[1][1][ww][lane];
-      m[0] = fmaxf(m[0], v.x); m[1] = fmaxf(m[1], v.y); m[2] = fmaxf(m[2], v.z); m[3] = fmaxf(m[3], v.w);
-    }
+    for (int ww = 0; ww < NW; ++ww) m = fmaxf(m, reinterpret_cast<const float*>(cs.red[1][1][ww])[jown]);
     if constexpr (BITS != MIXED) {
       // max_i RN(|y| / qmax) = RN(max_i |y| / qmax): rounding is monotone
       constexpr float QM = float((1 << (BITS - 1)) - 1);
-      const float iq = __frcp_rn(QM);
-#pragma unroll
-      for (int t = 0; t < 4; ++t) m[t] = fmul(m[t], iq);
+      m = fmul(m, __frcp_rn(QM));
     }
-    c[0] = make_float2(m[0], m[1]);
-    c[1] = make_float2(m[2], m[3]);
+    c_own = m;
+    if (lane < 16) cs.col_ic[jown] = recip_scale(c_own);
   }
+  __syncthreads();
 
   // --- two least-squares steps: c_j <- sum_i p y / sum_i p Q, p = b_i Q_ij -------------
 #pragma unroll
   for (int it = 0; it < 2; ++it) {
-    const f2 ic[2] = {make_float2(recip_scale(c[0].x), recip_scale(c[0].y)),
-                      make_float2(recip_scale(c[1].x), recip_scale(c[1].y))};
+    f2 ic[2];
+    {
+      const float4 i4 = *reinterpret_cast<const float4*>(&cs.col_ic[4 * lane]);
+      ic[0] = make_float2(i4.x, i4.y);
+      ic[1] = make_float2(i4.z, i4.w);
+    }
     V2<4> nd = tree<0, RPW / 2, 4>([&](int m) {
       // rows 2m and 2m+1 form one fused pair of each sum
       f2 Q[2][2], p[2][2];
@@ -431,23 +436,33 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
       }
       return leaf;
     });
-    float4 (*const num)[D / 4] = cs.red[it][0];
-    float4 (*const den)[D / 4] = cs.red[it][1];
-    put_partial(num, w, lane, nd.x[0], nd.x[1]);
-    put_partial(den, w, lane, nd.x[2], nd.x[3]);
+    put_partial(cs.red[it][0], w, lane, nd.x[0], nd.x[1]);
+    put_partial(cs.red[it][1], w, lane, nd.x[2], nd.x[3]);
     __syncthreads();
-    f2 nlo, nhi, dlo, dhi;
-    warp_tree(num, lane, nlo, nhi);
-    warp_tree(den, lane, dlo, dhi);
-    if (dlo.x > 0.0f) c[0].x = __fdiv_rn(nlo.x, dlo.x);
-    if (dlo.y > 0.0f) c[0].y = __fdiv_rn(nlo.y, dlo.y);
-    if (dhi.x > 0.0f) c[1].x = __fdiv_rn(nhi.x, dhi.x);
-    if (dhi.y > 0.0f) c[1].y = __fdiv_rn(nhi.y, dhi.y);
+    {
+      // lanes 0..15: numerator of column jown, lanes 16..31: its denominator
+      const float* part = reinterpret_cast<const float*>(cs.red[it][lane >> 4][0]);
+      float x[NW];
+#pragma unroll
+      for (int ww = 0; ww < NW; ++ww) x[ww] = part[ww * D + jown];
+      const float sum = fadd(fadd(fadd(x[0], x[1]), fadd(x[2], x[3])), fadd(fadd(x[4], x[5]), fadd(x[6], x[7])));
+      const float den = __shfl_down_sync(0xffffffffu, sum, 16);
+      if (lane < 16) {
+        if (den > 0.0f) c_own = __fdiv_rn(sum, den);
+        cs.col_ic[jown] = recip_scale(c_own);
+      }
+    }
+    __syncthreads();
   }
 
   // --- final codes with the final c, stored straight into the pool -------------------
-  const f2 ic[2] = {make_float2(recip_scale(c[0].x), recip_scale(c[0].y)),
-                    make_float2(recip_scale(c[1].x), recip_scale(c[1].y))};
+  f2 ic[2];
+  {
+    const float4 i4 = *reinterpret_cast<const float4*>(&cs.col_ic[4 * lane]);
+    ic[0] = make_float2(i4.x, i4.y);
+    ic[1] = make_float2(i4.z, i4.w);
+  }
+  if (lane < 16) c_global[jown] = c_own;
 #pragma unroll
   for (int rr = 0; rr < RPW; ++rr) {
     if constexpr (BITS == MIXED) {
@@ -481,8 +496,6 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
       store_codes<BITS>(codes_global + warp_code_start + rr * (D * BITS / 8), lane, t);
     }
   }
-  c_out[0] = c[0];
-  c_out[1] = c[1];
 }
 
 // ---------------------------------------------------------------------------------
@@ -578,9 +591,7 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
         *reinterpret_cast<uint2*>(hr.pivots + row_off(info) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
     }
   }
-  f2 c[2];
-  refit_store<BITS>(cs, wr, s, hr.scales, hr.codes, warp_code_start, c, o_out);
-  if (w == 0) *reinterpret_cast<float4*>(hr.scales + D + 4 * lane) = make_float4(c[0].x, c[0].y, c[1].x, c[1].y);
+  refit_store<BITS>(cs, wr, s, hr.scales, hr.scales + D, hr.codes, warp_code_start, o_out);
 }
 
 // A head whose rows are all FP16 pivots: decay, update, readout, store float16; r = c = 0.
@@ -714,9 +725,7 @@ __device__ __forceinline__ void quantize_warp(CtaSmem& cs, WarpRows& wr, const H
         *reinterpret_cast<uint2*>(hr.pivots + row_off(info) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
     }
   }
-  f2 c[2];
-  refit_store<BITS>(cs, wr, s, hr.scales, hr.codes, warp_code_start, c, nullptr);
-  if (w == 0) *reinterpret_cast<float4*>(hr.scales + D + 4 * lane) = make_float4(c[0].x, c[0].y, c[1].x, c[1].y);
+  refit_store<BITS>(cs, wr, s, hr.scales, hr.scales + D, hr.codes, warp_code_start, nullptr);
 }
 
 __global__ void __launch_bounds__(NT, 2)
