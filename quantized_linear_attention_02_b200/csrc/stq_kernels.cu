@@ -234,6 +234,7 @@ struct __align__(16) WarpRows {
 struct __align__(16) CtaSmem {
   float4 red[2][2][NW][D / 4];     // ping-pong partials: [buffer][quantity][warp][col/4]
   float col_ic[D];                 // 1/c_j of the current column scale, from its owner
+  float col_delta[D];              // delta_j = beta (v_j - u_j), from its owner
   WarpRows wr[NW];
 };
 
@@ -501,9 +502,24 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
 // ---------------------------------------------------------------------------------
 // One (request, head) of stq_decode_step, from this warp's staged rows.
 // ---------------------------------------------------------------------------------
+// Lane l < 16 of warp w owns column j = 16w + l: it sums the eight warps' partials of
+// u_j = (k^T S')_j in the tree ((w0+w1)+(w2+w3))+((w4+w5)+(w6+w7)) and publishes
+// delta_j = beta (v_j - u_j) through shared memory.
+__device__ __forceinline__ void publish_delta(CtaSmem& cs, int lane, int w, float v_own, float beta_s) {
+  if (lane < 16) {
+    const int j = 16 * w + lane;
+    const float* part = reinterpret_cast<const float*>(cs.red[0][0][0]);
+    float x[NW];
+#pragma unroll
+    for (int ww = 0; ww < NW; ++ww) x[ww] = part[ww * D + j];
+    const float u = fadd(fadd(fadd(x[0], x[1]), fadd(x[2], x[3])), fadd(fadd(x[4], x[5]), fadd(x[6], x[7])));
+    cs.col_delta[j] = fmul(beta_s, fadd(v_own, -u));
+  }
+}
+
 template <int BITS>
 __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const HeadRef& hr, int warp_code_start,
-                                            const f2 (&cin)[2], const float4& v4, float beta_s,
+                                            const f2 (&cin)[2], float v_own, float beta_s,
                                             float* o_out) {
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   f2 s[RPW][2];
@@ -555,14 +571,14 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
   }
   __syncthreads();
 
-  // ---- delta_j = beta (v_j - u_j); S = S' + k delta^T; readout partials ----------------
+  // ---- delta_j = beta (v_j - u_j) by its column owner; S = S' + k delta^T; readout ----
   f2 delta[2];
+  publish_delta(cs, lane, w, v_own, beta_s);
+  __syncthreads();
   {
-    f2 ulo, uhi;
-    warp_tree(cs.red[0][0], lane, ulo, uhi);
-    const f2 bt = dup(beta_s);
-    delta[0] = mul2(bt, add2(make_float2(v4.x, v4.y), make_float2(-ulo.x, -ulo.y)));
-    delta[1] = mul2(bt, add2(make_float2(v4.z, v4.w), make_float2(-uhi.x, -uhi.y)));
+    const float4 d4 = *reinterpret_cast<const float4*>(&cs.col_delta[4 * lane]);
+    delta[0] = make_float2(d4.x, d4.y);
+    delta[1] = make_float2(d4.z, d4.w);
   }
   {
     V2<2> o = tree<0, RPW / 2, 2>([&](int m) {
@@ -596,7 +612,7 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
 
 // A head whose rows are all FP16 pivots: decay, update, readout, store float16; r = c = 0.
 __device__ __forceinline__ void decode_pivot_warp(CtaSmem& cs, WarpRows& wr, const HeadRef& hr,
-                                                  const float4& v4, float beta_s, float* o_out) {
+                                                  float v_own, float beta_s, float* o_out) {
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int r0 = w * RPW;
   f2 s[RPW][2];
@@ -622,12 +638,12 @@ __device__ __forceinline__ void decode_pivot_warp(CtaSmem& cs, WarpRows& wr, con
   }
   __syncthreads();
   f2 delta[2];
+  publish_delta(cs, lane, w, v_own, beta_s);
+  __syncthreads();
   {
-    f2 ulo, uhi;
-    warp_tree(cs.red[0][0], lane, ulo, uhi);
-    const f2 bt = dup(beta_s);
-    delta[0] = mul2(bt, add2(make_float2(v4.x, v4.y), make_float2(-ulo.x, -ulo.y)));
-    delta[1] = mul2(bt, add2(make_float2(v4.z, v4.w), make_float2(-uhi.x, -uhi.y)));
+    const float4 d4 = *reinterpret_cast<const float4*>(&cs.col_delta[4 * lane]);
+    delta[0] = make_float2(d4.x, d4.y);
+    delta[1] = make_float2(d4.z, d4.w);
   }
   V2<2> o = tree<0, RPW / 2, 2>([&](int m) {
     const float4 k2 = *reinterpret_cast<const float4*>(&wr.kk[2 * m]);
@@ -661,7 +677,7 @@ __device__ __forceinline__ void decode_pivot_warp(CtaSmem& cs, WarpRows& wr, con
 // stq_decode_step: one CTA per (head, request) item, numbered head-major so that the
 // CTAs resident on an SM at the same time mostly run the same width's code path. Each
 // warp stages its own 16 rows (asynchronous 16-byte copies) and writes its own codes
-// back, so the CTA synchronises only for the four column exchanges.
+// back, so the CTA synchronises only for the five column exchanges.
 // ---------------------------------------------------------------------------------
 __global__ void __launch_bounds__(NT, 2)
 decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* __restrict__ q,
@@ -691,17 +707,17 @@ decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* 
   const float beta_s = beta[vi];
   const float4 c4 = *reinterpret_cast<const float4*>(hr.scales + D + 4 * lane);
   const f2 cin[2] = {make_float2(c4.x, c4.y), make_float2(c4.z, c4.w)};
-  const float4 v4 = *reinterpret_cast<const float4*>(v + vec + 4 * lane);
+  const float v_own = v[vec + 16 * w + (lane & 15)];
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncwarp();
   float* o_out = out + vec;
   switch (hr.bits) {
-    case 2: decode_warp<2>(cs, wr, hr, wstart, cin, v4, beta_s, o_out); break;
-    case 4: decode_warp<4>(cs, wr, hr, wstart, cin, v4, beta_s, o_out); break;
-    case 6: decode_warp<6>(cs, wr, hr, wstart, cin, v4, beta_s, o_out); break;
-    case 8: decode_warp<8>(cs, wr, hr, wstart, cin, v4, beta_s, o_out); break;
-    case PIVOT: decode_pivot_warp(cs, wr, hr, v4, beta_s, o_out); break;
-    default: decode_warp<MIXED>(cs, wr, hr, wstart, cin, v4, beta_s, o_out); break;
+    case 2: decode_warp<2>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
+    case 4: decode_warp<4>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
+    case 6: decode_warp<6>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
+    case 8: decode_warp<8>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
+    case PIVOT: decode_pivot_warp(cs, wr, hr, v_own, beta_s, o_out); break;
+    default: decode_warp<MIXED>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
   }
 }
 
