@@ -34,7 +34,6 @@ constexpr int NT = 256;   // threads per head-state
 constexpr int NW = 8;     // warps per head-state
 constexpr int RPW = 16;   // key rows per warp
 constexpr float MAGIC = 12582912.0f;        // 1.5 * 2^23
-constexpr float TWO23 = 8388608.0f;         // 2^23
 constexpr uint32_t FLOAT_2P23 = 0x4B000000u;
 constexpr float SMALLEST_NORMAL = 1.17549435e-38f;  // 2^-126
 constexpr int MIXED = 0;
@@ -84,7 +83,25 @@ __device__ __forceinline__ int row_off(uint32_t info) { return int(info >> 8); }
 // lane l owns codes 4l..4l+3 = bits [4bl, 4bl+4b) = bytes [bl/2, bl/2 + b/2)
 // ---------------------------------------------------------------------------------
 
-// The four codes of a lane as floats 2^23 + u (exact), from a 16-byte aligned row.
+// Bit position the unpacked code k of a lane sits at inside its float's mantissa. The
+// float is 2^(23 - pos) + u exactly (exponent 127 + 23 - pos, u * 2^pos in the mantissa,
+// which needs u * 2^pos < 2^23), so no code has to be shifted down to bit 0.
+template <int BITS>
+__host__ __device__ constexpr int code_pos(int k) {
+  return BITS == 8 ? 0 : BITS == 6 ? (k == 3 ? 17 : 6 * k) : BITS * k;
+}
+template <int BITS>
+__host__ __device__ constexpr uint32_t code_exp(int k) {
+  return uint32_t(127 + 23 - code_pos<BITS>(k)) << 23;
+}
+// 2^(23 - pos) + bias: subtracting it from the unpacked float gives Q = u - bias exactly.
+template <int BITS>
+__host__ __device__ constexpr float code_offset(int k) {
+  return float(1u << (23 - code_pos<BITS>(k))) + float(1 << (BITS - 1));
+}
+
+// The four codes of a lane as floats 2^(23 - pos_k) + u_k (exact), from a 16-byte
+// aligned row.
 template <int BITS>
 __device__ __forceinline__ void load_codes(const uint8_t* row, int lane, uint32_t (&c)[4]) {
   if constexpr (BITS == 8) {
@@ -94,25 +111,38 @@ __device__ __forceinline__ void load_codes(const uint8_t* row, int lane, uint32_
     c[2] = __byte_perm(w, FLOAT_2P23, 0x7542);
     c[3] = __byte_perm(w, FLOAT_2P23, 0x7543);
   } else {
-    uint32_t f;
+    constexpr uint32_t M = (1u << BITS) - 1u;
+    uint32_t f, f3;
     if constexpr (BITS == 4) {
       f = reinterpret_cast<const uint16_t*>(row)[lane];
+      f3 = f;
     } else if constexpr (BITS == 2) {
       f = row[lane];
+      f3 = f;
     } else {
-      // 6 bits: bytes 3l..3l+2, inside word 3l/4 and possibly the next one
+      // 6 bits: bytes 3l..3l+2, inside word 3l/4 and possibly the next one; code 3 is
+      // taken one bit lower (position 17) from a second funnel shift
       const uint32_t* wp = reinterpret_cast<const uint32_t*>(row);
       const int byte = 3 * lane, wi = byte >> 2, sh = (byte & 3) * 8;
       const uint32_t lo = wp[wi];
       const uint32_t hi = (sh > 8) ? wp[wi + 1] : 0u;  // wi + 1 <= 23 whenever sh > 8
       f = __funnelshift_r(lo, hi, sh);
+      f3 = __funnelshift_r(lo, hi, sh + 1);
     }
-    constexpr uint32_t M = (1u << BITS) - 1u;
-    c[0] = (f & M) | FLOAT_2P23;
-    c[1] = ((f >> BITS) & M) | FLOAT_2P23;
-    c[2] = ((f >> (2 * BITS)) & M) | FLOAT_2P23;
-    c[3] = ((f >> (3 * BITS)) & M) | FLOAT_2P23;
+    c[0] = (f & (M << code_pos<BITS>(0))) | code_exp<BITS>(0);
+    c[1] = (f & (M << code_pos<BITS>(1))) | code_exp<BITS>(1);
+    c[2] = (f & (M << code_pos<BITS>(2))) | code_exp<BITS>(2);
+    c[3] = (f3 & (M << code_pos<BITS>(3))) | code_exp<BITS>(3);
   }
+}
+
+// Q of the four codes as two float pairs.
+template <int BITS>
+__device__ __forceinline__ void codes_to_q(const uint32_t (&cd)[4], f2& q01, f2& q23) {
+  q01 = add2(make_float2(__uint_as_float(cd[0]), __uint_as_float(cd[1])),
+             make_float2(-code_offset<BITS>(0), -code_offset<BITS>(1)));
+  q23 = add2(make_float2(__uint_as_float(cd[2]), __uint_as_float(cd[3])),
+             make_float2(-code_offset<BITS>(2), -code_offset<BITS>(3)));
 }
 
 // Pack four biased codes (low bits of t = 1.5*2^23 + u) and store them into a row.
@@ -139,6 +169,41 @@ __device__ __forceinline__ void store_codes(uint8_t* row, int lane, const uint32
       *p8 = static_cast<uint8_t>(odd ? f : (f >> 16));
       *p16 = static_cast<uint16_t>(odd ? (f >> 8) : f);
     }
+  }
+}
+
+// Final codes in 16-bit lanes. t = fma(y, 1/c, 1.5*2^23 + bias) holds bias + n in its low
+// 16 bits (two's complement) whenever |n| < 2^15, n = rint(y / c); two such low halves
+// are clamped to [1, 2^b - 1] = bias + [-qmax, qmax] with one packed min and one packed
+// max, then packed. The caller guarantees |n| < 2^15 (see refit_store).
+__device__ __forceinline__ uint32_t clamp_s16x2(uint32_t x, uint32_t hi) {
+  uint32_t y;
+  asm("max.s16x2 %0, %1, %2;" : "=r"(y) : "r"(x), "r"(0x00010001u));
+  asm("min.s16x2 %0, %1, %2;" : "=r"(y) : "r"(y), "r"(hi));
+  return y;
+}
+
+template <int BITS>
+__device__ __forceinline__ void store_codes_s16(uint8_t* row, int lane, f2 t01, f2 t23, uint32_t hi) {
+  const uint32_t w01 = clamp_s16x2(__byte_perm(__float_as_uint(t01.x), __float_as_uint(t01.y), 0x5410), hi);
+  const uint32_t w23 = clamp_s16x2(__byte_perm(__float_as_uint(t23.x), __float_as_uint(t23.y), 0x5410), hi);
+  if constexpr (BITS == 8) {
+    reinterpret_cast<uint32_t*>(row)[lane] = __byte_perm(w01, w23, 0x6420);
+  } else if constexpr (BITS == 4) {
+    const uint32_t x01 = w01 | (w01 >> 12), x23 = w23 | (w23 >> 12);
+    reinterpret_cast<uint16_t*>(row)[lane] = static_cast<uint16_t>(__byte_perm(x01, x23, 0x0040));
+  } else if constexpr (BITS == 2) {
+    const uint32_t x = w01 | (w23 << 4);
+    row[lane] = static_cast<uint8_t>(x | (x >> 14));
+  } else {
+    const uint32_t x01 = w01 | (w01 >> 10), x23 = w23 | (w23 >> 10);
+    const uint32_t f = (x01 & 0xFFFu) | (x23 << 12);   // bits 24.. are not stored
+    const bool odd = lane & 1;
+    uint8_t* p = row + 3 * lane;
+    uint8_t* p8 = odd ? p : p + 2;
+    uint16_t* p16 = reinterpret_cast<uint16_t*>(odd ? p + 1 : p);
+    *p8 = static_cast<uint8_t>(odd ? f : (f >> 16));
+    *p16 = static_cast<uint16_t>(odd ? (f >> 8) : f);
   }
 }
 
@@ -206,13 +271,12 @@ __device__ __forceinline__ void put_partial(float4 (*red)[D / 4], int w, int lan
 
 // Restore one row of S' = D (r c Q) for this lane's 4 columns.
 template <int BITS>
-__device__ __forceinline__ void restore_row(const uint8_t* row, int lane, float rd, float tb,
+__device__ __forceinline__ void restore_row(const uint8_t* row, int lane, float rd,
                                             const f2 (&cin)[2], f2& s01, f2& s23) {
   uint32_t cd[4];
   load_codes<BITS>(row, lane, cd);
-  const f2 ntb = dup(-tb);
-  const f2 q01 = add2(make_float2(__uint_as_float(cd[0]), __uint_as_float(cd[1])), ntb);
-  const f2 q23 = add2(make_float2(__uint_as_float(cd[2]), __uint_as_float(cd[3])), ntb);
+  f2 q01, q23;
+  codes_to_q<BITS>(cd, q01, q23);
   s01 = mul2(mul2(q01, dup(rd)), cin[0]);
   s23 = mul2(mul2(q23, dup(rd)), cin[1]);
 }
@@ -226,7 +290,7 @@ struct __align__(16) WarpRows {
   f2 irr[RPW], bb[RPW];            // refit: (1/r_i, 1/r_i), (omega_i r_i^2, same)
   float dec[RPW];                  // row retention
   float g[RPW], om[RPW];           // row gain and omega
-  float qm[RPW], iq[RPW], mb[RPW], tb[RPW];   // per-row width constants (mixed heads)
+  float qm[RPW], iq[RPW], mb[RPW];   // per-row width constants (mixed heads)
   uint32_t info[RPW];              // bits | offset << 8
   uint8_t codes[RPW * D];          // this warp's rows of packed codes
 };
@@ -245,15 +309,14 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
 }
 
 // Per-row constants of a width (2/4/6/8, 16 = pivot).
-__device__ __forceinline__ void width_consts(int bits, float& qm, float& iq, float& mb, float& tb) {
+__device__ __forceinline__ void width_consts(int bits, float& qm, float& iq, float& mb) {
   if (bits == PIVOT) {
-    qm = 0.0f; iq = 0.0f; mb = MAGIC; tb = TWO23;
+    qm = 0.0f; iq = 0.0f; mb = MAGIC;
   } else {
     const int bias = 1 << (bits - 1);
     qm = float(bias - 1);
     iq = __frcp_rn(qm);
     mb = MAGIC + float(bias);
-    tb = TWO23 + float(bias);
   }
 }
 
@@ -267,9 +330,9 @@ __device__ __forceinline__ void load_warp_rows(const PoolDev& P, int h, WarpRows
     wr.info[lane] = info;
     wr.g[lane] = P.g[h * D + i];
     wr.om[lane] = P.omega[h * D + i];
-    float qm, iq, mb, tb;
-    width_consts(row_bits(info), qm, iq, mb, tb);
-    wr.qm[lane] = qm; wr.iq[lane] = iq; wr.mb[lane] = mb; wr.tb[lane] = tb;
+    float qm, iq, mb;
+    width_consts(row_bits(info), qm, iq, mb);
+    wr.qm[lane] = qm; wr.iq[lane] = iq; wr.mb[lane] = mb;
     if (k_vec != nullptr) {
       const float dec = gate_rows != nullptr ? gate_rows[i] : gate_s;
       const float kv = k_vec[i], qv = q_vec[i];
@@ -391,6 +454,8 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
     c_own = m;
     if (lane < 16) cs.col_ic[jown] = recip_scale(c_own);
   }
+  const float c0 = c_own;
+  int wide = 0, any_wide = 0;
   __syncthreads();
 
   // --- two least-squares steps: c_j <- sum_i p y / sum_i p Q, p = b_i Q_ij -------------
@@ -450,10 +515,16 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
       const float den = __shfl_down_sync(0xffffffffu, sum, 16);
       if (lane < 16) {
         if (den > 0.0f) c_own = __fdiv_rn(sum, den);
-        cs.col_ic[jown] = recip_scale(c_own);
+        const float icn = recip_scale(c_own);
+        cs.col_ic[jown] = icn;
+        // every least-squares step keeps c >= c_before / 2 (each term Q y >= c Q^2 / 2),
+        // so |n| = |rint(y / c)| <= qmax c0 / c + 1/2 < 2^15 unless rounding at the bottom
+        // of the float32 range broke that; then the column takes the float clamp
+        if (BITS != MIXED && it == 1) wide = !(fmul(c0, icn) < 128.0f);
       }
     }
-    __syncthreads();
+    if (BITS != MIXED && it == 1) any_wide = __syncthreads_or(wide);
+    else __syncthreads();
   }
 
   // --- final codes with the final c, stored straight into the pool -------------------
@@ -464,6 +535,19 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
     ic[1] = make_float2(i4.z, i4.w);
   }
   if (lane < 16) c_global[jown] = c_own;
+  if constexpr (BITS != MIXED) {
+    if (!any_wide) {
+      constexpr float MB = MAGIC + float(1 << (BITS - 1));
+      constexpr uint32_t HI = ((1u << BITS) - 1u) * 0x00010001u;
+#pragma unroll
+      for (int rr = 0; rr < RPW; ++rr) {
+        const f2 t01 = fma2(s[rr][0], ic[0], dup(MB));
+        const f2 t23 = fma2(s[rr][1], ic[1], dup(MB));
+        store_codes_s16<BITS>(codes_global + warp_code_start + rr * (D * BITS / 8), lane, t01, t23, HI);
+      }
+      return;
+    }
+  }
 #pragma unroll
   for (int rr = 0; rr < RPW; ++rr) {
     if constexpr (BITS == MIXED) {
@@ -531,12 +615,12 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
       const uint32_t info = wr.info[rr];
       const int bits = row_bits(info);
       const uint8_t* row = wr.codes + (row_off(info) - warp_code_start);
-      const float rd = wr.rdd[rr].x, tb = wr.tb[rr];
+      const float rd = wr.rdd[rr].x;
       switch (bits) {
-        case 2: restore_row<2>(row, lane, rd, tb, cin, s[rr][0], s[rr][1]); break;
-        case 4: restore_row<4>(row, lane, rd, tb, cin, s[rr][0], s[rr][1]); break;
-        case 6: restore_row<6>(row, lane, rd, tb, cin, s[rr][0], s[rr][1]); break;
-        case 8: restore_row<8>(row, lane, rd, tb, cin, s[rr][0], s[rr][1]); break;
+        case 2: restore_row<2>(row, lane, rd, cin, s[rr][0], s[rr][1]); break;
+        case 4: restore_row<4>(row, lane, rd, cin, s[rr][0], s[rr][1]); break;
+        case 6: restore_row<6>(row, lane, rd, cin, s[rr][0], s[rr][1]); break;
+        case 8: restore_row<8>(row, lane, rd, cin, s[rr][0], s[rr][1]); break;
         default: {
           const uint2 hv = *reinterpret_cast<const uint2*>(hr.pivots + row_off(info) * D + 4 * lane);
           f2 x, y;
@@ -547,13 +631,12 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
         }
       }
     } else {
-      constexpr float TB = TWO23 + float(1 << (BITS - 1));
       uint32_t cd[4];
       load_codes<BITS>(wr.codes + rr * (D * BITS / 8), lane, cd);
       const float4 r2 = *reinterpret_cast<const float4*>(&wr.rdd[rr & ~1]);
       const f2 rd = (rr & 1) ? make_float2(r2.z, r2.w) : make_float2(r2.x, r2.y);
-      const f2 q01 = add2(make_float2(__uint_as_float(cd[0]), __uint_as_float(cd[1])), dup(-TB));
-      const f2 q23 = add2(make_float2(__uint_as_float(cd[2]), __uint_as_float(cd[3])), dup(-TB));
+      f2 q01, q23;
+      codes_to_q<BITS>(cd, q01, q23);
       s[rr][0] = mul2(mul2(q01, rd), cin[0]);
       s[rr][1] = mul2(mul2(q23, rd), cin[1]);
     }
@@ -787,9 +870,8 @@ quantize_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float
 template <int BITS>
 __device__ __forceinline__ void dequant_row(const uint8_t* row, int lane, float r, const f2 (&cin)[2],
                                             float* dst) {
-  constexpr float TB = TWO23 + float(1 << (BITS - 1));
   f2 a, b;
-  restore_row<BITS>(row, lane, r, TB, cin, a, b);
+  restore_row<BITS>(row, lane, r, cin, a, b);
   *reinterpret_cast<float4*>(dst) = make_float4(a.x, a.y, b.x, b.y);
 }
 
