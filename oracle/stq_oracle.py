@@ -335,6 +335,33 @@ def refit(S, omega, row_bits, n_ls=2):
     return u, r, c, piv
 
 
+def absmax_quantise(S, row_bits):
+    """The uniform baseline quantiser of the pages: symmetric per-key-row absmax INT-b
+    (lens, calibration and evaluation-setup paragraphs name symmetric INT4/6/8 per-row
+    absmax quantisers as the uniform comparison). Reading: the row scale is
+    r_i = max_j |S_ij| * (1/qmax_i) with 1/qmax_i rounded once (the same form as the
+    dual-axis column start), codes Q_ij = clamp(rint(S_ij * (1/r_i)), -qmax_i, qmax_i)
+    with the product taken exactly, and the column scales are all 1, so the stored pool
+    has the dual-axis layout and dequantises as (Q r) * 1. Pivot rows: float16 as in
+    `refit`.
+
+    Returns (u, r, c, piv) like `refit`."""
+    S = np.asarray(S, dtype=F32)
+    row_bits = np.asarray(row_bits)
+    pivot = row_bits == PIVOT_BITS
+    qm = qmax_of(row_bits).astype(F32)
+    inv_qm = _recip(qm)
+    m = np.max(np.abs(S), axis=-1)
+    r = np.where(pivot, F32(0), m * inv_qm).astype(F32)
+    x = S.astype(F64) * _recip(r).astype(F64)[..., :, None]   # exact product
+    Q = np.clip(np.rint(x), -qm[..., :, None], qm[..., :, None]).astype(F32)
+    u = (Q.astype(np.int64) + bias_of(row_bits)[..., None])
+    u = np.where(pivot[..., None], 0, u)
+    c = np.ones(S.shape[:-2] + (S.shape[-1],), dtype=F32)
+    piv = np.where(pivot[..., None], S, F32(0)).astype(np.float16)
+    return u, r, c, piv
+
+
 def fp32_step(S_prev, q, k, v, decay, beta):
     """One FP32-state decode step (the unquantised path the pages compare against):
     S' = D_t S_{t-1} row-wise, the gated delta update, then the readout."""
@@ -343,18 +370,22 @@ def fp32_step(S_prev, q, k, v, decay, beta):
     return S, readout(S, q)
 
 
-def decode_step(u, r, c, piv, row_bits, omega, q, k, v, decay, beta, n_ls=2):
+def decode_step(u, r, c, piv, row_bits, omega, q, k, v, decay, beta, n_ls=2, scheme="stepquant"):
     """One packed-state decode step in the order the pages give (lens decode-order
     paragraph; bloombook section 4, fused kernel paragraph): restore the previous
     state, apply the gated delta update in floating point, read the output from the
     updated float32 state, then refit and requantise for storage.
 
     decay is per key row [..., d] (GDN: the head's alpha repeated over rows).
+    scheme "stepquant" requantises with `refit`, "row_absmax" with `absmax_quantise`.
     Returns (u, r, c, piv, o, S_float32_before_requantisation)."""
     Sp = dequantize(u, r, c, piv, row_bits, decay=decay)
     S = delta_update(Sp, k, v, beta)
     o = readout(S, q)
-    u2, r2, c2, piv2 = refit(S, omega, row_bits, n_ls=n_ls)
+    if scheme == "row_absmax":
+        u2, r2, c2, piv2 = absmax_quantise(S, row_bits)
+    else:
+        u2, r2, c2, piv2 = refit(S, omega, row_bits, n_ls=n_ls)
     return u2, r2, c2, piv2, o, S
 
 
