@@ -47,8 +47,11 @@ TRAFFIC = {"bytes": None, "kernel_sha256": None, "source": None}
 
 
 def kernel_sha():
-    p = os.path.join(ROOT, "quantized_linear_attention_02_b200", "csrc", "stq_kernels.cu")
-    return hashlib.sha256(open(p, "rb").read()).hexdigest()
+    """sha256 over the sources the decode kernel is compiled from."""
+    h = hashlib.sha256()
+    for f in ("stq_device.cuh", "stq_kernels.cu", "stq_internal.h"):
+        h.update(open(os.path.join(ROOT, "quantized_linear_attention_02_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
 
 
 def peaks():

@@ -24,7 +24,7 @@ def needs_build() -> bool:
         return True
     t = os.path.getmtime(LIB)
     deps = [os.path.join(HERE, s) for s in SOURCES]
-    deps += [os.path.join(HERE, "csrc", "stq_internal.h")]
+    deps += [os.path.join(HERE, "csrc", h) for h in ("stq_internal.h", "stq_device.cuh")]
     deps += [os.path.join(ROOT, "include", "stq.h")]
     return any(os.path.getmtime(p) > t for p in deps)
 
