@@ -80,14 +80,18 @@ def algorithmic_bytes(w, B):
     return per_req * B
 
 
-def algorithmic_flops(w, B):
+def algorithmic_flops(w, B, scheme="stepquant"):
     """float32 operations the rule prescribes per step (each rounded IEEE operation
     of the oracle's definition): per quantised element 31 for GDN (restore 2, k^T S 2,
     update 2, readout 2, |S| row sum 1, y 1, column max 1, least-squares step one 7,
     step two 9 with the clamp, final code 4), one more for KDA's per-row 1/qmax in
-    the column max; per FP16 pivot element 7 (decay, k^T S, update, readout)."""
+    the column max; 13 with the row-absmax quantiser (restore, k^T S, update, readout
+    8, row max 1, code 4); per FP16 pivot element 7 (decay, k^T S, update, readout)."""
     rb = W.row_bits(w)
-    per_q = 31 + (1 if w.kind == "kda" else 0)
+    if scheme == "row_absmax":
+        per_q = 13
+    else:
+        per_q = 31 + (1 if w.kind == "kda" else 0)
     nq = int((rb != 16).sum()) * D
     npv = int((rb == 16).sum()) * D
     return B * (per_q * nq + 7 * npv)
@@ -164,7 +168,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------
 # CPU oracle timing (reported baseline only)
 # ---------------------------------------------------------------------------------
-def oracle_rate(w, budget_s=10.0, reqs=1):
+def oracle_rate(w, budget_s=10.0, reqs=1, scheme="stepquant"):
     """Head-state steps/s of the CPU oracle on one thread, timed on a sample of the
     workload (`reqs` requests x all heads per call) for about budget_s seconds."""
     try:
@@ -181,7 +185,7 @@ def oracle_rate(w, budget_s=10.0, reqs=1):
     while True:
         x = W.step_inputs(w, "decode", calls, 0, reqs)
         u, r, c, piv, o, X = O.decode_step(u, r, c, piv, rb, om, x.q, x.k, x.v,
-                                           O.gate_rows(x.gate, w.kind, D), x.beta)
+                                           O.gate_rows(x.gate, w.kind, D), x.beta, scheme=scheme)
         heads += reqs * w.H
         calls += 1
         el = time.perf_counter() - t0
@@ -290,7 +294,7 @@ def stq_arm(args, rank, world, local_rank):
     else:
         n_slots = W.n_slots(B)
         slot_ids = [W.slot_of_request(b) for b in range(B)]
-    pool = stq.Pool(w.kind, n_slots, ub, om, device=dev)
+    pool = stq.Pool(w.kind, n_slots, ub, om, device=dev, scheme=args.scheme)
     slots = torch.tensor(slot_ids, dtype=torch.int32, device=dev)
     gen = torch.Generator(device=dev).manual_seed(1000 * args.workload + rank)
 
@@ -378,7 +382,7 @@ def stq_arm(args, rank, world, local_rank):
         return
     hbm_peak, smax, which = peaks()
     nbytes = algorithmic_bytes(w, B)
-    flops = algorithmic_flops(w, B)
+    flops = algorithmic_flops(w, B, args.scheme)
     sec = ms_step * 1e-3                 # one launch per step: the step time is the launch time
     hbm_ach = nbytes / sec / 1e9
     alu_peak = SMS * FP32_LANES_PER_SM * smax * 1e6 / 1e12
@@ -397,7 +401,7 @@ def stq_arm(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": w.name, "kind": w.kind, "B": B, "H": H, "d": D,
+        "config": {"workload": w.name, "kind": w.kind, "scheme": args.scheme, "B": B, "H": H, "d": D,
                    "global_batch": B * world, "bits": {str(b): int((ub == b).sum()) for b in sorted(set(ub.tolist()))},
                    "n_slots": n_slots, "l2": "inputs larger than L2 (packed state of the active slots "
                    f"{pool.sizes['slot_code_bytes'] * B / 1e9:.2f} GB, 8 rotating input sets)",
@@ -409,7 +413,7 @@ def stq_arm(args, rank, world, local_rank):
     if drift is not None:
         line["drift"] = drift
     if world == 1 and not args.no_cpu_baseline:
-        rate, info = oracle_rate(w, budget_s=args.cpu_budget)
+        rate, info = oracle_rate(w, budget_s=args.cpu_budget, scheme=args.scheme)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, **info}
     print(json.dumps(line), flush=True)
 
@@ -422,6 +426,8 @@ def main():
     ap.add_argument("--impl", choices=["stq", "reference"], default="stq")
     ap.add_argument("--workload", type=int, default=3, help="index into the workload list (3 = GDN B=512 6-bit)")
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--scheme", choices=["stepquant", "row_absmax"], default="stepquant",
+                    help="requantisation rule (row_absmax: the pages' uniform baseline)")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-budget", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -54,6 +54,16 @@ typedef enum {
 
 typedef enum { STQ_GDN = 0, STQ_KDA = 1 } stq_kind;
 
+/* How a decode step (and stq_quantize_init) requantises the updated state.
+ *   STQ_SCHEME_STEPQUANT: the dual-axis refit r_i c_j z_ij of the method (row scale from
+ *     the row's mean magnitude and influence, column scale from two omega-weighted
+ *     least-squares steps)  [bloombook section 4; singularity-lens dual-axis paragraph].
+ *   STQ_SCHEME_ROW_ABSMAX: the pages' uniform comparison quantiser, symmetric per-key-row
+ *     absmax: r_i = max_j |S_ij| * fl(1/qmax_i), codes rint(S_ij * fl(1/r_i)), all column
+ *     scales 1  [singularity-lens calibration and evaluation-setup paragraphs].
+ * Both keep the same pool layout, widths and FP16 pivot units. */
+typedef enum { STQ_SCHEME_STEPQUANT = 0, STQ_SCHEME_ROW_ABSMAX = 1 } stq_scheme;
+
 #define STQ_D 128
 #define STQ_PIVOT_BITS 16
 
@@ -68,6 +78,7 @@ typedef struct {
                                 (one width per key row); each 2, 4, 6, 8 or 16 (FP16
                                 pivot unit) */
   const float* omega;        /* host; [H*d] row influence omega_i, finite and > 0 */
+  int scheme;                /* stq_scheme; 0 (zero-initialised) = STQ_SCHEME_STEPQUANT */
 } stq_pool_desc;
 
 /* Buffer sizes (bytes) the caller allocates for a pool, from stq_pool_layout. */

@@ -43,7 +43,7 @@ size_t up16(size_t x) { return (x + 15) & ~size_t(15); }
 
 // Host-side layout of one pool, derived from the description.
 struct HostLayout {
-  int kind = 0, n_slots = 0, H = 0;
+  int kind = 0, n_slots = 0, H = 0, scheme = 0;
   std::vector<uint32_t> head_code_off, head_code_bytes, head_piv_first, head_piv_count, head_bits;
   std::vector<uint32_t> warp_code_off;
   std::vector<uint32_t> row_info;
@@ -58,12 +58,16 @@ stq_status build_layout(const stq_pool_desc* desc, HostLayout& L) {
   if (desc->kind != STQ_GDN && desc->kind != STQ_KDA)
     return fail(STQ_ERR_INVALID_ARG, "kind must be STQ_GDN (0) or STQ_KDA (1), got %d", desc->kind);
   if (desc->d != STQ_D) return fail(STQ_ERR_INVALID_ARG, "d must be %d, got %d", STQ_D, desc->d);
+  if (desc->scheme != STQ_SCHEME_STEPQUANT && desc->scheme != STQ_SCHEME_ROW_ABSMAX)
+    return fail(STQ_ERR_INVALID_ARG,
+                "scheme must be STQ_SCHEME_STEPQUANT (0) or STQ_SCHEME_ROW_ABSMAX (1), got %d", desc->scheme);
   if (desc->n_slots <= 0) return fail(STQ_ERR_INVALID_ARG, "n_slots must be > 0, got %d", desc->n_slots);
   if (desc->H <= 0 || desc->H > (1 << 20)) return fail(STQ_ERR_INVALID_ARG, "H out of range: %d", desc->H);
   if (desc->unit_bits == nullptr || desc->omega == nullptr)
     return fail(STQ_ERR_INVALID_ARG, "unit_bits and omega must be non-NULL host arrays");
   const int H = desc->H, D = STQ_D;
   L.kind = desc->kind;
+  L.scheme = desc->scheme;
   L.n_slots = desc->n_slots;
   L.H = H;
   L.head_code_off.assign(H, 0);
@@ -238,6 +242,7 @@ stq_status stq_pool_create(const stq_pool_desc* desc, void* d_codes, void* d_sca
   dv.g = reinterpret_cast<const float*>(mb + m.g);
   dv.omega = reinterpret_cast<const float*>(mb + m.omega);
   dv.err = reinterpret_cast<uint32_t*>(mb + m.err);
+  dv.scheme = L.scheme;
   p->meta = d_meta;
   *out = p;
   return ok();

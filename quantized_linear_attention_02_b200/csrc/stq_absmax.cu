@@ -1,0 +1,139 @@
+// Decode step and state quantisation with the pages' uniform comparison quantiser:
+// symmetric per-key-row absmax INT-b (singularity-lens, calibration and
+// evaluation-setup paragraphs). The restore, gated delta update and readout are the
+// decode kernel's own (stq_device.cuh); only the quantiser that ends the step differs:
+//   r_i = max_j |S_ij| * fl(1/qmax_i),  Q_ij = clamp(rint(S_ij * fl(1/r_i)), +-qmax_i),
+//   c_j = 1,
+// so the pool keeps the dual-axis layout and dequantises as (Q r) * 1. A row scale
+// below 2^-126 counts as zero (all-zero codes), as in the method's refit.
+#include "stq_device.cuh"
+
+namespace stq {
+namespace {
+
+struct AbsmaxStore {
+  template <int BITS>
+  static __device__ __forceinline__ void store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], float* r_global,
+                                               float* c_global, uint8_t* codes_global, int warp_code_start,
+                                               float* o_global) {
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r0 = w * RPW;
+
+    // --- row maxima of |S| (exact in any order): 4 columns per lane, then a
+    // reduce-scatter over the lanes that leaves row R(l) in lane l -----------------
+    float a[RPW];
+#pragma unroll
+    for (int rr = 0; rr < RPW; ++rr)
+      a[rr] = fmaxf(fmaxf(fabsf(s[rr][0].x), fabsf(s[rr][0].y)), fmaxf(fabsf(s[rr][1].x), fabsf(s[rr][1].y)));
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const bool up = lane & 1;
+      const float send = up ? a[t] : a[t + 8];
+      const float keep = up ? a[t + 8] : a[t];
+      a[t] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 1));
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const bool up = lane & 2;
+      const float send = up ? a[t] : a[t + 4];
+      const float keep = up ? a[t + 4] : a[t];
+      a[t] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+    }
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const bool up = lane & 4;
+      const float send = up ? a[t] : a[t + 2];
+      const float keep = up ? a[t + 2] : a[t];
+      a[t] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+    }
+    {
+      const bool up = lane & 8;
+      const float send = up ? a[0] : a[1];
+      const float keep = up ? a[1] : a[0];
+      a[0] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+    }
+    a[0] = fmaxf(a[0], __shfl_xor_sync(0xffffffffu, a[0], 16));
+    {
+      const int R = ((lane & 1) << 3) | ((lane & 2) << 1) | ((lane & 4) >> 1) | ((lane & 8) >> 3);
+      float iq;
+      bool pivot = false;
+      if constexpr (BITS == MIXED) {
+        iq = wr.iq[R];
+        pivot = row_bits(wr.info[R]) == PIVOT;
+      } else {
+        iq = __frcp_rn(float((1 << (BITS - 1)) - 1));
+      }
+      const float r = pivot ? 0.0f : fmul(a[0], iq);
+      if (lane < 16) {
+        const float ir = recip_scale(r);
+        wr.irr[R] = make_float2(ir, ir);
+        r_global[r0 + R] = r;
+      }
+    }
+    if (lane < 16) c_global[16 * w + lane] = 1.0f;
+    __syncwarp();
+
+    // --- codes: x = S * (1/r_i) taken exactly, rounded in the 2^23 binade ---------
+#pragma unroll
+    for (int rr = 0; rr < RPW; ++rr) {
+      const float4 i2 = *reinterpret_cast<const float4*>(&wr.irr[rr & ~1]);
+      const f2 ir = (rr & 1) ? make_float2(i2.z, i2.w) : make_float2(i2.x, i2.y);
+      if constexpr (BITS == MIXED) {
+        const uint32_t info = wr.info[rr];
+        const int bits = row_bits(info);
+        if (bits == PIVOT) continue;
+        const float mb = wr.mb[rr], q = wr.qm[rr];
+        const f2 t01 = fma2(s[rr][0], ir, dup(mb));
+        const f2 t23 = fma2(s[rr][1], ir, dup(mb));
+        const float lo_b = mb - q, hi_b = mb + q;
+        const uint32_t t[4] = {__float_as_uint(fminf(fmaxf(t01.x, lo_b), hi_b)),
+                               __float_as_uint(fminf(fmaxf(t01.y, lo_b), hi_b)),
+                               __float_as_uint(fminf(fmaxf(t23.x, lo_b), hi_b)),
+                               __float_as_uint(fminf(fmaxf(t23.y, lo_b), hi_b))};
+        uint8_t* row = codes_global + row_off(info);
+        switch (bits) {
+          case 2: store_codes<2>(row, lane, t); break;
+          case 4: store_codes<4>(row, lane, t); break;
+          case 6: store_codes<6>(row, lane, t); break;
+          default: store_codes<8>(row, lane, t); break;
+        }
+      } else {
+        // |S_ij| * fl(1/r_i) <= qmax (1 + 2^-22), so |n| <= qmax: the 16-bit lanes hold it
+        constexpr float MB = MAGIC + float(1 << (BITS - 1));
+        constexpr uint32_t HI = ((1u << BITS) - 1u) * 0x00010001u;
+        const f2 t01 = fma2(s[rr][0], ir, dup(MB));
+        const f2 t23 = fma2(s[rr][1], ir, dup(MB));
+        store_codes_s16<BITS>(codes_global + warp_code_start + rr * (D * BITS / 8), lane, t01, t23, HI);
+      }
+    }
+
+    // --- readout from the per-warp partials the caller left in red[1][0] ------------
+    if (o_global != nullptr) {
+      __syncthreads();
+      if (w == 0) {
+        f2 lo, hi;
+        warp_tree(cs.red[1][0], lane, lo, hi);
+        *reinterpret_cast<float4*>(o_global + 4 * lane) = make_float4(lo.x, lo.y, hi.x, hi.y);
+      }
+    }
+  }
+};
+
+}  // namespace
+
+cudaError_t launch_decode_absmax(const PoolDev& P, const int32_t* slots, int B, const float* q,
+                                 const float* k, const float* v, const float* gate,
+                                 const float* beta, float* out, cudaStream_t s) {
+  if (B == 0) return cudaSuccess;
+  decode_kernel<AbsmaxStore><<<B * P.H, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_absmax(const PoolDev& P, const int32_t* slots, int B, const float* S,
+                                   cudaStream_t s) {
+  if (B == 0) return cudaSuccess;
+  quantize_kernel<AbsmaxStore><<<B * P.H, NT, 0, s>>>(P, slots, B, S);
+  return cudaGetLastError();
+}
+
+}  // namespace stq

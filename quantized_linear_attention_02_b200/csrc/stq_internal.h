@@ -13,6 +13,8 @@ namespace stq {
 
 constexpr int D = 128;           // d_k = d_v
 constexpr int PIVOT = 16;        // width marker of an FP16 pivot unit
+constexpr int SCHEME_STEPQUANT = 0;    // dual-axis refit
+constexpr int SCHEME_ROW_ABSMAX = 1;   // symmetric per-key-row absmax baseline
 
 // Error bits written by kernels into the pool's device error word.
 constexpr uint32_t ERR_SLOT_RANGE = 1u;   // a slot index was outside [0, n_slots)
@@ -43,6 +45,7 @@ struct PoolDev {
   const float* g;                   // [H*D] row gain (omega_i / mean omega)^(-1/2)
   const float* omega;               // [H*D]
   uint32_t* err;                    // [4] sticky error bits
+  int scheme;                       // SCHEME_STEPQUANT or SCHEME_ROW_ABSMAX
 };
 
 // Byte layout of the meta buffer, computed on the host.
@@ -61,6 +64,13 @@ cudaError_t launch_quantize(const PoolDev& P, const int32_t* slots, int B, const
                             cudaStream_t s);
 cudaError_t launch_dequantize(const PoolDev& P, const int32_t* slots, int B, float* S_out,
                               cudaStream_t s);
+// The same two steps with the per-key-row absmax quantiser (stq_absmax.cu);
+// launch_decode / launch_quantize forward to them for a SCHEME_ROW_ABSMAX pool.
+cudaError_t launch_decode_absmax(const PoolDev& P, const int32_t* slots, int B, const float* q,
+                                 const float* k, const float* v, const float* gate,
+                                 const float* beta, float* out, cudaStream_t s);
+cudaError_t launch_quantize_absmax(const PoolDev& P, const int32_t* slots, int B, const float* S,
+                                   cudaStream_t s);
 cudaError_t launch_fp32_step(int kind, int B, int H, float* S, const float* q,
                              const float* k, const float* v, const float* gate,
                              const float* beta, float* out, cudaStream_t s);

@@ -429,6 +429,7 @@ cudaError_t launch_decode(const PoolDev& P, const int32_t* slots, int B, const f
                           const float* k, const float* v, const float* gate,
                           const float* beta, float* out, cudaStream_t s) {
   if (B == 0) return cudaSuccess;
+  if (P.scheme == SCHEME_ROW_ABSMAX) return launch_decode_absmax(P, slots, B, q, k, v, gate, beta, out, s);
   decode_kernel<StepQuantStore><<<B * P.H, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
   return cudaGetLastError();
 }
@@ -436,6 +437,7 @@ cudaError_t launch_decode(const PoolDev& P, const int32_t* slots, int B, const f
 cudaError_t launch_quantize(const PoolDev& P, const int32_t* slots, int B, const float* S,
                             cudaStream_t s) {
   if (B == 0) return cudaSuccess;
+  if (P.scheme == SCHEME_ROW_ABSMAX) return launch_quantize_absmax(P, slots, B, S, s);
   quantize_kernel<StepQuantStore><<<B * P.H, NT, 0, s>>>(P, slots, B, S);
   return cudaGetLastError();
 }

@@ -56,16 +56,22 @@ def test_layout_matches_oracle_layout(lib, w):
     assert got["max_head_bytes"] == max(heads)
 
 
+@pytest.mark.parametrize("w", W.WORKLOADS[1:3], ids=lambda w: w.name)
+def test_absmax_scheme_keeps_the_layout(lib, w):
+    args = (w.kind, W.n_slots(w.B), W.unit_bits(w), W.omega(w))
+    assert stq.layout(*args, "row_absmax") == stq.layout(*args)
+
+
 def test_six_bit_head_size(lib):
     got = stq.layout("gdn", 1, np.array([6], np.uint8), np.ones((1, 128), np.float32))
     assert got["slot_code_bytes"] == 128 * 96        # 4 codes in 3 bytes
 
 
-@pytest.mark.parametrize("bad", ["width", "omega_zero", "omega_nan", "kind", "slots"])
+@pytest.mark.parametrize("bad", ["width", "omega_zero", "omega_nan", "kind", "slots", "scheme"])
 def test_invalid_descriptions_rejected(lib, bad):
     ub = np.full(4, 6, np.uint8)
     om = np.ones((4, 128), np.float32)
-    kind, n_slots = "gdn", 3
+    kind, n_slots, scheme = "gdn", 3, "stepquant"
     if bad == "width":
         ub[2] = 5
     elif bad == "omega_zero":
@@ -76,8 +82,10 @@ def test_invalid_descriptions_rejected(lib, bad):
         kind = 7
     elif bad == "slots":
         n_slots = 0
+    elif bad == "scheme":
+        scheme = 2
     with pytest.raises(stq.StqError) as e:
-        stq.layout(kind, n_slots, ub, om)
+        stq.layout(kind, n_slots, ub, om, scheme)
     assert e.value.status == 1
     assert lib.stq_last_error()
 

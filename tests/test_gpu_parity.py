@@ -289,3 +289,73 @@ def test_host_entry_point_matches_device_entry_point():
     pool.check()
     assert torch.equal(pool.codes, codes_dev)
     assert torch.equal(h_out, out_dev.cpu())
+
+
+# ---------------------------------------------------------------------------------
+# the uniform baseline scheme: symmetric per-key-row absmax (same kernels, other
+# quantiser)
+# ---------------------------------------------------------------------------------
+def make_absmax_pool(w, bits=None):
+    ub = W.unit_bits(w) if bits is None else np.full_like(W.unit_bits(w), bits)
+    rb = W.row_bits(w) if bits is None else np.full((w.H, D), bits)
+    return stq.Pool(w.kind, W.n_slots(w.B), ub, W.omega(w), scheme="row_absmax"), O.Layout(rb), rb
+
+
+@pytest.mark.parametrize("widx,bits", [(1, None), (2, None), (1, 6), (2, 4)])
+def test_absmax_quantize_init_matches_oracle(widx, bits):
+    w = W.WORKLOADS[widx]
+    reqs = [0, w.B - 1]
+    pool, L, rb = make_absmax_pool(w, bits)
+    S0 = T.warm_state(w.index, tuple(reqs))
+    u, r, c, piv = O.absmax_quantise(S0, rb)
+    pool.quantize_init(slots_t(reqs), dev(S0))
+    pool.check()
+    ug, rg, cg, pg = T.read_pool_state(pool, L, [W.slot_of_request(b) for b in reqs])
+    T.compare_codes(ug, u, S0, r, c, rb, "absmax quantize_init")
+    assert np.array_equal(rg, r) and np.array_equal(cg, c)
+    assert np.array_equal(pg[:, rb == 16], piv[:, rb == 16])
+
+
+@pytest.mark.parametrize("widx,t,bits", [(1, 0, None), (2, 5, None), (1, 3, 8), (2, 9, 2)])
+def test_absmax_decode_step_teacher_forced(widx, t, bits):
+    w = W.WORKLOADS[widx]
+    reqs = [0, w.B - 1]
+    pool, L, rb = make_absmax_pool(w, bits)
+    S0 = T.warm_state(w.index, tuple(reqs))
+    u, r, c, piv = O.absmax_quantise(S0, rb)
+    slots = [W.slot_of_request(b) for b in reqs]
+    T.write_oracle_state(pool, L, slots, u, r, c, piv)
+    x = T.inputs_for(w, "decode", t, reqs)
+    u2, r2, c2, p2, o, X = O.decode_step(u, r, c, piv, rb, W.omega(w), x.q, x.k, x.v,
+                                         O.gate_rows(x.gate, w.kind, D), x.beta, scheme="row_absmax")
+    out = torch.empty((len(reqs), w.H, D), device="cuda")
+    pool.decode_step(slots_t(reqs), dev(x.q), dev(x.k), dev(x.v), dev(x.gate), dev(x.beta), out)
+    pool.check()
+    ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
+    T.compare_codes(ug, u2, X, r2, c2, rb, f"absmax {w.name} step {t}")
+    assert np.array_equal(rg, r2) and np.array_equal(cg, c2)
+    assert np.array_equal(pg[:, rb == 16], p2[:, rb == 16])
+    assert T.per_vector_rel_l2(out.cpu().numpy(), o).max() <= T.OUT_REL_L2
+
+
+@pytest.mark.parametrize("widx,steps", [(1, 16), (2, 16)])
+def test_absmax_decode_chain(widx, steps):
+    w = W.WORKLOADS[widx]
+    reqs = [1, w.B - 2]
+    pool, L, rb = make_absmax_pool(w)
+    S0 = T.warm_state(w.index, tuple(reqs))
+    u, r, c, piv = O.absmax_quantise(S0, rb)
+    slots = [W.slot_of_request(b) for b in reqs]
+    T.write_oracle_state(pool, L, slots, u, r, c, piv)
+    out = torch.empty((len(reqs), w.H, D), device="cuda")
+    for t in range(steps):
+        x = T.inputs_for(w, "decode", t, reqs)
+        u, r, c, piv, o, _ = O.decode_step(u, r, c, piv, rb, W.omega(w), x.q, x.k, x.v,
+                                           O.gate_rows(x.gate, w.kind, D), x.beta, scheme="row_absmax")
+        pool.decode_step(slots_t(reqs), dev(x.q), dev(x.k), dev(x.v), dev(x.gate), dev(x.beta), out)
+        assert T.per_vector_rel_l2(out.cpu().numpy(), o).max() <= T.OUT_REL_L2, f"step {t}"
+    pool.check()
+    ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
+    S_gpu = O.dequantize(ug, rg, cg, pg, rb)
+    S_or = O.dequantize(u, r, c, piv, rb)
+    assert T.rel_l2(S_gpu, S_or) <= T.CHAIN_REL_L2
