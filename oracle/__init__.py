@@ -1,7 +1,7 @@
 """CPU oracle for the packed Delta-rule state decode step (test infrastructure).
 
 This package is the plain, slow, obviously-correct restatement of what the decode
-step computes, used only by the tests, by `__graft_entry__.smoke()` and by the
+step (and of the offline bit allocation before it), used only by the tests, by `__graft_entry__.smoke()` and by the
 `cpu_baseline` / `--impl reference` legs of `bench.py`. The library's product path
 never imports, links or runs anything here, and nothing here imports the library:
 the two share no code, tables or constants. Only the seeded input generator
@@ -24,6 +24,13 @@ Parity status per function (what pins it, see tests/test_oracle_*.py):
                             sign symmetry, rank-1 fixed point)
   decode_step               pinned (error recurrence on paired FP32 / quantised runs,
                             readout taken before requantisation, all-pivot tracking)
+  absmax_quantise           pinned (row maximum to +-qmax, half-step bound, float64
+                            textbook absmax quantiser, symmetry, hand example)
+  stq_alloc.lifetime_weight pinned (closed form of the geometric series)
+  stq_alloc.allocate        pinned (brute force over all width choices on tiny
+                            instances, pivots = riskiest units, budget limits)
+  stq_alloc.row_sq_error,
+  stq_alloc.unit_distortion pinned (float64 numpy means; distortion falls with width)
 The refit rule itself (which scales the paper's authors use) is not printed on the
 pages; the rule here is the documented build rule, so agreement with the authors'
 own quantiser is unpinned.
