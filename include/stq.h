@@ -187,6 +187,45 @@ stq_status stq_fp32_decode_step(int kind, int B, int H, int d, float* d_S,
                                 const float* d_gate, const float* d_beta, float* d_out,
                                 void* stream);
 
+/* ---- Offline calibration: the lifetime-aware width allocation that fixes a pool's
+ * unit_bits before any decode step (bloombook section 3, lifetime weight, and section 4,
+ * "time" half: budgeted allocation and FP16 pivots; singularity-lens calibration
+ * paragraph: distortion per candidate width, candidates {2,4,6,8} or {4,6,8}). The
+ * per-width distortions come from the calibration states quantised with
+ * stq_quantize_init into a pool of one uniform width and read back with
+ * stq_dequantize; stq_row_sq_error measures them. ---------------------------------- */
+
+/* Per-row squared error of n_states 128x128 float32 states against their
+ * reconstructions: e[s*128 + i] (+)= sum_j (S[s,i,j] - S_hat[s,i,j])^2, the squares of
+ * the float32 differences summed as a balanced binary tree over j. accumulate != 0 adds
+ * to d_err (float32, one rounding) instead of overwriting it. Device pointers, 16-byte
+ * aligned; n_states >= 0. Enqueued on `stream`. */
+stq_status stq_row_sq_error(const float* d_S, const float* d_S_hat, int n_states, float* d_err,
+                            int accumulate, void* stream);
+
+/* Lifetime weights L_u = sum_{j=0}^{horizon-1} exp(2 j ell_u) of n units, ell_u the
+ * unit's mean log-retention (<= 0), summed term by term in double. Host arrays. */
+stq_status stq_lifetime_weights(const double* ell, int n, int horizon, double* out);
+
+/* Distortion of each unit from the row errors of N calibration states
+ * (h_row_err [N, H, 128], from stq_row_sq_error of states quantised at one width):
+ * GDN (kind 0) one value per head, sum_n sum_i omega_i e[n,h,i] / (N 128^2);
+ * KDA (kind 1) one value per key row (h, i), sum_n e[n,h,i] / (N 128).
+ * Sequential double sums (n outer, i inner). Host arrays; out has H (GDN) or H*128
+ * (KDA) entries. */
+stq_status stq_unit_distortion(int kind, int N, int H, const float* h_row_err,
+                               const float* h_omega, double* out);
+
+/* Widths for n units: the n_pivots units with the largest lifetime[u] * dist[u, last]
+ * (ties: lower index) get STQ_PIVOT_BITS; the others minimise
+ * sum_u lifetime[u] * dist[u, c_u] subject to sum_u cand_bits[c_u] <= budget * (their
+ * count), solved exactly (dynamic program over the total width; among equal costs the
+ * narrower width, then the smaller total). cand_bits: n_cand ascending even widths from
+ * {2,4,6,8}; dist [n, n_cand] row-major. Returns STQ_ERR_INVALID_ARG for an infeasible
+ * budget or bad candidates. Host arrays; the result goes to out_bits [n]. */
+stq_status stq_allocate_bits(int n, int n_cand, const int* cand_bits, const double* lifetime,
+                             const double* dist, double budget, int n_pivots, uint8_t* out_bits);
+
 /* Synchronise `stream`, read the pool's sticky device error bits, clear them, and
  * return STQ_ERR_DEVICE_CHECK if any was set (message names the check). */
 stq_status stq_pool_check(stq_pool* pool, void* stream);

@@ -7,14 +7,15 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libstq.so")
-SOURCES = ["csrc/stq_abi.cpp", "csrc/stq_kernels.cu", "csrc/stq_absmax.cu", "csrc/stq_static_staging.cu"]
+SOURCES = ["csrc/stq_abi.cpp", "csrc/stq_kernels.cu", "csrc/stq_absmax.cu", "csrc/stq_calib.cu",
+           "csrc/stq_static_staging.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17",
     "--fmad=false",                 # products are rounded before they are added
-    "-Xcompiler", "-fPIC,-O2,-Wall",
+    "-Xcompiler", "-fPIC,-O2,-Wall,-ffp-contract=off",   # host double sums: no fused multiply-add
     "-shared",
 ]
 

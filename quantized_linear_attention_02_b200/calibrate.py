@@ -1,0 +1,63 @@
+"""Offline, lifetime-aware width allocation of a pool (the step before the decode path).
+
+The method's offline stage (bloombook section 3, lifetime weight; section 4, the "time"
+half: budgeted allocation and FP16 pivots; singularity-lens calibration paragraph):
+every unit u (GDN head, KDA key row) gets a lifetime weight L_u from its mean
+log-retention, a distortion D_u(b) for each candidate width b measured on calibration
+states, and the widths that minimise sum_u L_u D_u(b_u) under a mean-bit budget, with
+the riskiest units kept as FP16 pivots.
+
+Every step runs in the library: the calibration states are quantised at each candidate
+width by the quantise kernel (a pool of one uniform width), read back by the dequantise
+kernel, and measured by the row-error kernel; lifetime weights, unit distortions and
+the allocation are the library's host functions. This module only sequences the calls.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import stq
+
+D = stq.D
+
+CANDIDATES = {4: (2, 4, 6, 8), 6: (4, 6, 8)}   # candidate widths per nominal budget
+
+
+def measure_distortions(kind, omega, states, cand_bits, stream=None):
+    """D_u(b) for every unit and candidate: states [N, H, 128, 128] float32 on the GPU.
+    Returns [n_units, n_cand] float64 (n_units = H for GDN, H*128 for KDA)."""
+    import torch
+    N, H = states.shape[0], states.shape[1]
+    om = np.ascontiguousarray(omega, dtype=np.float32)
+    slots = torch.arange(N, dtype=torch.int32, device=states.device)
+    S_hat = torch.empty_like(states)
+    err = torch.empty(N * H * D, dtype=torch.float32, device=states.device)
+    n_units = H if kind == "gdn" else H * D
+    out = np.empty((n_units, len(cand_bits)), np.float64)
+    for ci, b in enumerate(cand_bits):
+        ub = np.full(H if kind == "gdn" else H * D, b, np.uint8)
+        pool = stq.Pool(kind, N, ub, om, device=states.device)
+        pool.quantize_init(slots, states, stream)
+        pool.dequantize(slots, S_hat, stream)
+        pool.check(stream)
+        stq.row_sq_error(states, S_hat, err, stream=stream)
+        if stream is not None:
+            stream.synchronize()
+        else:
+            torch.cuda.synchronize()
+        out[:, ci] = stq.unit_distortion(kind, err.cpu().numpy().reshape(N, H, D), om)
+        pool.close()
+    return out
+
+
+def allocate(kind, omega, states, ell_units, budget, pivot_frac=0.02, horizon=1024, cand_bits=None):
+    """Widths per unit (GDN [H], KDA [H*128]; 16 = FP16 pivot) for a nominal budget of 4
+    or 6 bits, from calibration states [N, H, 128, 128] on the GPU and each unit's mean
+    log-retention ell_units. Returns (unit_bits uint8, details dict)."""
+    cand = tuple(cand_bits) if cand_bits is not None else CANDIDATES[int(budget)]
+    dist = measure_distortions(kind, omega, states, cand)
+    ell = np.ascontiguousarray(ell_units, dtype=np.float64).reshape(-1)
+    life = stq.lifetime_weights(ell, horizon)
+    n_piv = int(round(pivot_frac * ell.size))
+    bits = stq.allocate_bits(life, dist, cand, budget, n_piv)
+    return bits, {"lifetime": life, "distortion": dist, "candidates": cand, "n_pivots": n_piv}

@@ -67,6 +67,10 @@ def lib():
         "stq_dequantize": (_i, [_vp, _vp, _i, _vp, _vp]),
         "stq_fp32_decode_step": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
         "stq_pool_check": (_i, [_vp, _vp]),
+        "stq_row_sq_error": (_i, [_vp, _vp, _i, _vp, _i, _vp]),
+        "stq_lifetime_weights": (_i, [_vp, _i, _i, _vp]),
+        "stq_unit_distortion": (_i, [_i, _i, _i, _vp, _vp, _vp]),
+        "stq_allocate_bits": (_i, [_i, _i, _vp, _vp, _vp, ctypes.c_double, _i, _vp]),
         "stq_last_error": (ctypes.c_char_p, []),
         "stq_version": (ctypes.c_char_p, []),
     }
@@ -249,3 +253,49 @@ def fp32_decode_step(kind, S, q, k, v, gate, beta, out, stream=None):
                                       _ptr(v, torch.float32, "v", n), _ptr(gate, torch.float32, "gate", ng),
                                       _ptr(beta, torch.float32, "beta", B * H),
                                       _ptr(out, torch.float32, "out", n), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------------
+# offline calibration (lifetime-aware widths); see include/stq.h
+# ---------------------------------------------------------------------------------
+def row_sq_error(S, S_hat, err, accumulate=False, stream=None):
+    """err[s*128 + i] (+)= sum_j (S - S_hat)^2 over the rows of n_states 128x128 states."""
+    import torch
+    n = S.numel() // (D * D)
+    _check(lib().stq_row_sq_error(_ptr(S, torch.float32, "S", n * D * D),
+                                  _ptr(S_hat, torch.float32, "S_hat", n * D * D), n,
+                                  _ptr(err, torch.float32, "err", n * D), int(bool(accumulate)),
+                                  _stream(stream)))
+
+
+def _host(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def lifetime_weights(ell, horizon=1024):
+    """L_u = sum_{j<horizon} exp(2 j ell_u) (host)."""
+    e = _host(ell, np.float64).reshape(-1)
+    out = np.empty_like(e)
+    _check(lib().stq_lifetime_weights(e.ctypes.data, e.size, int(horizon), out.ctypes.data))
+    return out.reshape(np.shape(ell))
+
+
+def unit_distortion(kind, row_err, omega):
+    """Per-unit distortion from row errors [N, H, 128] (host float32)."""
+    e = _host(row_err, np.float32)
+    N, H = e.shape[0], e.shape[1]
+    om = _host(omega, np.float32)
+    out = np.empty(H if KINDS[kind] == STQ_GDN else H * D, np.float64)
+    _check(lib().stq_unit_distortion(KINDS[kind], N, H, e.ctypes.data, om.ctypes.data, out.ctypes.data))
+    return out
+
+
+def allocate_bits(lifetime, dist, cand_bits, budget, n_pivots):
+    """Widths per unit (16 = FP16 pivot) minimising the lifetime-weighted distortion."""
+    L = _host(lifetime, np.float64).reshape(-1)
+    Dm = _host(dist, np.float64)
+    cb = _host(cand_bits, np.int32)
+    out = np.empty(L.size, np.uint8)
+    _check(lib().stq_allocate_bits(L.size, cb.size, cb.ctypes.data, L.ctypes.data, Dm.ctypes.data,
+                                   float(budget), int(n_pivots), out.ctypes.data))
+    return out

@@ -233,3 +233,36 @@ def torch_scale_outlier_rows(S, w: Workload):
     hh = torch.arange(w.H, device=S.device)[:, None]
     S[:, hh, torch.as_tensor(rows, device=S.device), :] *= OUTLIER_FACTOR
     return S
+
+
+# ---------------------------------------------------------------------------------
+# synthetic calibration data for the offline width allocation
+# ---------------------------------------------------------------------------------
+CALIB_JITTER = 0.1      # per-step log-retention = mean * (1 + U(-0.1, 0.1))
+
+
+def calibration_log_retention(w: Workload) -> np.ndarray:
+    """Mean log-retention of every unit in the synthetic calibration data (GDN [H],
+    KDA [H, d], float64), drawn once per unit from U(gate_low, gate_high) so that units
+    differ in memory length (half-lives ln 0.5 / l from a few steps to several
+    hundred). The pages estimate it from 32 WikiText-2 segments, which are not here."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([w.index, 7])))
+    shape = (w.H,) if w.kind == "gdn" else (w.H, w.d)
+    return rng.uniform(w.gate_low, w.gate_high, size=shape)
+
+
+def calibration_step_inputs(w: Workload, step: int, n_seq: int) -> StepInputs:
+    """Inputs of calibration step `step` for n_seq sequences: q, k, v, beta drawn as
+    decode inputs; the gate of unit u is exp(l_u (1 + e)), e ~ U(-CALIB_JITTER,
+    CALIB_JITTER) per (sequence, unit), so its mean log-retention is l_u."""
+    _, cols = outlier_sets(w)
+    ell_u = calibration_log_retention(w)
+    parts = []
+    for s in range(n_seq):
+        rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([w.index, 8, step, s])))
+        x = _draw(rng, w, 1, cols)
+        jit = rng.uniform(-CALIB_JITTER, CALIB_JITTER, size=ell_u.shape)
+        gate = np.exp(ell_u * (1.0 + jit))[None].astype(np.float32)
+        parts.append(StepInputs(x.q, x.k, x.v, gate, x.beta))
+    cat = lambda name: np.concatenate([getattr(p, name) for p in parts], axis=0)
+    return StepInputs(cat("q"), cat("k"), cat("v"), cat("gate"), cat("beta"))

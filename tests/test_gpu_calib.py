@@ -1,0 +1,89 @@
+"""GPU parity of the offline width allocation: the row-error kernel against the oracle's
+tree sums, and the whole allocation (quantise each candidate width, dequantise, measure,
+weigh by lifetime, allocate) against the oracle's pipeline on the same synthetic
+calibration states."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+from oracle import stq_alloc as A  # noqa: E402
+from oracle import stq_oracle as O  # noqa: E402
+from quantized_linear_attention_02_b200 import build, calibrate, stq  # noqa: E402
+from quantized_linear_attention_02_b200 import workload as W  # noqa: E402
+
+D = 128
+F32 = np.float32
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    build.build()
+    stq.lib()
+
+
+def dev(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def test_row_sq_error_bit_exact_and_accumulate():
+    rng = np.random.default_rng(0)
+    S = rng.standard_normal((5, 3, D, D)).astype(F32)
+    Sh = (S + rng.standard_normal(S.shape).astype(F32) * F32(0.03)).astype(F32)
+    err = torch.empty(5 * 3 * D, device="cuda")
+    stq.row_sq_error(dev(S), dev(Sh), err)
+    ref = A.row_sq_error(S, Sh).reshape(-1)
+    assert np.array_equal(err.cpu().numpy(), ref)
+    stq.row_sq_error(dev(S), dev(S * F32(0.5)), err, accumulate=True)
+    ref2 = (ref + A.row_sq_error(S, S * F32(0.5)).reshape(-1)).astype(F32)
+    torch.cuda.synchronize()
+    assert np.array_equal(err.cpu().numpy(), ref2)
+
+
+def _calibration_states(w, n_seq, steps):
+    """FP32 runs from zero over the synthetic calibration inputs: oracle on the CPU and
+    the FP32 step kernel on the GPU (bit-exact with each other)."""
+    S = np.zeros((n_seq, w.H, D, D), F32)
+    Sg = torch.zeros((n_seq, w.H, D, D), device="cuda")
+    out = torch.empty((n_seq, w.H, D), device="cuda")
+    for t in range(steps):
+        x = W.calibration_step_inputs(w, t, n_seq)
+        S, _ = O.fp32_step(S, x.q, x.k, x.v, O.gate_rows(x.gate, w.kind, D), x.beta)
+        stq.fp32_decode_step(w.kind, Sg, dev(x.q), dev(x.k), dev(x.v), dev(x.gate), dev(x.beta), out)
+    torch.cuda.synchronize()
+    assert np.array_equal(Sg.cpu().numpy(), S)
+    return S, Sg
+
+
+@pytest.mark.parametrize("widx,budget,n_seq,steps", [(1, 6, 4, 32), (1, 4, 4, 32), (2, 4, 2, 24)])
+def test_allocation_pipeline_matches_oracle(widx, budget, n_seq, steps):
+    w = W.WORKLOADS[widx]
+    om = W.omega(w)
+    ell = W.calibration_log_retention(w)
+    S, Sg = _calibration_states(w, n_seq, steps)
+    bits, info = calibrate.allocate(w.kind, om, Sg, ell, budget, pivot_frac=0.02)
+    cand = calibrate.CANDIDATES[budget]
+    # the oracle's pipeline on the same states
+    dist = np.empty((w.n_units, len(cand)))
+    for ci, b in enumerate(cand):
+        rb = np.full((w.H, D), b)
+        u, r, c, piv = O.refit(S, om, rb)
+        e = A.row_sq_error(S, O.dequantize(u, r, c, piv, rb))
+        dist[:, ci] = A.unit_distortion(w.kind, e, om)
+    # codes may differ by one at a rounding boundary (at most 1e-5 of them), so the
+    # distortions agree to rounding, not bit for bit
+    assert np.allclose(info["distortion"], dist, rtol=1e-4, atol=0)
+    life = A.lifetime_weight(ell.reshape(-1))
+    ref = A.allocate(life, info["distortion"], cand, budget, info["n_pivots"])
+    assert np.array_equal(bits.astype(np.int64), ref)
+    ref_or = A.allocate(life, dist, cand, budget, info["n_pivots"])
+    assert np.mean(bits.astype(np.int64) == ref_or) >= 0.99
+    # the allocation spends the budget on the units that keep errors longest
+    rest = bits != 16
+    assert bits[rest].astype(int).mean() <= budget
+    lo = np.argsort(life)[: life.size // 4]
+    hi = np.argsort(life)[-life.size // 4:]
+    assert bits[hi][bits[hi] != 16].mean() >= bits[lo][bits[lo] != 16].mean()
