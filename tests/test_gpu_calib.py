@@ -87,3 +87,28 @@ def test_allocation_pipeline_matches_oracle(widx, budget, n_seq, steps):
     lo = np.argsort(life)[: life.size // 4]
     hi = np.argsort(life)[-life.size // 4:]
     assert bits[hi][bits[hi] != 16].mean() >= bits[lo][bits[lo] != 16].mean()
+
+
+@pytest.mark.parametrize("widx", [1, 2])
+def test_error_lifetime_diagnostic_matches_oracle(widx):
+    """A short paired run (FP32 vs uniform INT6 absmax, shared inputs): the GPU's
+    accumulated per-unit squared state error equals the oracle's to chain tolerance."""
+    from quantized_linear_attention_02_b200 import diagnostics
+    w = W.WORKLOADS[widx]
+    n_seq, steps = 2, 8
+    r = diagnostics.error_lifetime(w, n_seq=n_seq, steps=steps, bits=6)
+    rb = np.full((w.H, D), 6)
+    S = np.zeros((n_seq, w.H, D, D), F32)
+    u, rr, c, piv = O.absmax_quantise(S, rb)
+    acc = np.zeros((n_seq, w.H, D), F32)
+    for t in range(steps):
+        x = W.calibration_step_inputs(w, t, n_seq)
+        dec = O.gate_rows(x.gate, w.kind, D)
+        u, rr, c, piv, _, _ = O.decode_step(u, rr, c, piv, rb, W.omega(w), x.q, x.k, x.v, dec, x.beta,
+                                            scheme="row_absmax")
+        S, _ = O.fp32_step(S, x.q, x.k, x.v, dec, x.beta)
+        acc = (acc + A.row_sq_error(O.dequantize(u, rr, c, piv, rb), S)).astype(F32)
+    rows = acc.astype(np.float64).sum(axis=0)
+    err = rows.sum(axis=1) if w.kind == "gdn" else rows.reshape(-1)
+    assert np.allclose(r["accumulated_sq_error"], err, rtol=1e-3, atol=1e-30)
+    assert np.allclose(r["half_life"], np.log(0.5) / W.calibration_log_retention(w).reshape(-1))
