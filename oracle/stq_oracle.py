@@ -343,7 +343,7 @@ def absmax_quantise(S, row_bits):
     dual-axis column start), codes Q_ij = clamp(rint(S_ij * (1/r_i)), -qmax_i, qmax_i)
     with the product taken exactly, and the column scales are all 1, so the stored pool
     has the dual-axis layout and dequantises as (Q r) * 1. Pivot rows: float16 as in
-    `refit`.
+    `refit`; a head whose rows are all pivots stores r = c = 0 as under `refit`.
 
     Returns (u, r, c, piv) like `refit`."""
     S = np.asarray(S, dtype=F32)
@@ -357,7 +357,10 @@ def absmax_quantise(S, row_bits):
     Q = np.clip(np.rint(x), -qm[..., :, None], qm[..., :, None]).astype(F32)
     u = (Q.astype(np.int64) + bias_of(row_bits)[..., None])
     u = np.where(pivot[..., None], 0, u)
-    c = np.ones(S.shape[:-2] + (S.shape[-1],), dtype=F32)
+    # unit column scales; a head without any quantised row stores c = 0, like its r
+    has_codes = np.any(~pivot, axis=-1)
+    c = np.broadcast_to(np.where(has_codes, F32(1), F32(0))[..., None],
+                        S.shape[:-2] + (S.shape[-1],)).astype(F32)
     piv = np.where(pivot[..., None], S, F32(0)).astype(np.float16)
     return u, r, c, piv
 

@@ -123,3 +123,11 @@ def test_decode_step_readout_does_not_depend_on_the_scheme():
     b = O.decode_step(u, r, c, piv, rb, om, q, k, v, dec, beta, scheme="row_absmax")
     assert np.array_equal(a[4], b[4]) and np.array_equal(a[5], b[5])
     assert np.array_equal(b[0], O.absmax_quantise(b[5], rb)[0])
+
+
+def test_absmax_all_pivot_head_stores_zero_scales():
+    S = np.random.default_rng(60).standard_normal((1, 2, 128, 128)).astype(F32)
+    rb = np.full((2, 128), 6)
+    rb[1] = 16
+    u, r, c, piv = O.absmax_quantise(S, rb)
+    assert np.all(c[0, 0] == 1) and np.all(c[0, 1] == 0) and np.all(r[0, 1] == 0)
