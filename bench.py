@@ -41,9 +41,13 @@ FALLBACK_HBM_GBS = 6650.0
 SMS = 148
 FP32_LANES_PER_SM = 128
 
-# ncu dram bytes (read + write) per launch of decode_kernel on the default workload,
-# and the sha256 of the kernel source they were taken with (a changed kernel voids them).
-TRAFFIC = {"bytes": None, "kernel_sha256": None, "source": None}
+# ncu dram bytes (read + write) per launch of decode_kernel on the default workload
+# (GDN B = 512, dual-axis refit), and the sha256 of the kernel sources they were taken
+# with (a changed kernel voids them).
+TRAFFIC = {"bytes": 2 * (193_313_792 + 124_232_960),
+           "kernel_sha256": "88937c4bbce30c2ee12ffde164e3d36b7a5bbc1c98287cd3d092d577967838cd",
+           "source": "profiles/decode_kernel_gdn_b256_h48_nominal6.md: dram read + write of one "
+                     "B = 256 launch, doubled for B = 512 (traffic grows with B)"}
 
 
 def kernel_sha():
@@ -168,6 +172,74 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------
 # CPU oracle timing (reported baseline only)
 # ---------------------------------------------------------------------------------
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _oracle_worker(args):
+    """One process of the all-cores oracle timing: decode steps of one request over a
+    shard of the heads for about budget_s seconds (one BLAS thread)."""
+    widx, heads, budget_s, scheme = args
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(limits=1)
+    except Exception:  # pragma: no cover
+        pass
+    from oracle import stq_oracle as O
+    w = W.WORKLOADS[widx]
+    sub = np.asarray(heads)
+    rb, om = W.row_bits(w)[sub], W.omega(w)[sub]
+    rng = np.random.default_rng(int(sub[0]))
+    S = (rng.standard_normal((1, sub.size, D, D)) * 0.1).astype(np.float32)
+    u, r, c, piv = O.refit(S, om, rb)
+    n, t0, calls = 0, time.perf_counter(), 0
+    while True:
+        x = W.step_inputs(w, "decode", calls, 0, 1)
+        u, r, c, piv, o, X = O.decode_step(u, r, c, piv, rb, om, x.q[:, sub], x.k[:, sub], x.v[:, sub],
+                                           O.gate_rows(x.gate[:, sub], w.kind, D), x.beta[:, sub],
+                                           scheme=scheme)
+        n += sub.size
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            return n, el
+
+
+def oracle_rate_all_cores(w, budget_s=10.0, scheme="stepquant"):
+    """Head-state steps/s of the oracle on every host core: one spawned process per core,
+    each on its own shard of one request's heads (processes are spawned, never forked
+    from a process that has used the GPU)."""
+    import multiprocessing as mp
+    cores = len(os.sched_getaffinity(0))
+    n = max(1, min(cores, w.H))
+    shards = [list(range(w.H))[i::n] for i in range(n)]
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(n) as pool:
+        res = pool.map(_oracle_worker, [(w.index, sh, budget_s, scheme) for sh in shards])
+    heads = sum(r[0] for r in res)
+    el = max(r[1] for r in res)
+    return heads / el, {"cores": n, "sample": f"{n} processes, each one request x {len(shards[0])} "
+                                               f"heads of {w.name}, {el:.1f} s"}
+
+
+def oracle_quantize_rate(w, budget_s=3.0):
+    """Head-states/s of the oracle's quantiser alone (one thread)."""
+    from oracle import stq_oracle as O
+    rb, om = W.row_bits(w), W.omega(w)
+    S = (np.random.default_rng(1).standard_normal((1, w.H, D, D)) * 0.1).astype(np.float32)
+    n, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        O.refit(S, om, rb)
+        n += w.H
+    return n / (time.perf_counter() - t0)
+
+
 def oracle_rate(w, budget_s=10.0, reqs=1, scheme="stepquant"):
     """Head-state steps/s of the CPU oracle on one thread, timed on a sample of the
     workload (`reqs` requests x all heads per call) for about budget_s seconds."""
@@ -387,7 +459,10 @@ def stq_arm(args, rank, world, local_rank):
     hbm_ach = nbytes / sec / 1e9
     alu_peak = SMS * FP32_LANES_PER_SM * smax * 1e6 / 1e12
     alu_ach = flops / sec / 1e12
-    traffic = TRAFFIC["bytes"] if TRAFFIC["kernel_sha256"] == kernel_sha() else None
+    traffic = None      # counters exist for the default workload and the current kernel only
+    if (TRAFFIC["kernel_sha256"] == kernel_sha() and w.index == 3 and B == 512
+            and args.scheme == "stepquant"):
+        traffic = TRAFFIC["bytes"]
     hbm = {"bound": "hbm", "achieved": hbm_ach, "peak": hbm_peak, "unit": "GB/s",
            "frac": hbm_ach / hbm_peak, "traffic": traffic, "peak_source": which,
            "algorithmic_bytes_per_launch": nbytes}
@@ -414,7 +489,13 @@ def stq_arm(args, rank, world, local_rank):
         line["drift"] = drift
     if world == 1 and not args.no_cpu_baseline:
         rate, info = oracle_rate(w, budget_s=args.cpu_budget, scheme=args.scheme)
-        line["cpu_baseline"] = {"value": rate, "unit": UNIT, **info}
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, **info, "cpu": cpu_model()}
+        if not args.no_cpu_all_cores:
+            rate_all, info_all = oracle_rate_all_cores(w, budget_s=args.cpu_budget, scheme=args.scheme)
+            line["cpu_baseline"]["all_cores"] = {"value": rate_all, "unit": UNIT, **info_all}
+        if args.scheme == "stepquant":
+            line["cpu_baseline"]["quantize_only"] = {"value": oracle_quantize_rate(w), "unit": "head-states/s",
+                                                     "cores": 1}
     print(json.dumps(line), flush=True)
 
 
@@ -431,6 +512,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-budget", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-cpu-all-cores", action="store_true", help="skip the all-cores oracle timing")
     ap.add_argument("--drift-steps", type=int, default=0,
                     help="after timing, chain this many steps on 64 requests against the FP32 state")
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling captures only)")
