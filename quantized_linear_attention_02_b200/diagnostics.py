@@ -30,13 +30,17 @@ from . import workload as W
 D = stq.D
 
 
-def error_lifetime(w, n_seq=4, steps=2046, bits=6, scheme="row_absmax", device="cuda"):
-    """Returns dict with per-unit half-life, accumulated squared error and Spearman rho."""
+def error_lifetime(w, n_seq=4, steps=2046, bits=6, scheme="row_absmax", device="cuda", unit_bits=None,
+                   first_seq=0):
+    """Returns dict with per-unit half-life, accumulated squared error and Spearman rho.
+    unit_bits (GDN [H], KDA [H*128]) overrides the uniform width `bits`; the runs use
+    calibration sequences first_seq .. first_seq + n_seq - 1."""
     import torch
     from scipy.stats import spearmanr
     H = w.H
     n_units = H if w.kind == "gdn" else H * D
-    pool = stq.Pool(w.kind, n_seq, np.full(n_units, bits, np.uint8), W.omega(w), device=device, scheme=scheme)
+    ub = np.full(n_units, bits, np.uint8) if unit_bits is None else np.asarray(unit_bits, np.uint8)
+    pool = stq.Pool(w.kind, n_seq, ub, W.omega(w), device=device, scheme=scheme)
     slots = torch.arange(n_seq, dtype=torch.int32, device=device)
     S = torch.zeros((n_seq, H, D, D), device=device)
     pool.quantize_init(slots, S)
@@ -45,7 +49,7 @@ def error_lifetime(w, n_seq=4, steps=2046, bits=6, scheme="row_absmax", device="
     o_q = torch.empty((n_seq, H, D), device=device)
     o_f = torch.empty_like(o_q)
     for t in range(steps):
-        x = W.calibration_step_inputs(w, t, n_seq)
+        x = W.calibration_step_inputs(w, t, n_seq, first_seq)
         q, k, v, g, b = (torch.from_numpy(a).to(device) for a in (x.q, x.k, x.v, x.gate, x.beta))
         pool.decode_step(slots, q, k, v, g, b, o_q)
         stq.fp32_decode_step(w.kind, S, q, k, v, g, b, o_f)

@@ -251,14 +251,15 @@ def calibration_log_retention(w: Workload) -> np.ndarray:
     return rng.uniform(w.gate_low, w.gate_high, size=shape)
 
 
-def calibration_step_inputs(w: Workload, step: int, n_seq: int) -> StepInputs:
-    """Inputs of calibration step `step` for n_seq sequences: q, k, v, beta drawn as
-    decode inputs; the gate of unit u is exp(l_u (1 + e)), e ~ U(-CALIB_JITTER,
-    CALIB_JITTER) per (sequence, unit), so its mean log-retention is l_u."""
+def calibration_step_inputs(w: Workload, step: int, n_seq: int, first_seq: int = 0) -> StepInputs:
+    """Inputs of calibration step `step` for sequences first_seq .. first_seq + n_seq - 1:
+    q, k, v, beta drawn as decode inputs; the gate of unit u is exp(l_u (1 + e)),
+    e ~ U(-CALIB_JITTER, CALIB_JITTER) per (sequence, unit), so its mean log-retention
+    is l_u."""
     _, cols = outlier_sets(w)
     ell_u = calibration_log_retention(w)
     parts = []
-    for s in range(n_seq):
+    for s in range(first_seq, first_seq + n_seq):
         rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([w.index, 8, step, s])))
         x = _draw(rng, w, 1, cols)
         jit = rng.uniform(-CALIB_JITTER, CALIB_JITTER, size=ell_u.shape)
