@@ -243,6 +243,9 @@ stq_status stq_pool_create(const stq_pool_desc* desc, void* d_codes, void* d_sca
   dv.omega = reinterpret_cast<const float*>(mb + m.omega);
   dv.err = reinterpret_cast<uint32_t*>(mb + m.err);
   dv.scheme = L.scheme;
+  dv.any_mixed = 0;
+  for (int h = 0; h < L.H; ++h)
+    if (L.head_bits[h] == 0) dv.any_mixed = 1;
   p->meta = d_meta;
   *out = p;
   return ok();

@@ -125,7 +125,10 @@ cudaError_t launch_decode_absmax(const PoolDev& P, const int32_t* slots, int B, 
                                  const float* k, const float* v, const float* gate,
                                  const float* beta, float* out, cudaStream_t s) {
   if (B == 0) return cudaSuccess;
-  decode_kernel<AbsmaxStore><<<B * P.H, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+  if (P.any_mixed)
+    decode_kernel<AbsmaxStore, true><<<B * P.H, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+  else
+    decode_kernel<AbsmaxStore, false><<<B * P.H, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
   return cudaGetLastError();
 }
 

@@ -287,6 +287,7 @@ struct __align__(16) CtaSmem {
   float col_ic[D];                 // 1/c_j of the current column scale, from its owner
   float col_delta[D];              // delta_j = beta (v_j - u_j), from its owner
   WarpRows wr[NW];
+  uint32_t tail[4];                // the last warp's last row may read one word past its codes
 };
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -366,10 +367,23 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
       const uint8_t* row = wr.codes + (row_off(info) - warp_code_start);
       const float rd = wr.rdd[rr].x;
       switch (bits) {
-        case 2: restore_row<2>(row, lane, rd, cin, s[rr][0], s[rr][1]); break;
-        case 4: restore_row<4>(row, lane, rd, cin, s[rr][0], s[rr][1]); break;
-        case 6: restore_row<6>(row, lane, rd, cin, s[rr][0], s[rr][1]); break;
-        case 8: restore_row<8>(row, lane, rd, cin, s[rr][0], s[rr][1]); break;
+        case 2: case 4: case 6: case 8: {
+          // any width b: the lane's 4b bits start at bit 4 b l of the row; the word after
+          // them is inside the staging area (the next row, the next warp's rows or `tail`)
+          const uint32_t* wp = reinterpret_cast<const uint32_t*>(row);
+          const int bitpos = 4 * bits * lane;
+          const uint32_t f = __funnelshift_r(wp[bitpos >> 5], wp[(bitpos >> 5) + 1], bitpos & 31);
+          const uint32_t M = (1u << bits) - 1u;
+          // 2^23 + bias as a float: the bias sits in the mantissa
+          const f2 ntb = dup(-__uint_as_float(FLOAT_2P23 | (1u << (bits - 1))));
+          const f2 q01 = add2(make_float2(__uint_as_float((f & M) | FLOAT_2P23),
+                                          __uint_as_float(((f >> bits) & M) | FLOAT_2P23)), ntb);
+          const f2 q23 = add2(make_float2(__uint_as_float(((f >> (2 * bits)) & M) | FLOAT_2P23),
+                                          __uint_as_float(((f >> (3 * bits)) & M) | FLOAT_2P23)), ntb);
+          s[rr][0] = mul2(mul2(q01, dup(rd)), cin[0]);
+          s[rr][1] = mul2(mul2(q23, dup(rd)), cin[1]);
+          break;
+        }
         default: {
           const uint2 hv = *reinterpret_cast<const uint2*>(hr.pivots + row_off(info) * D + 4 * lane);
           f2 x, y;
@@ -511,7 +525,7 @@ __device__ __forceinline__ void decode_pivot_warp(CtaSmem& cs, WarpRows& wr, con
 // warp stages its own 16 rows (asynchronous 16-byte copies) and writes its own codes
 // back, so the CTA synchronises only for the five column exchanges.
 // ---------------------------------------------------------------------------------
-template <class Store>
+template <class Store, bool kMixed>
 __global__ void __launch_bounds__(NT, 2)
 decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* __restrict__ q,
               const float* __restrict__ k, const float* __restrict__ v,
@@ -550,7 +564,10 @@ decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* 
     case 6: decode_warp<6, Store>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
     case 8: decode_warp<8, Store>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
     case PIVOT: decode_pivot_warp(cs, wr, hr, v_own, beta_s, o_out); break;
-    default: decode_warp<MIXED, Store>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
+    default:
+      // heads whose rows have different widths (only pools with such heads launch this)
+      if constexpr (kMixed) decode_warp<MIXED, Store>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out);
+      break;
   }
 }
 

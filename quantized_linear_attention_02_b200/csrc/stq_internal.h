@@ -46,6 +46,7 @@ struct PoolDev {
   const float* omega;               // [H*D]
   uint32_t* err;                    // [4] sticky error bits
   int scheme;                       // SCHEME_STEPQUANT or SCHEME_ROW_ABSMAX
+  int any_mixed;                    // 1 if some head's rows have different widths
 };
 
 // Byte layout of the meta buffer, computed on the host.

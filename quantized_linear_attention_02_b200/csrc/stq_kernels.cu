@@ -430,7 +430,10 @@ cudaError_t launch_decode(const PoolDev& P, const int32_t* slots, int B, const f
                           const float* beta, float* out, cudaStream_t s) {
   if (B == 0) return cudaSuccess;
   if (P.scheme == SCHEME_ROW_ABSMAX) return launch_decode_absmax(P, slots, B, q, k, v, gate, beta, out, s);
-  decode_kernel<StepQuantStore><<<B * P.H, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+  if (P.any_mixed)
+    decode_kernel<StepQuantStore, true><<<B * P.H, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+  else
+    decode_kernel<StepQuantStore, false><<<B * P.H, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
   return cudaGetLastError();
 }
 
