@@ -188,11 +188,12 @@ class Pool:
     """Host image of a state pool: codes [n_slots, slot_code_bytes] uint8,
     scales [n_slots, H, 2, d] float32, pivots [n_slots, n_pivot_rows, d] float16."""
 
-    def __init__(self, layout: Layout, n_slots: int):
+    def __init__(self, layout: Layout, n_slots: int, scale16: bool = False):
         self.layout = layout
         self.n_slots = n_slots
         self.codes = np.zeros((n_slots, layout.slot_code_bytes), dtype=np.uint8)
-        self.scales = np.zeros((n_slots, layout.H, 2, layout.d), dtype=F32)
+        # compact pools keep r and c as float16 (values already float16-representable)
+        self.scales = np.zeros((n_slots, layout.H, 2, layout.d), dtype=np.float16 if scale16 else F32)
         self.pivots = np.zeros((n_slots, max(layout.n_pivot_rows, 0), layout.d), dtype=np.float16)
 
     def write_heads(self, slots, u, r, c, piv):
@@ -226,8 +227,8 @@ class Pool:
                     else:
                         o = L.row_code_offset[h, i]
                         u[bi, h, i] = unpack_row(self.codes[s, o:o + L.code_len[h, i]], b, L.d)
-        r = self.scales[list(slots), :, 0].copy()
-        c = self.scales[list(slots), :, 1].copy()
+        r = self.scales[list(slots), :, 0].astype(F32)
+        c = self.scales[list(slots), :, 1].astype(F32)
         return u, r, c, piv
 
 
@@ -298,12 +299,23 @@ def _recip(a):
     return np.where(ok, F32(1) / safe, F32(0)).astype(F32)
 
 
-def refit(S, omega, row_bits, n_ls=2):
+def _half(x):
+    """Round float32 values to IEEE binary16 (to nearest, ties to even) and back."""
+    return np.asarray(x, dtype=F32).astype(np.float16).astype(F32)
+
+
+def refit(S, omega, row_bits, n_ls=2, scale16=False):
     """Dual-axis refit of a float32 state and its codes (bloombook section 4,
     X_ij = r_i c_j z_ij with an omega-weighted column fit; lens dual-axis paragraph;
     ai-trend Method (2)).
 
     S [..., d, d] float32; omega [H, d] float32 (> 0); row_bits [H, d].
+    scale16: compact storage of the scales as binary16 (reading: r is rounded to
+    binary16 as soon as it is formed, so y, the weights and the codes use the stored r;
+    the column start and both least-squares steps run in float32; the final c is
+    rounded to binary16 before the codes are requantised with it, so the stored
+    (r, c, Q) stay consistent).
+
     Returns (u biased codes int64 [..., d, d], r [..., d], c [..., d],
     piv float16 [..., d, d] (meaningful on pivot rows only))."""
     S = np.asarray(S, dtype=F32)
@@ -316,6 +328,8 @@ def refit(S, omega, row_bits, n_ls=2):
     # row scale: mean |S_ij| over the row times g_i (division by d is exact)
     m = tree_sum(np.abs(S), axis=-1) * F32(1.0 / d)
     r = np.where(pivot, F32(0), m * g).astype(F32)
+    if scale16:
+        r = _half(r)
     inv_r = _recip(r)
     y = S * inv_r[..., :, None]
     # column scale start: no element clips
@@ -328,6 +342,8 @@ def refit(S, omega, row_bits, n_ls=2):
         den = tree_dot(p, Q, axis=-2)
         safe = np.where(den > 0, den, F32(1))
         c = np.where(den > 0, num / safe, c).astype(F32)
+    if scale16:
+        c = _half(c)
     Q = _quantise(y, _recip(c), qm)
     u = (Q.astype(np.int64) + bias_of(row_bits)[..., None])
     u = np.where(pivot[..., None], 0, u)
@@ -335,7 +351,7 @@ def refit(S, omega, row_bits, n_ls=2):
     return u, r, c, piv
 
 
-def absmax_quantise(S, row_bits):
+def absmax_quantise(S, row_bits, scale16=False):
     """The uniform baseline quantiser of the pages: symmetric per-key-row absmax INT-b
     (lens, calibration and evaluation-setup paragraphs name symmetric INT4/6/8 per-row
     absmax quantisers as the uniform comparison). Reading: the row scale is
@@ -353,6 +369,8 @@ def absmax_quantise(S, row_bits):
     inv_qm = _recip(qm)
     m = np.max(np.abs(S), axis=-1)
     r = np.where(pivot, F32(0), m * inv_qm).astype(F32)
+    if scale16:        # compact scales: the codes are fitted to the stored binary16 r
+        r = _half(r)
     x = S.astype(F64) * _recip(r).astype(F64)[..., :, None]   # exact product
     Q = np.clip(np.rint(x), -qm[..., :, None], qm[..., :, None]).astype(F32)
     u = (Q.astype(np.int64) + bias_of(row_bits)[..., None])
@@ -373,22 +391,24 @@ def fp32_step(S_prev, q, k, v, decay, beta):
     return S, readout(S, q)
 
 
-def decode_step(u, r, c, piv, row_bits, omega, q, k, v, decay, beta, n_ls=2, scheme="stepquant"):
+def decode_step(u, r, c, piv, row_bits, omega, q, k, v, decay, beta, n_ls=2, scheme="stepquant",
+                scale16=False):
     """One packed-state decode step in the order the pages give (lens decode-order
     paragraph; bloombook section 4, fused kernel paragraph): restore the previous
     state, apply the gated delta update in floating point, read the output from the
     updated float32 state, then refit and requantise for storage.
 
     decay is per key row [..., d] (GDN: the head's alpha repeated over rows).
-    scheme "stepquant" requantises with `refit`, "row_absmax" with `absmax_quantise`.
+    scheme "stepquant" requantises with `refit`, "row_absmax" with `absmax_quantise`;
+    scale16 stores the scales as binary16.
     Returns (u, r, c, piv, o, S_float32_before_requantisation)."""
     Sp = dequantize(u, r, c, piv, row_bits, decay=decay)
     S = delta_update(Sp, k, v, beta)
     o = readout(S, q)
     if scheme == "row_absmax":
-        u2, r2, c2, piv2 = absmax_quantise(S, row_bits)
+        u2, r2, c2, piv2 = absmax_quantise(S, row_bits, scale16=scale16)
     else:
-        u2, r2, c2, piv2 = refit(S, omega, row_bits, n_ls=n_ls)
+        u2, r2, c2, piv2 = refit(S, omega, row_bits, n_ls=n_ls, scale16=scale16)
     return u2, r2, c2, piv2, o, S
 
 
