@@ -69,16 +69,16 @@ def peaks():
 # ---------------------------------------------------------------------------------
 # algorithmic counts per step
 # ---------------------------------------------------------------------------------
-def algorithmic_bytes(w, B):
+def algorithmic_bytes(w, B, scale_bits=32):
     """Bytes a decode step must move: every head's packed codes (or FP16 pivot rows)
     read and written, its scales r[128], c[128] read and written (heads with any
-    quantised row), q, k, v, gate, beta read and o written."""
+    quantised row; 4 or 2 bytes each), q, k, v, gate, beta read and o written."""
     rb = W.row_bits(w).astype(np.int64)
     per_req = 0
     for h in range(w.H):
         piv = rb[h] == 16
         codes = int((D * rb[h][~piv] // 8).sum()) + int(piv.sum()) * D * 2
-        scales = 2 * D * 4 if (~piv).any() else 0
+        scales = 2 * D * (scale_bits // 8) if (~piv).any() else 0
         per_req += 2 * (codes + scales)
         per_req += 3 * D * 4 + (4 if w.kind == "gdn" else D * 4) + 4 + D * 4
     return per_req * B
@@ -366,7 +366,7 @@ def stq_arm(args, rank, world, local_rank):
     else:
         n_slots = W.n_slots(B)
         slot_ids = [W.slot_of_request(b) for b in range(B)]
-    pool = stq.Pool(w.kind, n_slots, ub, om, device=dev, scheme=args.scheme)
+    pool = stq.Pool(w.kind, n_slots, ub, om, device=dev, scheme=args.scheme, scale_bits=args.scale_bits)
     slots = torch.tensor(slot_ids, dtype=torch.int32, device=dev)
     gen = torch.Generator(device=dev).manual_seed(1000 * args.workload + rank)
 
@@ -453,7 +453,7 @@ def stq_arm(args, rank, world, local_rank):
     if rank != 0:
         return
     hbm_peak, smax, which = peaks()
-    nbytes = algorithmic_bytes(w, B)
+    nbytes = algorithmic_bytes(w, B, args.scale_bits)
     flops = algorithmic_flops(w, B, args.scheme)
     sec = ms_step * 1e-3                 # one launch per step: the step time is the launch time
     hbm_ach = nbytes / sec / 1e9
@@ -461,7 +461,7 @@ def stq_arm(args, rank, world, local_rank):
     alu_ach = flops / sec / 1e12
     traffic = None      # counters exist for the default workload and the current kernel only
     if (TRAFFIC["kernel_sha256"] == kernel_sha() and w.index == 3 and B == 512
-            and args.scheme == "stepquant"):
+            and args.scheme == "stepquant" and args.scale_bits == 32):
         traffic = TRAFFIC["bytes"]
     hbm = {"bound": "hbm", "achieved": hbm_ach, "peak": hbm_peak, "unit": "GB/s",
            "frac": hbm_ach / hbm_peak, "traffic": traffic, "peak_source": which,
@@ -476,7 +476,8 @@ def stq_arm(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": w.name, "kind": w.kind, "scheme": args.scheme, "B": B, "H": H, "d": D,
+        "config": {"workload": w.name, "kind": w.kind, "scheme": args.scheme, "scale_bits": args.scale_bits,
+                   "B": B, "H": H, "d": D,
                    "global_batch": B * world, "bits": {str(b): int((ub == b).sum()) for b in sorted(set(ub.tolist()))},
                    "n_slots": n_slots, "l2": "inputs larger than L2 (packed state of the active slots "
                    f"{pool.sizes['slot_code_bytes'] * B / 1e9:.2f} GB, 8 rotating input sets)",
@@ -509,6 +510,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--scheme", choices=["stepquant", "row_absmax"], default="stepquant",
                     help="requantisation rule (row_absmax: the pages' uniform baseline)")
+    ap.add_argument("--scale-bits", type=int, choices=[32, 16], default=32,
+                    help="storage of the scales r, c (16: the compact binary16 layout)")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-budget", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -79,12 +79,16 @@ typedef struct {
                                 pivot unit) */
   const float* omega;        /* host; [H*d] row influence omega_i, finite and > 0 */
   int scheme;                /* stq_scheme; 0 (zero-initialised) = STQ_SCHEME_STEPQUANT */
+  int scale_bits;            /* storage of r and c: 32 (float32; 0 means 32) or 16
+                                (IEEE binary16, the compact layout: r is rounded to
+                                binary16 when formed, the final c before the codes are
+                                fitted to it, so the stored triple stays consistent) */
 } stq_pool_desc;
 
 /* Buffer sizes (bytes) the caller allocates for a pool, from stq_pool_layout. */
 typedef struct {
   size_t codes_bytes;        /* packed codes, all slots */
-  size_t scales_bytes;       /* float32 r[d], c[d] per (slot, head) */
+  size_t scales_bytes;       /* r[d], c[d] per (slot, head), float32 or binary16 */
   size_t pivots_bytes;       /* float16 pivot rows, all slots */
   size_t meta_bytes;         /* device metadata the library writes at create time */
   size_t slot_code_bytes;    /* bytes of packed codes per slot */
@@ -98,7 +102,8 @@ typedef struct stq_pool stq_pool;
  * of its non-pivot units back to back (row i of width b takes 16*b bytes; code j of a
  * row is bits [b*j, b*j+b) of a little-endian bit stream, stored as
  * u = Q + 2^(b-1)); the float16 rows of its pivot units in (head, row) order; and
- * r[128], c[128] per head. Returns STQ_ERR_INVALID_ARG on a bad description. */
+ * r[128], c[128] per head (float32, or binary16 when scale_bits is 16). Returns
+ * STQ_ERR_INVALID_ARG on a bad description. */
 stq_status stq_pool_layout(const stq_pool_desc* desc, stq_pool_sizes* out);
 
 /* Bind caller-allocated device buffers (sizes from stq_pool_layout) to a new pool

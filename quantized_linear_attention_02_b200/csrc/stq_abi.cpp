@@ -43,7 +43,7 @@ size_t up16(size_t x) { return (x + 15) & ~size_t(15); }
 
 // Host-side layout of one pool, derived from the description.
 struct HostLayout {
-  int kind = 0, n_slots = 0, H = 0, scheme = 0;
+  int kind = 0, n_slots = 0, H = 0, scheme = 0, scale_bytes = 4;
   std::vector<uint32_t> head_code_off, head_code_bytes, head_piv_first, head_piv_count, head_bits;
   std::vector<uint32_t> warp_code_off;
   std::vector<uint32_t> row_info;
@@ -68,6 +68,9 @@ stq_status build_layout(const stq_pool_desc* desc, HostLayout& L) {
   const int H = desc->H, D = STQ_D;
   L.kind = desc->kind;
   L.scheme = desc->scheme;
+  if (desc->scale_bits != 0 && desc->scale_bits != 32 && desc->scale_bits != 16)
+    return fail(STQ_ERR_INVALID_ARG, "scale_bits must be 16 or 32 (0 = 32), got %d", desc->scale_bits);
+  L.scale_bytes = desc->scale_bits == 16 ? 2 : 4;
   L.n_slots = desc->n_slots;
   L.H = H;
   L.head_code_off.assign(H, 0);
@@ -180,7 +183,7 @@ stq_status stq_pool_layout(const stq_pool_desc* desc, stq_pool_sizes* out) {
   const size_t ns = size_t(desc->n_slots);
   out->slot_code_bytes = size_t(L.slot_code_bytes);
   out->codes_bytes = ns * size_t(L.slot_code_bytes);
-  out->scales_bytes = ns * size_t(L.H) * 2 * STQ_D * sizeof(float);
+  out->scales_bytes = ns * size_t(L.H) * 2 * STQ_D * size_t(L.scale_bytes);
   out->pivots_bytes = ns * size_t(L.n_pivot_rows) * STQ_D * 2;
   out->meta_bytes = stq::meta_layout(L.H).total;
   out->n_pivot_rows = L.n_pivot_rows;
@@ -230,7 +233,8 @@ stq_status stq_pool_create(const stq_pool_desc* desc, void* d_codes, void* d_sca
   dv.max_head_bytes = L.max_head_bytes;
   dv.slot_code_bytes = L.slot_code_bytes;
   dv.codes = static_cast<uint8_t*>(d_codes);
-  dv.scales = static_cast<float*>(d_scales);
+  dv.scales = d_scales;
+  dv.scale16 = L.scale_bytes == 2;
   dv.pivots = static_cast<uint16_t*>(d_pivots);
   dv.head_code_off = reinterpret_cast<const uint32_t*>(mb + m.head_code_off);
   dv.head_code_bytes = reinterpret_cast<const uint32_t*>(mb + m.head_code_bytes);

@@ -13,9 +13,8 @@ namespace {
 
 struct AbsmaxStore {
   template <int BITS>
-  static __device__ __forceinline__ void store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], float* r_global,
-                                               float* c_global, uint8_t* codes_global, int warp_code_start,
-                                               float* o_global) {
+  static __device__ __forceinline__ void store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], const Scales& sc,
+                                               uint8_t* codes_global, int warp_code_start, float* o_global) {
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r0 = w * RPW;
 
@@ -63,14 +62,14 @@ struct AbsmaxStore {
       } else {
         iq = __frcp_rn(float((1 << (BITS - 1)) - 1));
       }
-      const float r = pivot ? 0.0f : fmul(a[0], iq);
+      const float r = sc.stored(pivot ? 0.0f : fmul(a[0], iq));   // codes fit the stored r
       if (lane < 16) {
         const float ir = recip_scale(r);
         wr.irr[R] = make_float2(ir, ir);
-        r_global[r0 + R] = r;
+        sc.put(r0 + R, r);
       }
     }
-    if (lane < 16) c_global[16 * w + lane] = 1.0f;
+    if (lane < 16) sc.put(D + 16 * w + lane, 1.0f);
     __syncwarp();
 
     // --- codes: x = S * (1/r_i) taken exactly, rounded in the 2^23 binade ---------
@@ -98,7 +97,8 @@ struct AbsmaxStore {
           default: store_codes<8>(row, lane, t); break;
         }
       } else {
-        // |S_ij| * fl(1/r_i) <= qmax (1 + 2^-22), so |n| <= qmax: the 16-bit lanes hold it
+        // |S_ij| * fl(1/r_i) <= qmax (1 + 2^-22) (binary16 r: <= qmax (1 + 2^-10)), so
+        // |n| <= qmax + 1: the 16-bit lanes hold it
         constexpr float MB = MAGIC + float(1 << (BITS - 1));
         constexpr uint32_t HI = ((1u << BITS) - 1u) * 0x00010001u;
         const f2 t01 = fma2(s[rr][0], ir, dup(MB));

@@ -3,9 +3,10 @@
 // the kernel bodies. The quantiser that ends a decode step (and stq_quantize_init) is a
 // policy `Store` with
 //   template <int BITS> static __device__ void store(CtaSmem&, WarpRows&,
-//       f2 (&s)[RPW][2], float* r, float* c, uint8_t* codes, int warp_code_start,
+//       f2 (&s)[RPW][2], const Scales& sc, uint8_t* codes, int warp_code_start,
 //       float* o);
-// which quantises the warp's 16 rows s (float32 state), writes codes and scales and, when
+// which quantises the warp's 16 rows s (float32 state), writes codes and scales (r at
+// Scales index i, c at D + j) and, when
 // o is not null, the readout whose per-warp partials are in red[1][0].
 // The float32 evaluation order is described at the top of stq_kernels.cu.
 #pragma once
@@ -201,10 +202,35 @@ __device__ __forceinline__ void copy16(void* dst, const void* src, int bytes) {
   for (int t = threadIdx.x; t < (bytes >> 4); t += NT) d[t] = s[t];
 }
 
+// r[D] then c[D] of one head in its slot: float32, or binary16 in a compact pool.
+struct Scales {
+  void* p;
+  bool h16;
+  __device__ __forceinline__ float get(int i) const {
+    return h16 ? __half2float(static_cast<const __half*>(p)[i]) : static_cast<const float*>(p)[i];
+  }
+  __device__ __forceinline__ float4 get4(int i) const {   // i a multiple of 4
+    if (!h16) return *reinterpret_cast<const float4*>(static_cast<const float*>(p) + i);
+    const uint2 b = *reinterpret_cast<const uint2*>(static_cast<const __half*>(p) + i);
+    return make_float4(__half2float(__ushort_as_half(uint16_t(b.x & 0xFFFFu))),
+                       __half2float(__ushort_as_half(uint16_t(b.x >> 16))),
+                       __half2float(__ushort_as_half(uint16_t(b.y & 0xFFFFu))),
+                       __half2float(__ushort_as_half(uint16_t(b.y >> 16))));
+  }
+  __device__ __forceinline__ void put(int i, float v) const {
+    if (h16) static_cast<__half*>(p)[i] = __float2half_rn(v);
+    else static_cast<float*>(p)[i] = v;
+  }
+  // the value the pool will hold: binary16 rounding (to nearest even) in a compact pool
+  __device__ __forceinline__ float stored(float v) const {
+    return h16 ? __half2float(__float2half_rn(v)) : v;
+  }
+};
+
 struct HeadRef {
   uint8_t* codes;      // global: this head's codes in its slot
   uint16_t* pivots;    // global: this head's first pivot row in its slot
-  float* scales;       // global: r[D], c[D] of this head in its slot
+  Scales sc;           // global: r[D], c[D] of this head in its slot
   int code_bytes;
   int piv_count;
   int bits;            // uniform width of the head, 16 if all pivot, 0 if mixed
@@ -218,7 +244,8 @@ __device__ __forceinline__ HeadRef head_ref(const PoolDev& P, int slot, int h) {
   r.bits = int(P.head_bits[h]);
   r.codes = P.codes + uint64_t(slot) * P.slot_code_bytes + P.head_code_off[h];
   r.pivots = P.pivots + (uint64_t(slot) * P.n_pivot_rows + P.head_piv_first[h]) * D;
-  r.scales = P.scales + (uint64_t(slot) * P.H + h) * 2 * D;
+  r.sc.h16 = P.scale16 != 0;
+  r.sc.p = static_cast<uint8_t*>(P.scales) + (uint64_t(slot) * P.H + h) * 2 * D * (P.scale16 ? 2 : 4);
   r.piv_stage_off = r.code_bytes;  // code bytes are a multiple of 16
   return r;
 }
@@ -310,7 +337,7 @@ __device__ __forceinline__ void width_consts(int bits, float& qm, float& iq, flo
 
 // Lanes 0..15 of warp w: the per-row data of rows 16w..16w+15 of head h.
 __device__ __forceinline__ void load_warp_rows(const PoolDev& P, int h, WarpRows& wr, int lane, int r0,
-                                               const float* k_vec, const float* q_vec, const float* r_in,
+                                               const float* k_vec, const float* q_vec, const Scales* r_in,
                                                const float* gate_rows, float gate_s) {
   if (lane < RPW) {
     const int i = r0 + lane;
@@ -324,7 +351,7 @@ __device__ __forceinline__ void load_warp_rows(const PoolDev& P, int h, WarpRows
     if (k_vec != nullptr) {
       const float dec = gate_rows != nullptr ? gate_rows[i] : gate_s;
       const float kv = k_vec[i], qv = q_vec[i];
-      const float rd = fmul(dec, r_in[i]);
+      const float rd = fmul(dec, r_in->get(i));
       wr.dec[lane] = dec;
       wr.kk[lane] = make_float2(kv, kv);
       wr.qq[lane] = make_float2(qv, qv);
@@ -453,7 +480,7 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
         *reinterpret_cast<uint2*>(hr.pivots + row_off(info) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
     }
   }
-  Store::template store<BITS>(cs, wr, s, hr.scales, hr.scales + D, hr.codes, warp_code_start, o_out);
+  Store::template store<BITS>(cs, wr, s, hr.sc, hr.codes, warp_code_start, o_out);
 }
 
 // A head whose rows are all FP16 pivots: decay, update, readout, store float16; r = c = 0.
@@ -516,7 +543,7 @@ __device__ __forceinline__ void decode_pivot_warp(CtaSmem& cs, WarpRows& wr, con
     warp_tree(cs.red[1][0], lane, lo, hi);
     *reinterpret_cast<float4*>(o_out + 4 * lane) = make_float4(lo.x, lo.y, hi.x, hi.y);
   }
-  if (tid < 2 * D) hr.scales[tid] = 0.0f;
+  if (tid < 2 * D) hr.sc.put(tid, 0.0f);
 }
 
 // ---------------------------------------------------------------------------------
@@ -550,9 +577,9 @@ decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* 
   for (int o = 16 * lane; o < wend - wstart; o += 16 * 32) cp_async16(wr.codes + o, hr.codes + wstart + o);
   asm volatile("cp.async.commit_group;" ::: "memory");
   const float gate_s = (P.kind == 0) ? gate[vi] : 0.0f;
-  load_warp_rows(P, h, wr, lane, r0, k + vec, q + vec, hr.scales, P.kind == 0 ? nullptr : gate + vec, gate_s);
+  load_warp_rows(P, h, wr, lane, r0, k + vec, q + vec, &hr.sc, P.kind == 0 ? nullptr : gate + vec, gate_s);
   const float beta_s = beta[vi];
-  const float4 c4 = *reinterpret_cast<const float4*>(hr.scales + D + 4 * lane);
+  const float4 c4 = hr.sc.get4(D + 4 * lane);
   const f2 cin[2] = {make_float2(c4.x, c4.y), make_float2(c4.z, c4.w)};
   const float v_own = v[vec + 16 * w + (lane & 15)];
   asm volatile("cp.async.wait_all;" ::: "memory");
@@ -591,7 +618,7 @@ __device__ __forceinline__ void quantize_warp(CtaSmem& cs, WarpRows& wr, const H
         *reinterpret_cast<uint2*>(hr.pivots + row_off(info) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
     }
   }
-  Store::template store<BITS>(cs, wr, s, hr.scales, hr.scales + D, hr.codes, warp_code_start, nullptr);
+  Store::template store<BITS>(cs, wr, s, hr.sc, hr.codes, warp_code_start, nullptr);
 }
 
 template <class Store>
@@ -626,7 +653,7 @@ quantize_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float
         *reinterpret_cast<uint2*>(hr.pivots + i * D + 4 * lane) =
             half4_bits(make_float2(x.x, x.y), make_float2(x.z, x.w));
       }
-      if (tid < 2 * D) hr.scales[tid] = 0.0f;
+      if (tid < 2 * D) hr.sc.put(tid, 0.0f);
       break;
     default: quantize_warp<MIXED, Store>(cs, wr, hr, wstart, src); break;
   }

@@ -30,7 +30,7 @@ struct PoolDev {
   int max_head_bytes;       // largest per-head code + pivot bytes (staging size)
   uint64_t slot_code_bytes;
   uint8_t* codes;           // [n_slots, slot_code_bytes]
-  float* scales;            // [n_slots, H, 2, D]
+  void* scales;             // [n_slots, H, 2, D] float32, or binary16 if scale16
   uint16_t* pivots;         // [n_slots, n_pivot_rows, D] float16 bits
   // metadata (device)
   const uint32_t* head_code_off;    // [H] byte offset of head h's codes in a slot
@@ -47,6 +47,7 @@ struct PoolDev {
   uint32_t* err;                    // [4] sticky error bits
   int scheme;                       // SCHEME_STEPQUANT or SCHEME_ROW_ABSMAX
   int any_mixed;                    // 1 if some head's rows have different widths
+  int scale16;                      // 1: r and c stored as binary16
 };
 
 // Byte layout of the meta buffer, computed on the host.

@@ -38,9 +38,8 @@ namespace {
 // and one for the new 1/c.
 // ---------------------------------------------------------------------------------
 template <int BITS>
-__device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], float* r_global,
-                                            float* c_global, uint8_t* codes_global, int warp_code_start,
-                                            float* o_global) {
+__device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], const Scales& sc,
+                                            uint8_t* codes_global, int warp_code_start, float* o_global) {
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r0 = w * RPW;
 
@@ -82,12 +81,13 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
     // lane l now holds the sum of row R(l): bits 0..3 of l chose halves 8, 4, 2, 1
     const int R = ((lane & 1) << 3) | ((lane & 2) << 1) | ((lane & 4) >> 1) | ((lane & 8) >> 3);
     const bool pivot = (BITS == MIXED) ? (row_bits(wr.info[R]) == PIVOT) : false;
-    const float r = pivot ? 0.0f : fmul(fmul(a[0], 0.0078125f), wr.g[R]);
+    // a compact pool rounds r to binary16 here: y, the weights and the codes use it
+    const float r = sc.stored(pivot ? 0.0f : fmul(fmul(a[0], 0.0078125f), wr.g[R]));
     if (lane < 16) {
       const float ir = recip_scale(r), bv = fmul(wr.om[R], fmul(r, r));
       wr.irr[R] = make_float2(ir, ir);
       wr.bb[R] = make_float2(bv, bv);
-      r_global[r0 + R] = r;
+      sc.put(r0 + R, r);
     }
   }
   __syncwarp();
@@ -199,6 +199,7 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
       const float den = __shfl_down_sync(0xffffffffu, sum, 16);
       if (lane < 16) {
         if (den > 0.0f) c_own = __fdiv_rn(sum, den);
+        if (it == 1) c_own = sc.stored(c_own);   // the final c as the pool will hold it
         const float icn = recip_scale(c_own);
         cs.col_ic[jown] = icn;
         // every least-squares step keeps c >= c_before / 2 (each term Q y >= c Q^2 / 2),
@@ -218,7 +219,7 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
     ic[0] = make_float2(i4.x, i4.y);
     ic[1] = make_float2(i4.z, i4.w);
   }
-  if (lane < 16) c_global[jown] = c_own;
+  if (lane < 16) sc.put(D + jown, c_own);
   if constexpr (BITS != MIXED) {
     if (!any_wide) {
       constexpr float MB = MAGIC + float(1 << (BITS - 1));
@@ -270,9 +271,9 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
 // The quantiser of the method: dual-axis refit (refit_store).
 struct StepQuantStore {
   template <int BITS>
-  static __device__ __forceinline__ void store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], float* r,
-                                               float* c, uint8_t* codes, int warp_code_start, float* o) {
-    refit_store<BITS>(cs, wr, s, r, c, codes, warp_code_start, o);
+  static __device__ __forceinline__ void store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], const Scales& sc,
+                                               uint8_t* codes, int warp_code_start, float* o) {
+    refit_store<BITS>(cs, wr, s, sc, codes, warp_code_start, o);
   }
 };
 
@@ -303,11 +304,11 @@ dequant_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, float* __res
   const HeadRef hr = head_ref(P, slot, h);
   if (tid < D) {
     info_s[tid] = P.row_info[h * D + tid];
-    r_s[tid] = hr.scales[tid];
+    r_s[tid] = hr.sc.get(tid);
   }
   copy16(stage, hr.codes, hr.code_bytes);
   copy16(stage + hr.piv_stage_off, hr.pivots, hr.piv_count * D * 2);
-  const float4 c4 = *reinterpret_cast<const float4*>(hr.scales + D + 4 * lane);
+  const float4 c4 = hr.sc.get4(D + 4 * lane);
   const f2 cin[2] = {make_float2(c4.x, c4.y), make_float2(c4.z, c4.w)};
   __syncthreads();
   float* dst = S_out + uint64_t(item) * D * D;

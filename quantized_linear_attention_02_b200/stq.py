@@ -30,7 +30,8 @@ class StqError(RuntimeError):
 class _Desc(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int), ("n_slots", ctypes.c_int), ("H", ctypes.c_int),
                 ("d", ctypes.c_int), ("unit_bits", ctypes.POINTER(ctypes.c_uint8)),
-                ("omega", ctypes.POINTER(ctypes.c_float)), ("scheme", ctypes.c_int)]
+                ("omega", ctypes.POINTER(ctypes.c_float)), ("scheme", ctypes.c_int),
+                ("scale_bits", ctypes.c_int)]
 
 
 class _Sizes(ctypes.Structure):
@@ -87,20 +88,20 @@ def _check(status):
         raise StqError(status, lib().stq_last_error().decode())
 
 
-def _desc(kind, n_slots, unit_bits, omega, scheme="stepquant"):
+def _desc(kind, n_slots, unit_bits, omega, scheme="stepquant", scale_bits=32):
     ub = np.ascontiguousarray(unit_bits, dtype=np.uint8)
     om = np.ascontiguousarray(omega, dtype=np.float32)
     H = om.shape[0]
     d = _Desc(KINDS[kind] if isinstance(kind, str) else int(kind), int(n_slots), int(H), D,
               ub.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
               om.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),
-              SCHEMES[scheme] if isinstance(scheme, str) else int(scheme))
+              SCHEMES[scheme] if isinstance(scheme, str) else int(scheme), int(scale_bits))
     return d, (ub, om)   # keep the arrays alive with the struct
 
 
-def layout(kind, n_slots, unit_bits, omega, scheme="stepquant") -> dict:
+def layout(kind, n_slots, unit_bits, omega, scheme="stepquant", scale_bits=32) -> dict:
     """Buffer sizes of a pool (host only; no CUDA call)."""
-    d, keep = _desc(kind, n_slots, unit_bits, omega, scheme)
+    d, keep = _desc(kind, n_slots, unit_bits, omega, scheme, scale_bits)
     s = _Sizes()
     _check(lib().stq_pool_layout(ctypes.byref(d), ctypes.byref(s)))
     return {f: getattr(s, f) for f, _ in _Sizes._fields_}
@@ -130,23 +131,25 @@ class Pool:
     """A packed state pool on the current CUDA device. The buffers are torch tensors
     owned here; the library handle only references them."""
 
-    def __init__(self, kind, n_slots, unit_bits, omega, device=None, scheme="stepquant"):
+    def __init__(self, kind, n_slots, unit_bits, omega, device=None, scheme="stepquant", scale_bits=32):
         import torch
         self.kind = kind
         self.kind_id = KINDS[kind]
         self.scheme = scheme
+        self.scale_bits = int(scale_bits)
         self.n_slots = int(n_slots)
         self.unit_bits = np.ascontiguousarray(unit_bits, dtype=np.uint8)
         self.omega = np.ascontiguousarray(omega, dtype=np.float32)
         self.H = self.omega.shape[0]
-        self.sizes = layout(kind, n_slots, self.unit_bits, self.omega, scheme)
+        self.sizes = layout(kind, n_slots, self.unit_bits, self.omega, scheme, scale_bits)
         dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         s = self.sizes
         self.codes = torch.zeros(max(s["codes_bytes"], 16), dtype=torch.uint8, device=dev)
-        self.scales = torch.zeros(s["scales_bytes"] // 4, dtype=torch.float32, device=dev)
+        sdt = torch.float16 if self.scale_bits == 16 else torch.float32
+        self.scales = torch.zeros(s["scales_bytes"] // (2 if self.scale_bits == 16 else 4), dtype=sdt, device=dev)
         self.pivots = torch.zeros(max(s["pivots_bytes"] // 2, 8), dtype=torch.float16, device=dev)
         self.meta = torch.zeros(s["meta_bytes"], dtype=torch.uint8, device=dev)
-        d, keep = _desc(kind, n_slots, self.unit_bits, self.omega, scheme)
+        d, keep = _desc(kind, n_slots, self.unit_bits, self.omega, scheme, scale_bits)
         h = ctypes.c_void_p()
         _check(lib().stq_pool_create(ctypes.byref(d), ctypes.c_void_p(self.codes.data_ptr()),
                                      ctypes.c_void_p(self.scales.data_ptr()),

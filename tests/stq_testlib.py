@@ -53,7 +53,7 @@ def write_oracle_state(pool, layout, slots, u, r, c, piv):
     """Put an oracle-packed state into the library pool's buffers (host image ->
     device copy of the same bytes)."""
     import torch
-    img = O.Pool(layout, pool.n_slots)
+    img = O.Pool(layout, pool.n_slots, scale16=getattr(pool, "scale_bits", 32) == 16)
     img.write_heads(list(range(len(slots))), u, r, c, piv)   # rows 0..n-1 of the image
     for n, s in enumerate(slots):
         pool.codes_view()[s].copy_(torch.from_numpy(img.codes[n]))
@@ -65,7 +65,7 @@ def write_oracle_state(pool, layout, slots, u, r, c, piv):
 def read_pool_state(pool, layout, slots):
     """Read the library pool's bytes for the given slots and decode them with the
     oracle's unpacker: (u, r, c, piv)."""
-    img = O.Pool(layout, len(slots))
+    img = O.Pool(layout, len(slots), scale16=getattr(pool, "scale_bits", 32) == 16)
     for n, s in enumerate(slots):
         img.codes[n] = pool.codes_view()[s].cpu().numpy()
         img.scales[n] = pool.scales_view()[s].cpu().numpy()

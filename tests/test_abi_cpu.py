@@ -62,12 +62,21 @@ def test_absmax_scheme_keeps_the_layout(lib, w):
     assert stq.layout(*args, "row_absmax") == stq.layout(*args)
 
 
+@pytest.mark.parametrize("w", W.WORKLOADS[1:3], ids=lambda w: w.name)
+def test_binary16_scales_halve_the_scale_bytes(lib, w):
+    args = (w.kind, W.n_slots(w.B), W.unit_bits(w), W.omega(w))
+    a, b = stq.layout(*args), stq.layout(*args, "stepquant", 16)
+    assert b["scales_bytes"] * 2 == a["scales_bytes"]
+    assert {k: v for k, v in a.items() if k != "scales_bytes"} == {k: v for k, v in b.items() if k != "scales_bytes"}
+    assert stq.layout(*args, "stepquant", 0) == a
+
+
 def test_six_bit_head_size(lib):
     got = stq.layout("gdn", 1, np.array([6], np.uint8), np.ones((1, 128), np.float32))
     assert got["slot_code_bytes"] == 128 * 96        # 4 codes in 3 bytes
 
 
-@pytest.mark.parametrize("bad", ["width", "omega_zero", "omega_nan", "kind", "slots", "scheme"])
+@pytest.mark.parametrize("bad", ["width", "omega_zero", "omega_nan", "kind", "slots", "scheme", "scale_bits"])
 def test_invalid_descriptions_rejected(lib, bad):
     ub = np.full(4, 6, np.uint8)
     om = np.ones((4, 128), np.float32)
@@ -84,8 +93,9 @@ def test_invalid_descriptions_rejected(lib, bad):
         n_slots = 0
     elif bad == "scheme":
         scheme = 2
+    scale_bits = 8 if bad == "scale_bits" else 32
     with pytest.raises(stq.StqError) as e:
-        stq.layout(kind, n_slots, ub, om, scheme)
+        stq.layout(kind, n_slots, ub, om, scheme, scale_bits)
     assert e.value.status == 1
     assert lib.stq_last_error()
 

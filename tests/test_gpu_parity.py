@@ -359,3 +359,53 @@ def test_absmax_decode_chain(widx, steps):
     S_gpu = O.dequantize(ug, rg, cg, pg, rb)
     S_or = O.dequantize(u, r, c, piv, rb)
     assert T.rel_l2(S_gpu, S_or) <= T.CHAIN_REL_L2
+
+
+# ---------------------------------------------------------------------------------
+# compact pools: r and c stored as binary16 (both quantisers)
+# ---------------------------------------------------------------------------------
+def _quantiser(scheme):
+    if scheme == "row_absmax":
+        return lambda S, om, rb: O.absmax_quantise(S, rb, scale16=True)
+    return lambda S, om, rb: O.refit(S, om, rb, scale16=True)
+
+
+@pytest.mark.parametrize("widx", [1, 2])
+@pytest.mark.parametrize("scheme", ["stepquant", "row_absmax"])
+def test_scale16_quantize_step_and_chain(widx, scheme):
+    w = W.WORKLOADS[widx]
+    reqs = [0, w.B - 1]
+    rb, om = W.row_bits(w), W.omega(w)
+    pool = stq.Pool(w.kind, W.n_slots(w.B), W.unit_bits(w), om, scheme=scheme, scale_bits=16)
+    L = O.Layout(rb)
+    slots = [W.slot_of_request(b) for b in reqs]
+    S0 = T.warm_state(w.index, tuple(reqs))
+    # quantise: same codes and binary16 scales as the oracle
+    u, r, c, piv = _quantiser(scheme)(S0, om, rb)
+    pool.quantize_init(slots_t(reqs), dev(S0))
+    pool.check()
+    ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
+    if T.compare_codes(ug, u, S0, r, c, rb, "scale16 quantize_init") == 0:
+        assert np.array_equal(rg, r) and np.array_equal(cg, c)
+    # chained steps from the oracle's packed state
+    T.write_oracle_state(pool, L, slots, u, r, c, piv)
+    out = torch.empty((len(reqs), w.H, D), device="cuda")
+    for t in range(16):
+        x = T.inputs_for(w, "decode", t, reqs)
+        u2, r2, c2, p2, o, X = O.decode_step(u, r, c, piv, rb, om, x.q, x.k, x.v,
+                                             O.gate_rows(x.gate, w.kind, D), x.beta,
+                                             scheme=scheme, scale16=True)
+        pool.decode_step(slots_t(reqs), dev(x.q), dev(x.k), dev(x.v), dev(x.gate), dev(x.beta), out)
+        assert T.per_vector_rel_l2(out.cpu().numpy(), o).max() <= T.OUT_REL_L2, f"step {t}"
+        if t == 0:     # teacher-forced first step: the step rule itself
+            ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
+            if T.compare_codes(ug, u2, X, r2, c2, rb, "scale16 step") == 0:
+                assert np.array_equal(rg, r2) and np.array_equal(cg, c2)
+        u, r, c, piv = u2, r2, c2, p2
+    pool.check()
+    ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
+    assert T.rel_l2(O.dequantize(ug, rg, cg, pg, rb), O.dequantize(u, r, c, piv, rb)) <= T.CHAIN_REL_L2
+    # the dequantiser reads binary16 scales
+    Sd = torch.empty((len(reqs), w.H, D, D), device="cuda")
+    pool.dequantize(slots_t(reqs), Sd)
+    assert np.array_equal(Sd.cpu().numpy(), O.dequantize(ug, rg, cg, pg, rb))
