@@ -12,8 +12,8 @@ namespace stq {
 namespace {
 
 struct AbsmaxStore {
-  template <int BITS>
-  static __device__ __forceinline__ void store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], const Scales& sc,
+  template <int BITS, class Sc>
+  static __device__ __forceinline__ void store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], const Sc& sc,
                                                uint8_t* codes_global, int warp_code_start, float* o_global) {
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r0 = w * RPW;
@@ -125,17 +125,22 @@ cudaError_t launch_decode_absmax(const PoolDev& P, const int32_t* slots, int B, 
                                  const float* k, const float* v, const float* gate,
                                  const float* beta, float* out, cudaStream_t s) {
   if (B == 0) return cudaSuccess;
-  if (P.any_mixed)
-    decode_kernel<AbsmaxStore, true><<<B * P.H, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
-  else
-    decode_kernel<AbsmaxStore, false><<<B * P.H, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+  const unsigned grid = unsigned(B) * unsigned(P.H);
+  if (P.scale16) {
+    if (P.any_mixed) decode_kernel<AbsmaxStore, true, true><<<grid, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+    else decode_kernel<AbsmaxStore, false, true><<<grid, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+  } else {
+    if (P.any_mixed) decode_kernel<AbsmaxStore, true, false><<<grid, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+    else decode_kernel<AbsmaxStore, false, false><<<grid, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_absmax(const PoolDev& P, const int32_t* slots, int B, const float* S,
                                    cudaStream_t s) {
   if (B == 0) return cudaSuccess;
-  quantize_kernel<AbsmaxStore><<<B * P.H, NT, 0, s>>>(P, slots, B, S);
+  if (P.scale16) quantize_kernel<AbsmaxStore, true><<<B * P.H, NT, 0, s>>>(P, slots, B, S);
+  else quantize_kernel<AbsmaxStore, false><<<B * P.H, NT, 0, s>>>(P, slots, B, S);
   return cudaGetLastError();
 }
 

@@ -3,7 +3,7 @@
 // the kernel bodies. The quantiser that ends a decode step (and stq_quantize_init) is a
 // policy `Store` with
 //   template <int BITS> static __device__ void store(CtaSmem&, WarpRows&,
-//       f2 (&s)[RPW][2], const Scales& sc, uint8_t* codes, int warp_code_start,
+//       f2 (&s)[RPW][2], const Scales<H16>& sc, uint8_t* codes, int warp_code_start,
 //       float* o);
 // which quantises the warp's 16 rows s (float32 state), writes codes and scales (r at
 // Scales index i, c at D + j) and, when
@@ -202,50 +202,56 @@ __device__ __forceinline__ void copy16(void* dst, const void* src, int bytes) {
   for (int t = threadIdx.x; t < (bytes >> 4); t += NT) d[t] = s[t];
 }
 
-// r[D] then c[D] of one head in its slot: float32, or binary16 in a compact pool.
+// r[D] then c[D] of one head in its slot: float32, or binary16 (H16) in a compact pool.
+template <bool H16>
 struct Scales {
   void* p;
-  bool h16;
   __device__ __forceinline__ float get(int i) const {
-    return h16 ? __half2float(static_cast<const __half*>(p)[i]) : static_cast<const float*>(p)[i];
+    if constexpr (H16) return __half2float(static_cast<const __half*>(p)[i]);
+    else return static_cast<const float*>(p)[i];
   }
   __device__ __forceinline__ float4 get4(int i) const {   // i a multiple of 4
-    if (!h16) return *reinterpret_cast<const float4*>(static_cast<const float*>(p) + i);
-    const uint2 b = *reinterpret_cast<const uint2*>(static_cast<const __half*>(p) + i);
-    return make_float4(__half2float(__ushort_as_half(uint16_t(b.x & 0xFFFFu))),
-                       __half2float(__ushort_as_half(uint16_t(b.x >> 16))),
-                       __half2float(__ushort_as_half(uint16_t(b.y & 0xFFFFu))),
-                       __half2float(__ushort_as_half(uint16_t(b.y >> 16))));
+    if constexpr (!H16) {
+      return *reinterpret_cast<const float4*>(static_cast<const float*>(p) + i);
+    } else {
+      const uint2 b = *reinterpret_cast<const uint2*>(static_cast<const __half*>(p) + i);
+      return make_float4(__half2float(__ushort_as_half(uint16_t(b.x & 0xFFFFu))),
+                         __half2float(__ushort_as_half(uint16_t(b.x >> 16))),
+                         __half2float(__ushort_as_half(uint16_t(b.y & 0xFFFFu))),
+                         __half2float(__ushort_as_half(uint16_t(b.y >> 16))));
+    }
   }
   __device__ __forceinline__ void put(int i, float v) const {
-    if (h16) static_cast<__half*>(p)[i] = __float2half_rn(v);
+    if constexpr (H16) static_cast<__half*>(p)[i] = __float2half_rn(v);
     else static_cast<float*>(p)[i] = v;
   }
   // the value the pool will hold: binary16 rounding (to nearest even) in a compact pool
   __device__ __forceinline__ float stored(float v) const {
-    return h16 ? __half2float(__float2half_rn(v)) : v;
+    if constexpr (H16) return __half2float(__float2half_rn(v));
+    else return v;
   }
 };
 
+template <bool H16>
 struct HeadRef {
   uint8_t* codes;      // global: this head's codes in its slot
   uint16_t* pivots;    // global: this head's first pivot row in its slot
-  Scales sc;           // global: r[D], c[D] of this head in its slot
+  Scales<H16> sc;      // global: r[D], c[D] of this head in its slot
   int code_bytes;
   int piv_count;
   int bits;            // uniform width of the head, 16 if all pivot, 0 if mixed
   int piv_stage_off;   // byte offset of the pivot rows in the staging buffer
 };
 
-__device__ __forceinline__ HeadRef head_ref(const PoolDev& P, int slot, int h) {
-  HeadRef r;
+template <bool H16>
+__device__ __forceinline__ HeadRef<H16> head_ref(const PoolDev& P, int slot, int h) {
+  HeadRef<H16> r;
   r.code_bytes = int(P.head_code_bytes[h]);
   r.piv_count = int(P.head_piv_count[h]);
   r.bits = int(P.head_bits[h]);
   r.codes = P.codes + uint64_t(slot) * P.slot_code_bytes + P.head_code_off[h];
   r.pivots = P.pivots + (uint64_t(slot) * P.n_pivot_rows + P.head_piv_first[h]) * D;
-  r.sc.h16 = P.scale16 != 0;
-  r.sc.p = static_cast<uint8_t*>(P.scales) + (uint64_t(slot) * P.H + h) * 2 * D * (P.scale16 ? 2 : 4);
+  r.sc.p = static_cast<uint8_t*>(P.scales) + (uint64_t(slot) * P.H + h) * 2 * D * (H16 ? 2 : 4);
   r.piv_stage_off = r.code_bytes;  // code bytes are a multiple of 16
   return r;
 }
@@ -336,8 +342,9 @@ __device__ __forceinline__ void width_consts(int bits, float& qm, float& iq, flo
 }
 
 // Lanes 0..15 of warp w: the per-row data of rows 16w..16w+15 of head h.
+template <bool H16>
 __device__ __forceinline__ void load_warp_rows(const PoolDev& P, int h, WarpRows& wr, int lane, int r0,
-                                               const float* k_vec, const float* q_vec, const Scales* r_in,
+                                               const float* k_vec, const float* q_vec, const Scales<H16>* r_in,
                                                const float* gate_rows, float gate_s) {
   if (lane < RPW) {
     const int i = r0 + lane;
@@ -378,8 +385,8 @@ __device__ __forceinline__ void publish_delta(CtaSmem& cs, int lane, int w, floa
   }
 }
 
-template <int BITS, class Store>
-__device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const HeadRef& hr, int warp_code_start,
+template <int BITS, class Store, bool H16>
+__device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const HeadRef<H16>& hr, int warp_code_start,
                                             const f2 (&cin)[2], float v_own, float beta_s,
                                             float* o_out) {
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
@@ -484,7 +491,8 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
 }
 
 // A head whose rows are all FP16 pivots: decay, update, readout, store float16; r = c = 0.
-__device__ __forceinline__ void decode_pivot_warp(CtaSmem& cs, WarpRows& wr, const HeadRef& hr,
+template <bool H16>
+__device__ __forceinline__ void decode_pivot_warp(CtaSmem& cs, WarpRows& wr, const HeadRef<H16>& hr,
                                                   float v_own, float beta_s, float* o_out) {
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int r0 = w * RPW;
@@ -552,7 +560,7 @@ __device__ __forceinline__ void decode_pivot_warp(CtaSmem& cs, WarpRows& wr, con
 // warp stages its own 16 rows (asynchronous 16-byte copies) and writes its own codes
 // back, so the CTA synchronises only for the five column exchanges.
 // ---------------------------------------------------------------------------------
-template <class Store, bool kMixed>
+template <class Store, bool kMixed, bool H16>
 __global__ void __launch_bounds__(NT, 2)
 decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* __restrict__ q,
               const float* __restrict__ k, const float* __restrict__ v,
@@ -567,7 +575,7 @@ decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* 
     if (tid == 0) atomicOr(P.err, ERR_SLOT_RANGE);
     return;
   }
-  const HeadRef hr = head_ref(P, slot, h);
+  const HeadRef<H16> hr = head_ref<H16>(P, slot, h);
   const int vi = bq * P.H + h;
   const uint64_t vec = uint64_t(vi) * D;
   WarpRows& wr = cs.wr[w];
@@ -586,14 +594,14 @@ decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* 
   __syncwarp();
   float* o_out = out + vec;
   switch (hr.bits) {
-    case 2: decode_warp<2, Store>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
-    case 4: decode_warp<4, Store>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
-    case 6: decode_warp<6, Store>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
-    case 8: decode_warp<8, Store>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
+    case 2: decode_warp<2, Store, H16>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
+    case 4: decode_warp<4, Store, H16>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
+    case 6: decode_warp<6, Store, H16>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
+    case 8: decode_warp<8, Store, H16>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
     case PIVOT: decode_pivot_warp(cs, wr, hr, v_own, beta_s, o_out); break;
     default:
       // heads whose rows have different widths (only pools with such heads launch this)
-      if constexpr (kMixed) decode_warp<MIXED, Store>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out);
+      if constexpr (kMixed) decode_warp<MIXED, Store, H16>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out);
       break;
   }
 }
@@ -601,8 +609,8 @@ decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* 
 // ---------------------------------------------------------------------------------
 // stq_quantize_init: float32 states -> packed pool.
 // ---------------------------------------------------------------------------------
-template <int BITS, class Store>
-__device__ __forceinline__ void quantize_warp(CtaSmem& cs, WarpRows& wr, const HeadRef& hr, int warp_code_start,
+template <int BITS, class Store, bool H16>
+__device__ __forceinline__ void quantize_warp(CtaSmem& cs, WarpRows& wr, const HeadRef<H16>& hr, int warp_code_start,
                                               const float* src) {
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int r0 = w * RPW;
@@ -621,7 +629,7 @@ __device__ __forceinline__ void quantize_warp(CtaSmem& cs, WarpRows& wr, const H
   Store::template store<BITS>(cs, wr, s, hr.sc, hr.codes, warp_code_start, nullptr);
 }
 
-template <class Store>
+template <class Store, bool H16>
 __global__ void __launch_bounds__(NT, 2)
 quantize_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* __restrict__ S) {
   __shared__ CtaSmem cs;
@@ -634,17 +642,17 @@ quantize_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float
     if (tid == 0) atomicOr(P.err, ERR_SLOT_RANGE);
     return;
   }
-  const HeadRef hr = head_ref(P, slot, h);
+  const HeadRef<H16> hr = head_ref<H16>(P, slot, h);
   WarpRows& wr = cs.wr[w];
-  load_warp_rows(P, h, wr, lane, r0, nullptr, nullptr, nullptr, nullptr, 0.0f);
+  load_warp_rows<H16>(P, h, wr, lane, r0, nullptr, nullptr, nullptr, nullptr, 0.0f);
   __syncwarp();
   const int wstart = int(P.warp_code_off[h * NW + w]);
   const float* src = S + uint64_t(item) * D * D;
   switch (hr.bits) {
-    case 2: quantize_warp<2, Store>(cs, wr, hr, wstart, src); break;
-    case 4: quantize_warp<4, Store>(cs, wr, hr, wstart, src); break;
-    case 6: quantize_warp<6, Store>(cs, wr, hr, wstart, src); break;
-    case 8: quantize_warp<8, Store>(cs, wr, hr, wstart, src); break;
+    case 2: quantize_warp<2, Store, H16>(cs, wr, hr, wstart, src); break;
+    case 4: quantize_warp<4, Store, H16>(cs, wr, hr, wstart, src); break;
+    case 6: quantize_warp<6, Store, H16>(cs, wr, hr, wstart, src); break;
+    case 8: quantize_warp<8, Store, H16>(cs, wr, hr, wstart, src); break;
     case PIVOT:
 #pragma unroll
       for (int rr = 0; rr < RPW; ++rr) {
@@ -655,7 +663,7 @@ quantize_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float
       }
       if (tid < 2 * D) hr.sc.put(tid, 0.0f);
       break;
-    default: quantize_warp<MIXED, Store>(cs, wr, hr, wstart, src); break;
+    default: quantize_warp<MIXED, Store, H16>(cs, wr, hr, wstart, src); break;
   }
 }
 

@@ -37,8 +37,8 @@ namespace {
 // Five CTA barriers: column maximum, and per least-squares step one for the partial sums
 // and one for the new 1/c.
 // ---------------------------------------------------------------------------------
-template <int BITS>
-__device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], const Scales& sc,
+template <int BITS, class Sc>
+__device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], const Sc& sc,
                                             uint8_t* codes_global, int warp_code_start, float* o_global) {
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r0 = w * RPW;
@@ -205,10 +205,10 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
         // every least-squares step keeps c >= c_before / 2 (each term Q y >= c Q^2 / 2),
         // so |n| = |rint(y / c)| <= qmax c0 / c + 1/2 < 2^15 unless rounding at the bottom
         // of the float32 range broke that; then the column takes the float clamp
-        if (BITS != MIXED && it == 1) wide = !(fmul(c0, icn) < 128.0f);
+        if (it == 1) wide = !(fmul(c0, icn) < 128.0f);
       }
     }
-    if (BITS != MIXED && it == 1) any_wide = __syncthreads_or(wide);
+    if (it == 1) any_wide = __syncthreads_or(wide);
     else __syncthreads();
   }
 
@@ -230,6 +230,40 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
         const f2 t23 = fma2(s[rr][1], ic[1], dup(MB));
         store_codes_s16<BITS>(codes_global + warp_code_start + rr * (D * BITS / 8), lane, t01, t23, HI);
       }
+      return;
+    }
+  } else {
+    if (!any_wide) {
+      // Mixed widths: clamp in 16-bit lanes, pack any width without a branch, and put
+      // each lane's b/2 bytes into the warp's staging area (the staged codes are consumed
+      // by now; it has the pool's layout), then copy the area out with 16-byte stores.
+      uint8_t* stage = wr.codes;
+#pragma unroll
+      for (int rr = 0; rr < RPW; ++rr) {
+        const uint32_t info = wr.info[rr];
+        const int bits = row_bits(info);
+        if (bits == PIVOT) continue;
+        const f2 mb = dup(wr.mb[rr]);
+        const f2 t01 = fma2(s[rr][0], ic[0], mb);
+        const f2 t23 = fma2(s[rr][1], ic[1], mb);
+        const uint32_t M = (1u << bits) - 1u;
+        const uint32_t w01 = clamp_s16x2(__byte_perm(__float_as_uint(t01.x), __float_as_uint(t01.y), 0x5410), M * 0x00010001u);
+        const uint32_t w23 = clamp_s16x2(__byte_perm(__float_as_uint(t23.x), __float_as_uint(t23.y), 0x5410), M * 0x00010001u);
+        const uint32_t x01 = (w01 & M) | (w01 >> (16 - bits));      // u0 | u1 << b
+        const uint32_t x23 = (w23 & M) | (w23 >> (16 - bits));      // u2 | u3 << b
+        const uint32_t f = x01 | (x23 << (2 * bits));
+        uint8_t* dst = stage + (row_off(info) - warp_code_start) + ((bits * lane) >> 1);
+        dst[0] = static_cast<uint8_t>(f);
+        if (bits >= 4) dst[1] = static_cast<uint8_t>(f >> 8);
+        if (bits >= 6) dst[2] = static_cast<uint8_t>(f >> 16);
+        if (bits >= 8) dst[3] = static_cast<uint8_t>(f >> 24);
+      }
+      // bytes of this warp's rows: 16 b per quantised row
+      const uint32_t my = lane < RPW ? (row_bits(wr.info[lane]) == PIVOT ? 0u : 16u * row_bits(wr.info[lane])) : 0u;
+      const int bytes = int(__reduce_add_sync(0xffffffffu, my));
+      __syncwarp();
+      for (int o = 16 * lane; o < bytes; o += 16 * 32)
+        *reinterpret_cast<uint4*>(codes_global + warp_code_start + o) = *reinterpret_cast<const uint4*>(stage + o);
       return;
     }
   }
@@ -270,8 +304,8 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
 
 // The quantiser of the method: dual-axis refit (refit_store).
 struct StepQuantStore {
-  template <int BITS>
-  static __device__ __forceinline__ void store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], const Scales& sc,
+  template <int BITS, class Sc>
+  static __device__ __forceinline__ void store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], const Sc& sc,
                                                uint8_t* codes, int warp_code_start, float* o) {
     refit_store<BITS>(cs, wr, s, sc, codes, warp_code_start, o);
   }
@@ -288,6 +322,7 @@ __device__ __forceinline__ void dequant_row(const uint8_t* row, int lane, float 
   *reinterpret_cast<float4*>(dst) = make_float4(a.x, a.y, b.x, b.y);
 }
 
+template <bool H16>
 __global__ void __launch_bounds__(NT)
 dequant_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, float* __restrict__ S_out) {
   extern __shared__ __align__(16) uint8_t stage[];
@@ -301,7 +336,7 @@ dequant_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, float* __res
     if (tid == 0) atomicOr(P.err, ERR_SLOT_RANGE);
     return;
   }
-  const HeadRef hr = head_ref(P, slot, h);
+  const HeadRef<H16> hr = head_ref<H16>(P, slot, h);
   if (tid < D) {
     info_s[tid] = P.row_info[h * D + tid];
     r_s[tid] = hr.sc.get(tid);
@@ -423,6 +458,7 @@ cudaError_t prepare(K kernel, int dyn, int static_bytes, int* done_per_device) {
 }
 
 int g_dequant_dyn[64];
+int g_dequant_dyn16[64];
 
 }  // namespace
 
@@ -431,10 +467,14 @@ cudaError_t launch_decode(const PoolDev& P, const int32_t* slots, int B, const f
                           const float* beta, float* out, cudaStream_t s) {
   if (B == 0) return cudaSuccess;
   if (P.scheme == SCHEME_ROW_ABSMAX) return launch_decode_absmax(P, slots, B, q, k, v, gate, beta, out, s);
-  if (P.any_mixed)
-    decode_kernel<StepQuantStore, true><<<B * P.H, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
-  else
-    decode_kernel<StepQuantStore, false><<<B * P.H, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+  const unsigned grid = unsigned(B) * unsigned(P.H);
+  if (P.scale16) {
+    if (P.any_mixed) decode_kernel<StepQuantStore, true, true><<<grid, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+    else decode_kernel<StepQuantStore, false, true><<<grid, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+  } else {
+    if (P.any_mixed) decode_kernel<StepQuantStore, true, false><<<grid, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+    else decode_kernel<StepQuantStore, false, false><<<grid, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+  }
   return cudaGetLastError();
 }
 
@@ -442,7 +482,8 @@ cudaError_t launch_quantize(const PoolDev& P, const int32_t* slots, int B, const
                             cudaStream_t s) {
   if (B == 0) return cudaSuccess;
   if (P.scheme == SCHEME_ROW_ABSMAX) return launch_quantize_absmax(P, slots, B, S, s);
-  quantize_kernel<StepQuantStore><<<B * P.H, NT, 0, s>>>(P, slots, B, S);
+  if (P.scale16) quantize_kernel<StepQuantStore, true><<<B * P.H, NT, 0, s>>>(P, slots, B, S);
+  else quantize_kernel<StepQuantStore, false><<<B * P.H, NT, 0, s>>>(P, slots, B, S);
   return cudaGetLastError();
 }
 
@@ -450,9 +491,15 @@ cudaError_t launch_dequantize(const PoolDev& P, const int32_t* slots, int B, flo
                               cudaStream_t s) {
   if (B == 0) return cudaSuccess;
   const int dyn = stage_bytes(P);
-  cudaError_t e = prepare(dequant_kernel, dyn, 2 * D * 4, g_dequant_dyn);
-  if (e != cudaSuccess) return e;
-  dequant_kernel<<<B * P.H, NT, dyn, s>>>(P, slots, B, S_out);
+  if (P.scale16) {
+    cudaError_t e = prepare(dequant_kernel<true>, dyn, 2 * D * 4, g_dequant_dyn16);
+    if (e != cudaSuccess) return e;
+    dequant_kernel<true><<<B * P.H, NT, dyn, s>>>(P, slots, B, S_out);
+  } else {
+    cudaError_t e = prepare(dequant_kernel<false>, dyn, 2 * D * 4, g_dequant_dyn);
+    if (e != cudaSuccess) return e;
+    dequant_kernel<false><<<B * P.H, NT, dyn, s>>>(P, slots, B, S_out);
+  }
   return cudaGetLastError();
 }
 
