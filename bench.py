@@ -44,8 +44,8 @@ FP32_LANES_PER_SM = 128
 # ncu dram bytes (read + write) per launch of decode_kernel on the default workload
 # (GDN B = 512, dual-axis refit), and the sha256 of the kernel sources they were taken
 # with (a changed kernel voids them).
-TRAFFIC = {"bytes": 2 * (193_313_792 + 124_232_960),
-           "kernel_sha256": "88937c4bbce30c2ee12ffde164e3d36b7a5bbc1c98287cd3d092d577967838cd",
+TRAFFIC = {"bytes": 2 * (193_273_600 + 123_231_488),
+           "kernel_sha256": "07816bfe652c95833ef7d11cbd54d4b0bcf20aeed002659210d0eadc15147692",
            "source": "profiles/decode_kernel_gdn_b256_h48_nominal6.md: dram read + write of one "
                      "B = 256 launch, doubled for B = 512 (traffic grows with B)"}
 
