@@ -186,12 +186,12 @@ __device__ __forceinline__ void store_codes_s16(uint8_t* row, int lane, f2 t01, 
   } else {
     const uint32_t x01 = w01 | (w01 >> 10), x23 = w23 | (w23 >> 10);
     const uint32_t f = (x01 & 0xFFFu) | (x23 << 12);   // bits 24.. are not stored
-    const bool odd = lane & 1;
-    uint8_t* p = row + 3 * lane;
-    uint8_t* p8 = odd ? p : p + 2;
-    uint16_t* p16 = reinterpret_cast<uint16_t*>(odd ? p + 1 : p);
-    *p8 = static_cast<uint8_t>(odd ? f : (f >> 16));
-    *p16 = static_cast<uint16_t>(odd ? (f >> 8) : f);
+    // even lanes: 16 bits at byte 3l, 8 bits at 3l + 2; odd lanes: 8 bits at 3l, 16 at 3l + 1
+    const int odd = lane & 1;
+    uint8_t* p8 = row + 3 * lane + 2 - 2 * odd;
+    uint16_t* p16 = reinterpret_cast<uint16_t*>(row + 3 * lane + odd);
+    *p8 = static_cast<uint8_t>(f >> (16 - 16 * odd));
+    *p16 = static_cast<uint16_t>(f >> (8 * odd));
   }
 }
 
