@@ -44,8 +44,8 @@ FP32_LANES_PER_SM = 128
 # ncu dram bytes (read + write) per launch of decode_kernel on the default workload
 # (GDN B = 512, dual-axis refit), and the sha256 of the kernel sources they were taken
 # with (a changed kernel voids them).
-TRAFFIC = {"bytes": 2 * (193_273_600 + 123_231_488),
-           "kernel_sha256": "07816bfe652c95833ef7d11cbd54d4b0bcf20aeed002659210d0eadc15147692",
+TRAFFIC = {"bytes": 2 * (193_261_568 + 123_363_840),
+           "kernel_sha256": "3f58e06bb960e1b5bbb983ff698ba47d89f8cc2fc12b955f86680aca7464f5a4",
            "source": "profiles/decode_kernel_gdn_b256_h48_nominal6.md: dram read + write of one "
                      "B = 256 launch, doubled for B = 512 (traffic grows with B)"}
 
