@@ -450,6 +450,27 @@ def stq_arm(args, rank, world, local_rank):
         e2e = {"value": whole_job_rate(B * H, world, te / n_e), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": B * H * D * 4, "steps": n_e}
 
+    # the FP32-state step on the same shapes (the pages' comparison point for the
+    # state-update speed-up), timed the same way; per rank, no collective
+    fp32_ms = None
+    if args.fp32_steps > 0:
+        S32 = torch.zeros((B, H, D, D), device=dev)
+        for i in range(3):
+            q_, k_, v_, g_, b_ = inputs[i % n_sets]
+            stq.fp32_decode_step(w.kind, S32, q_, k_, v_, g_, b_, out, stream)
+        torch.cuda.synchronize()
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for i in range(args.fp32_steps):
+            q_, k_, v_, g_, b_ = inputs[i % n_sets]
+            stq.fp32_decode_step(w.kind, S32, q_, k_, v_, g_, b_, out, stream)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        fp32_ms = g0.elapsed_time(g1) / args.fp32_steps
+        del S32
+        torch.cuda.empty_cache()
+
     if rank != 0:
         return
     hbm_peak, smax, which = peaks()
@@ -488,6 +509,11 @@ def stq_arm(args, rank, world, local_rank):
     }
     if drift is not None:
         line["drift"] = drift
+    if fp32_ms is not None:
+        line["fp32_state_step"] = {
+            "ms_per_step": fp32_ms, "steps": args.fp32_steps,
+            "packed_speedup_vs_fp32": fp32_ms / ms_step,
+            "note": "FP32-state gated delta step (fp32_step_kernel) on the same shapes and inputs"}
     if world == 1 and not args.no_cpu_baseline:
         rate, info = oracle_rate(w, budget_s=args.cpu_budget, scheme=args.scheme)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, **info, "cpu": cpu_model()}
@@ -516,6 +542,8 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-cpu-all-cores", action="store_true", help="skip the all-cores oracle timing")
+    ap.add_argument("--fp32-steps", type=int, default=200,
+                    help="time this many FP32-state steps on the same shapes (0: skip)")
     ap.add_argument("--drift-steps", type=int, default=0,
                     help="after timing, chain this many steps on 64 requests against the FP32 state")
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling captures only)")
