@@ -21,6 +21,7 @@ import hashlib
 import json
 import os
 import statistics
+import tempfile
 import subprocess
 import sys
 import time
@@ -130,7 +131,8 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.path = os.path.join(os.environ.get("STQ_CLOCKS_DIR", tempfile.gettempdir()),
+                                 f"stq_clocks_{os.getpid()}_gpu{gpu_index}.csv")
 
     def start(self):
         try:

@@ -13,7 +13,7 @@ singularity-lens calibration paragraph; ai-trend review, Method (1)):
     for a 4-bit budget and {4,6,8} for a 6-bit one;
   * a few highest-risk units are kept in FP16 as pivots.
 
-Readings where the pages are silent (also listed in the design doc):
+Readings where the pages are silent:
   * J = 1024, the decode length of the pages' throughput protocol.
   * Risk of a unit = L_u D_u(b_max): the weighted distortion it keeps even at the widest
     integer width (the pages keep in FP16 the units "a bit or two more" cannot save).

@@ -10,7 +10,7 @@ Errors Matter in Delta-Rule Recurrent State Quantization" (arXiv 2609.38169):
   ai-trend    = ai-trend.me review
   zhichai     = zhichai.net forum page
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   * Arithmetic precision: the state and its update are float32 (the pages compare
     everything against an FP32 state and read out in floating point before
     requantising: lens, decode-order paragraph; zhichai forum reply).
