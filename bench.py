@@ -46,16 +46,21 @@ FP32_LANES_PER_SM = 128
 # (GDN B = 512, dual-axis refit), and the sha256 of the kernel sources they were taken
 # with (a changed kernel voids them).
 TRAFFIC = {"bytes": 2 * (193_261_568 + 123_363_840),
-           "kernel_sha256": "3f58e06bb960e1b5bbb983ff698ba47d89f8cc2fc12b955f86680aca7464f5a4",
+           "kernel_sha256": "7ac10199c237573a9aca385d8b9e9920f52047f3bb456c253cf580dc91c6cabb",
            "source": "profiles/decode_kernel_gdn_b256_h48_nominal6.md: dram read + write of one "
                      "B = 256 launch, doubled for B = 512 (traffic grows with B)"}
 
 
 def kernel_sha():
-    """sha256 over the sources the decode kernel is compiled from."""
+    """sha256 over the code (comments and blank lines dropped) of the sources the decode
+    kernel is compiled from: a comment edit keeps the counters, a code edit voids them."""
+    import re
     h = hashlib.sha256()
     for f in ("stq_device.cuh", "stq_kernels.cu", "stq_internal.h"):
-        h.update(open(os.path.join(ROOT, "quantized_linear_attention_02_b200", "csrc", f), "rb").read())
+        src = open(os.path.join(ROOT, "quantized_linear_attention_02_b200", "csrc", f)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update("\n".join(ln.rstrip() for ln in src.splitlines() if ln.strip()).encode())
     return h.hexdigest()
 
 

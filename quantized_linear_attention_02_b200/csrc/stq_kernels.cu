@@ -21,8 +21,13 @@
 //     fma(a_2m, b_2m, a_2m+1 * b_2m+1); the state update is S = fma(k, delta, S'); every
 //     other product is rounded on its own (explicit _rn forms, --fmad=false);
 //   * the quantiser's x = y * inv_c is taken exactly: fma(y, inv_c, 1.5*2^23) rounds the
-//     exact product to the nearest integer (ties to even) inside the 2^23 binade, and
-//     clamping is done in that binade, where the low bits are the (biased) code.
+//     exact product to the nearest integer (ties to even) inside the 2^23 binade, where
+//     the low bits are the (biased) code; the least-squares step clamps in that binade,
+//     the final codes clamp in 16-bit lanes (same result, see refit_store).
+//
+// This file holds the dual-axis refit (the quantiser of the method), the dequantise and
+// FP32-state kernels and the launchers; the kernel bodies shared with the row-absmax
+// baseline are in stq_device.cuh.
 #include "stq_device.cuh"
 
 namespace stq {
