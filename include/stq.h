@@ -29,7 +29,10 @@
  *     pool handle owns only host memory (freed by stq_pool_destroy).
  *   - Kernels check slot indices against n_slots; a bad index sets a sticky error
  *     bit in the pool's device metadata and that (request, head) is skipped.
- *     stq_pool_check() reads and clears it.
+ *     stq_pool_check() reads and clears it. A checked build of the library (compiled
+ *     with STQ_CHECKS; stq_version() then says "checked") also records stored codes 0
+ *     (never written by the quantiser: an uninitialised or corrupted slot) and
+ *     non-finite updated states; those heads are still processed.
  *   - No call may list the same slot twice in one batch.
  *   - Errors: a non-zero stq_status; stq_last_error() gives a message (thread-local).
  *   - No C++ exception crosses this boundary.
@@ -49,7 +52,7 @@ typedef enum {
   STQ_ERR_INVALID_ARG = 1,   /* a size, kind, width or pointer is invalid */
   STQ_ERR_ALIGNMENT = 2,     /* a device pointer is not 16-byte aligned */
   STQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
-  STQ_ERR_DEVICE_CHECK = 4   /* a kernel found a bad slot index (stq_pool_check) */
+  STQ_ERR_DEVICE_CHECK = 4   /* a kernel recorded a device check (stq_pool_check) */
 } stq_status;
 
 typedef enum { STQ_GDN = 0, STQ_KDA = 1 } stq_kind;

@@ -20,31 +20,35 @@ FLAGS = [
 ]
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+LIB_CHECKED = os.path.join(HERE, "libstq_checked.so")
+
+
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(HERE, s) for s in SOURCES]
     deps += [os.path.join(HERE, "csrc", h) for h in ("stq_internal.h", "stq_device.cuh")]
     deps += [os.path.join(ROOT, "include", "stq.h")]
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra=None) -> str:
-    if not force and not needs_build():
-        return LIB
-    cmd = [NVCC] + FLAGS + (extra or []) + ["-I", os.path.join(ROOT, "include"),
-                                            "-I", os.path.join(HERE, "csrc"), "-o", LIB]
+def build(force: bool = False, verbose: bool = False, extra=None, checked: bool = False) -> str:
+    """Compile libstq.so; checked=True compiles libstq_checked.so with STQ_CHECKS (device
+    checks that record stored codes 0 and non-finite states in the pool's error word)."""
+    lib = LIB_CHECKED if checked else LIB
+    if not force and not needs_build(lib):
+        return lib
+    cmd = [NVCC] + FLAGS + (["-DSTQ_CHECKS"] if checked else []) + (extra or [])
+    cmd += ["-I", os.path.join(ROOT, "include"), "-I", os.path.join(HERE, "csrc"), "-o", lib + ".tmp"]
     cmd += [os.path.join(HERE, s) for s in SOURCES]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
-    tmp = LIB + ".tmp"
-    cmd[cmd.index(LIB)] = tmp
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True,
+    build(force="--force" in sys.argv, verbose=True, checked="--checked" in sys.argv,
           extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None)

@@ -173,7 +173,11 @@ extern "C" {
 
 const char* stq_last_error(void) { return g_last_error.c_str(); }
 
+#ifdef STQ_CHECKS
+const char* stq_version(void) { return "stq 0.1 (sm_100a, checked)"; }
+#else
 const char* stq_version(void) { return "stq 0.1 (sm_100a)"; }
+#endif
 
 stq_status stq_pool_layout(const stq_pool_desc* desc, stq_pool_sizes* out) {
   if (out == nullptr) return fail(STQ_ERR_INVALID_ARG, "out is NULL");
@@ -406,8 +410,11 @@ stq_status stq_pool_check(stq_pool* pool, void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "clear of device error word");
     if (bits[0] & stq::ERR_SLOT_RANGE)
       return fail(STQ_ERR_DEVICE_CHECK, "a slot index was outside [0, n_slots); those heads were skipped");
-    if (bits[0] & stq::ERR_TIMEOUT)
-      return fail(STQ_ERR_DEVICE_CHECK, "a kernel gave up waiting for its staged inputs; its outputs are incomplete");
+    if (bits[0] & stq::ERR_CODE)
+      return fail(STQ_ERR_DEVICE_CHECK, "a stored code was 0, which the quantiser never writes: "
+                                        "a slot was decoded before stq_quantize_init or is corrupted");
+    if (bits[0] & stq::ERR_NONFINITE)
+      return fail(STQ_ERR_DEVICE_CHECK, "the updated state held a NaN or an infinity (non-finite inputs?)");
     return fail(STQ_ERR_DEVICE_CHECK, "device error bits 0x%x", bits[0]);
   }
   return ok();

@@ -241,11 +241,13 @@ struct HeadRef {
   int piv_count;
   int bits;            // uniform width of the head, 16 if all pivot, 0 if mixed
   int piv_stage_off;   // byte offset of the pivot rows in the staging buffer
+  uint32_t* err;       // the pool's sticky error word (checked builds record into it)
 };
 
 template <bool H16>
 __device__ __forceinline__ HeadRef<H16> head_ref(const PoolDev& P, int slot, int h) {
   HeadRef<H16> r;
+  r.err = P.err;
   r.code_bytes = int(P.head_code_bytes[h]);
   r.piv_count = int(P.head_piv_count[h]);
   r.bits = int(P.head_bits[h]);
@@ -391,6 +393,9 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
                                             float* o_out) {
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   f2 s[RPW][2];
+#ifdef STQ_CHECKS
+  bool zero_code = false;   // a stored code 0: never written by the quantiser
+#endif
 
   // ---- restore S' = D (r c Q) and the column sums u_j = sum_i k_i S'_ij ---------------
 #pragma unroll
@@ -408,6 +413,10 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
           const int bitpos = 4 * bits * lane;
           const uint32_t f = __funnelshift_r(wp[bitpos >> 5], wp[(bitpos >> 5) + 1], bitpos & 31);
           const uint32_t M = (1u << bits) - 1u;
+#ifdef STQ_CHECKS
+          zero_code |= (f & M) == 0 || ((f >> bits) & M) == 0 || ((f >> (2 * bits)) & M) == 0 ||
+                       ((f >> (3 * bits)) & M) == 0;
+#endif
           // 2^23 + bias as a float: the bias sits in the mantissa
           const f2 ntb = dup(-__uint_as_float(FLOAT_2P23 | (1u << (bits - 1))));
           const f2 q01 = add2(make_float2(__uint_as_float((f & M) | FLOAT_2P23),
@@ -430,6 +439,11 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
     } else {
       uint32_t cd[4];
       load_codes<BITS>(wr.codes + rr * (D * BITS / 8), lane, cd);
+#ifdef STQ_CHECKS
+      // the mantissa of an unpacked code holds u << pos: zero exactly when u = 0
+      zero_code |= ((cd[0] & 0x7FFFFFu) == 0) || ((cd[1] & 0x7FFFFFu) == 0) ||
+                   ((cd[2] & 0x7FFFFFu) == 0) || ((cd[3] & 0x7FFFFFu) == 0);
+#endif
       const float4 r2 = *reinterpret_cast<const float4*>(&wr.rdd[rr & ~1]);
       const f2 rd = (rr & 1) ? make_float2(r2.z, r2.w) : make_float2(r2.x, r2.y);
       f2 q01, q23;
@@ -487,6 +501,18 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
         *reinterpret_cast<uint2*>(hr.pivots + row_off(info) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
     }
   }
+#ifdef STQ_CHECKS
+  {
+    bool nonfinite = false;
+#pragma unroll
+    for (int rr = 0; rr < RPW; ++rr)
+      nonfinite |= !isfinite(s[rr][0].x) || !isfinite(s[rr][0].y) || !isfinite(s[rr][1].x) ||
+                   !isfinite(s[rr][1].y);
+    const uint32_t bits = (__any_sync(0xffffffffu, zero_code) ? ERR_CODE : 0u) |
+                          (__any_sync(0xffffffffu, nonfinite) ? ERR_NONFINITE : 0u);
+    if (lane == 0 && bits) atomicOr(hr.err, bits);
+  }
+#endif
   Store::template store<BITS>(cs, wr, s, hr.sc, hr.codes, warp_code_start, o_out);
 }
 

@@ -18,7 +18,11 @@ constexpr int SCHEME_ROW_ABSMAX = 1;   // symmetric per-key-row absmax baseline
 
 // Error bits written by kernels into the pool's device error word.
 constexpr uint32_t ERR_SLOT_RANGE = 1u;   // a slot index was outside [0, n_slots)
-constexpr uint32_t ERR_TIMEOUT = 2u;      // a wait for staged inputs gave up
+// Checked builds only (compiled with STQ_CHECKS): the decode step and the dequantiser
+// also record
+constexpr uint32_t ERR_CODE = 2u;         //   a stored code 0, which the quantiser never
+                                          //   writes (an uninitialised or corrupted slot)
+constexpr uint32_t ERR_NONFINITE = 4u;    //   a NaN or infinity in the updated state
 
 // Device view of a pool: caller-owned state buffers plus the metadata the library
 // uploaded into the caller-owned meta buffer. Passed to kernels by value.

@@ -47,14 +47,16 @@ _i = ctypes.c_int
 
 
 def lib():
-    """Load libstq.so (built in-tree by build.py); raise if it is missing."""
+    """Load libstq.so (built in-tree by build.py; the environment variable STQ_LIBRARY may
+    name another build of it, e.g. the checked one); raise if it is missing."""
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+    path = os.environ.get("STQ_LIBRARY", LIB_PATH)
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
                            "`python -m quantized_linear_attention_02_b200.build`")
-    L = ctypes.CDLL(LIB_PATH)
+    L = ctypes.CDLL(path)
     sig = {
         "stq_pool_layout": (_i, [ctypes.POINTER(_Desc), ctypes.POINTER(_Sizes)]),
         "stq_pool_create": (_i, [ctypes.POINTER(_Desc), _vp, _vp, _vp, _vp, ctypes.POINTER(_vp)]),
