@@ -409,3 +409,38 @@ def test_scale16_quantize_step_and_chain(widx, scheme):
     Sd = torch.empty((len(reqs), w.H, D, D), device="cuda")
     pool.dequantize(slots_t(reqs), Sd)
     assert np.array_equal(Sd.cpu().numpy(), O.dequantize(ug, rg, cg, pg, rb))
+
+
+# ---------------------------------------------------------------------------------
+# every width on the uniform-width code paths (each head one width), both kinds
+# ---------------------------------------------------------------------------------
+@pytest.mark.parametrize("widx", [1, 2])
+@pytest.mark.parametrize("bits", [2, 4, 6, 8])
+def test_uniform_width_paths_step(widx, bits):
+    w = W.WORKLOADS[widx]
+    reqs = [0, 1]
+    rb = np.full((w.H, D), bits)
+    ub = np.full(w.H if w.kind == "gdn" else w.H * D, bits, np.uint8)
+    om = W.omega(w)
+    pool = stq.Pool(w.kind, 4, ub, om)
+    L = O.Layout(rb)
+    slots = [1, 3]
+    S0 = T.warm_state(w.index, tuple(reqs))
+    u, r, c, piv = O.refit(S0, om, rb)
+    pool.quantize_init(torch.tensor(slots, dtype=torch.int32, device="cuda"), dev(S0))
+    pool.check()
+    ug, rg, cg, _ = T.read_pool_state(pool, L, slots)
+    if T.compare_codes(ug, u, S0, r, c, rb, f"{bits}-bit quantize") == 0:
+        assert np.array_equal(rg, r) and np.array_equal(cg, c)
+    T.write_oracle_state(pool, L, slots, u, r, c, piv)
+    x = T.inputs_for(w, "decode", 3, reqs)
+    u2, r2, c2, p2, o, X = O.decode_step(u, r, c, piv, rb, om, x.q, x.k, x.v,
+                                         O.gate_rows(x.gate, w.kind, D), x.beta)
+    out = torch.empty((2, w.H, D), device="cuda")
+    pool.decode_step(torch.tensor(slots, dtype=torch.int32, device="cuda"), dev(x.q), dev(x.k), dev(x.v),
+                     dev(x.gate), dev(x.beta), out)
+    pool.check()
+    ug, rg, cg, _ = T.read_pool_state(pool, L, slots)
+    if T.compare_codes(ug, u2, X, r2, c2, rb, f"{bits}-bit step") == 0:
+        assert np.array_equal(rg, r2) and np.array_equal(cg, c2)
+    assert T.per_vector_rel_l2(out.cpu().numpy(), o).max() <= T.OUT_REL_L2
