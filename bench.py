@@ -454,8 +454,61 @@ def stq_arm(args, rank, world, local_rank):
             dist.barrier()
         te = max_over_ranks(f0.elapsed_time(f1), world, dev)
         h2d = sum(x.numel() * 4 for x in pin[0])
-        e2e = {"value": whole_job_rate(B * H, world, te / n_e), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": B * H * D * 4, "steps": n_e}
+        serial = {"value": whole_job_rate(B * H, world, te / n_e), "unit": UNIT,
+                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": B * H * D * 4, "steps": n_e,
+                  "form": "stq_decode_step_host: copies in, step, copy out on one stream"}
+
+        # The same steps pipelined two deep, as a serving loop would run them: step i's
+        # inputs go up on a copy stream while step i-1 computes, its readout comes down on
+        # a third stream while step i+1 computes; the decode steps stay in order on the
+        # compute stream (each reads the state the previous one wrote).
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        dbuf = [[torch.empty_like(x) for x in inputs[0]] for _ in range(2)]
+        d_out = [torch.empty((B, H, D), device=dev) for _ in range(2)]
+        h_outs = [torch.empty((B, H, D), dtype=torch.float32).pin_memory() for _ in range(2)]
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_step = [torch.cuda.Event() for _ in range(2)]
+        ev_free = [torch.cuda.Event() for _ in range(2)]
+        for j in range(2):
+            ev_free[j].record(stream)
+
+        def piped(i):
+            j = i % 2
+            up.wait_event(ev_free[j])                 # step i-2 is done with buffer j
+            with torch.cuda.stream(up):
+                for dst, src in zip(dbuf[j], pin[i % 2]):
+                    dst.copy_(src, non_blocking=True)
+            ev_in[j].record(up)
+            stream.wait_event(ev_in[j])
+            pool.decode_step(slots, *dbuf[j], d_out[j], stream)
+            ev_step[j].record(stream)
+            down.wait_event(ev_step[j])
+            with torch.cuda.stream(down):
+                h_outs[j].copy_(d_out[j], non_blocking=True)
+            ev_free[j].record(down)
+
+        for i in range(3):
+            piped(i)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        p0 = torch.cuda.Event(enable_timing=True)
+        p1 = torch.cuda.Event(enable_timing=True)
+        p0.record(stream)
+        for i in range(n_e):
+            piped(i)
+        for j in range(2):
+            stream.wait_event(ev_free[j])             # the last readouts are on the host
+        p1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        tp = max_over_ranks(p0.elapsed_time(p1), world, dev)
+        e2e = {"value": whole_job_rate(B * H, world, tp / n_e), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": B * H * D * 4, "steps": n_e,
+               "form": "stq_decode_step on device buffers, host copies pipelined two deep "
+                       "(H2D, step and D2H on three streams)",
+               "serial": serial}
 
     # the FP32-state step on the same shapes (the pages' comparison point for the
     # state-update speed-up), timed the same way; per rank, no collective
