@@ -34,6 +34,12 @@
  *     (never written by the quantiser: an uninitialised or corrupted slot) and
  *     non-finite updated states; those heads are still processed.
  *   - No call may list the same slot twice in one batch.
+ *   - Stream capture: stq_decode_step, stq_quantize_init, stq_dequantize,
+ *     stq_decode_step_host and stq_row_sq_error only enqueue work on `stream` (no
+ *     allocation, no synchronisation), so they can be recorded into a CUDA graph. Make
+ *     the first call of stq_dequantize and of stq_decode_step_host_static on a device
+ *     outside capture (each sets itself up once per device); stq_pool_check
+ *     synchronises and cannot be captured.
  *   - Errors: a non-zero stq_status; stq_last_error() gives a message (thread-local).
  *   - No C++ exception crosses this boundary.
  */
