@@ -444,3 +444,62 @@ def test_uniform_width_paths_step(widx, bits):
     if T.compare_codes(ug, u2, X, r2, c2, rb, f"{bits}-bit step") == 0:
         assert np.array_equal(rg, r2) and np.array_equal(cg, c2)
     assert T.per_vector_rel_l2(out.cpu().numpy(), o).max() <= T.OUT_REL_L2
+
+
+# ---------------------------------------------------------------------------------
+# degenerate scales inside a head: zero rows and columns, rows whose scale falls below
+# 2^-126 (their reciprocal counts as 0), a row five decades larger than the rest, and
+# a head whose every row is below 2^-126 (c = 0: no least-squares denominator)
+# ---------------------------------------------------------------------------------
+def _degenerate_state(w, reqs):
+    S = T.warm_state(w.index, tuple(reqs)).copy()
+    rb = W.row_bits(w)
+    heads = [h for h in range(w.H) if rb[h, 0] != 16][:2]
+    h0, h1 = heads
+    S[0, h0, [3, 40], :] = 0.0
+    S[0, h0, :, [7, 100]] = 0.0
+    S[0, h0, 50, :] *= F32(1e-39)           # subnormal row: r < 2^-126
+    S[0, h0, 60, :] *= F32(1e5)             # (FP16 pivot rows stay finite after the step)
+    S[0, h1] *= F32(1e-40)                  # every row below 2^-126
+    return S, h0, h1
+
+
+@pytest.mark.parametrize("widx", [1, 2])
+@pytest.mark.parametrize("scheme", ["stepquant", "row_absmax"])
+def test_degenerate_rows_and_columns(widx, scheme):
+    w = W.WORKLOADS[widx]
+    reqs = [0, w.B - 1]
+    rb, om = W.row_bits(w), W.omega(w)
+    pool = stq.Pool(w.kind, W.n_slots(w.B), W.unit_bits(w), om, scheme=scheme)
+    L = O.Layout(rb)
+    slots = [W.slot_of_request(b) for b in reqs]
+    S0, h0, h1 = _degenerate_state(w, reqs)
+    quantise = (lambda S: O.absmax_quantise(S, rb)) if scheme == "row_absmax" else (lambda S: O.refit(S, om, rb))
+    u, r, c, piv = quantise(S0)
+    assert np.all(r[0, h1] == 0) or np.all(r[0, h1] < np.float32(2.0 ** -126))
+    pool.quantize_init(slots_t(reqs), dev(S0))
+    pool.check()
+    ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
+    if T.compare_codes(ug, u, S0, r, c, rb, "degenerate quantize_init") == 0:
+        assert np.array_equal(rg, r) and np.array_equal(cg, c)
+    piv_rows = rb == 16
+    assert np.array_equal(pg[:, piv_rows], piv[:, piv_rows])
+    # one step from the oracle's packed state; k_i = 0 keeps the zero rows zero and
+    # v_j = 0 (with u_j = 0) keeps the zero columns zero
+    T.write_oracle_state(pool, L, slots, u, r, c, piv)
+    x = T.inputs_for(w, "decode", 0, reqs)
+    k = x.k.copy()
+    v = x.v.copy()
+    k[0, h0, [3, 40]] = 0.0
+    v[0, h0, [7, 100]] = 0.0
+    u2, r2, c2, p2, o, X = O.decode_step(u, r, c, piv, rb, om, x.q, k, v,
+                                         O.gate_rows(x.gate, w.kind, D), x.beta, scheme=scheme)
+    assert np.all(X[0, h0, [3, 40]] == 0) and np.all(X[0, h0][:, [7, 100]] == 0)
+    out = torch.empty((len(reqs), w.H, D), device="cuda")
+    pool.decode_step(slots_t(reqs), dev(x.q), dev(k), dev(v), dev(x.gate), dev(x.beta), out)
+    pool.check()
+    ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
+    if T.compare_codes(ug, u2, X, r2, c2, rb, "degenerate step") == 0:
+        assert np.array_equal(rg, r2) and np.array_equal(cg, c2)
+    assert np.array_equal(pg[:, piv_rows], p2[:, piv_rows])
+    assert T.per_vector_rel_l2(out.cpu().numpy(), o).max() <= T.OUT_REL_L2
