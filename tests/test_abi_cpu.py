@@ -56,6 +56,34 @@ def test_layout_matches_oracle_layout(lib, w):
     assert got["max_head_bytes"] == max(heads)
 
 
+@pytest.mark.parametrize("seed", range(12))
+def test_layout_matches_oracle_layout_random_widths(lib, seed):
+    # random width maps: either kind, 1..5 heads, every width, pivot-only heads
+    rng = np.random.default_rng(500 + seed)
+    kind = ("gdn", "kda")[seed % 2]
+    H = int(rng.integers(1, 6))
+    n_slots = int(rng.integers(1, 9))
+    widths = np.array([2, 4, 6, 8, 16], np.uint8)
+    if kind == "gdn":
+        ub = rng.choice(widths, H)
+        rb = np.repeat(ub[:, None], 128, 1)
+    else:
+        rb = rng.choice(widths, (H, 128), p=[0.2, 0.3, 0.2, 0.2, 0.1]).astype(np.uint8)
+        if H > 1:
+            rb[H - 1] = 16 if seed % 4 == 1 else rb[H - 1]      # an all-pivot head
+        ub = rb.reshape(-1)
+    om = rng.lognormal(0, 1, (H, 128)).astype(np.float32)
+    got = stq.layout(kind, n_slots, ub.astype(np.uint8), om)
+    L = O.Layout(rb)
+    assert got["slot_code_bytes"] == L.slot_code_bytes
+    assert got["codes_bytes"] == n_slots * L.slot_code_bytes
+    assert got["n_pivot_rows"] == L.n_pivot_rows
+    assert got["scales_bytes"] == n_slots * H * 2 * 128 * 4
+    assert got["pivots_bytes"] == n_slots * L.n_pivot_rows * 128 * 2
+    heads = [int(L.code_len[h].sum() + 256 * (rb[h] == 16).sum()) for h in range(H)]
+    assert got["max_head_bytes"] == max(heads)
+
+
 @pytest.mark.parametrize("w", W.WORKLOADS[1:3], ids=lambda w: w.name)
 def test_absmax_scheme_keeps_the_layout(lib, w):
     args = (w.kind, W.n_slots(w.B), W.unit_bits(w), W.omega(w))
