@@ -40,6 +40,22 @@ def warm_state(widx: int, reqs: tuple, steps: int | None = None) -> np.ndarray:
     return W.scale_outlier_rows(S, w)
 
 
+def warm_states(widx: int, reqs, steps: int | None = None) -> np.ndarray:
+    """warm_state of several requests, one request per worker process (the warm-up of
+    each request is independent of the others). The pool is started with `spawn`, so it
+    is safe after CUDA is initialised; the workers run NumPy only."""
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    import os
+    reqs = [int(b) for b in reqs]
+    n = min(len(reqs), len(os.sched_getaffinity(0)))
+    if n <= 1:
+        return warm_state(widx, tuple(reqs), steps)
+    with cf.ProcessPoolExecutor(n, mp_context=mp.get_context("spawn")) as ex:
+        parts = list(ex.map(warm_state, [widx] * len(reqs), [(b,) for b in reqs], [steps] * len(reqs)))
+    return np.concatenate(parts, 0)
+
+
 def _cat(parts):
     return W.StepInputs(*[np.concatenate([getattr(p, n) for p in parts], 0)
                           for n in ("q", "k", "v", "gate", "beta")])

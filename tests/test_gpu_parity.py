@@ -166,11 +166,11 @@ def test_decode_chain(widx, steps):
 def test_full_size_sampled(widx):
     w = W.WORKLOADS[widx]
     pool, L, om = make_pool(w)
-    sample = [int(b) for b in W.parity_sample(w, 3)]
+    sample = [int(b) for b in W.parity_sample(w, 8)]
     # every request gets a state; the sampled ones get oracle-built ones
     g = torch.Generator(device="cuda").manual_seed(1234 + widx)
     S_all = torch.randn((w.B, w.H, D, D), device="cuda", generator=g) * 0.05
-    S0 = T.warm_state(widx, tuple(sample))
+    S0 = T.warm_states(widx, sample)
     S_all[sample] = dev(S0)
     all_slots = slots_t(range(w.B))
     pool.quantize_init(all_slots, S_all)

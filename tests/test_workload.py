@@ -45,3 +45,13 @@ def test_outlier_columns_scaled():
     h = 5
     mask = np.zeros(128, bool); mask[cols[h]] = True
     assert np.std(x.v[:, h, mask]) > 5 * np.std(x.v[:, h, ~mask])
+
+
+def test_parallel_warm_states_equal_serial():
+    # the spawn-pool warm-up the full-size parity tests use gives the serial states
+    import stq_testlib as T
+    w = W.WORKLOADS[2]
+    reqs = [3, 17, 40]
+    a = T.warm_states(w.index, reqs, steps=6)
+    b = T.warm_state(w.index, tuple(reqs), 6)
+    assert a.dtype == np.float32 and np.array_equal(a, b)
