@@ -16,7 +16,7 @@ singularity-lens calibration paragraph; ai-trend review, Method (1)):
 Readings where the pages are silent:
   * J = 1024, the decode length of the pages' throughput protocol.
   * Risk of a unit = L_u D_u(b_max): the weighted distortion it keeps even at the widest
-    integer width (the pages keep in FP16 the units "a bit or two more" cannot save).
+    integer width (the pages keep in FP16 the units that a few more bits would not rescue).
     The n_pivots riskiest units (ties: lower unit index first) become pivots first.
   * The remaining units share the budget: sum of their widths <= budget * (their count),
     solved exactly by dynamic programming over the total width in steps of 2 bits;
