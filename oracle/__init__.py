@@ -1,8 +1,9 @@
 """CPU oracle for the packed Delta-rule state decode step (test infrastructure).
 
 This package is the plain, slow, obviously-correct restatement of what the decode
-step (and of the offline bit allocation before it), used only by the tests, by `__graft_entry__.smoke()` and by the
-`cpu_baseline` / `--impl reference` legs of `bench.py`. The library's product path
+step computes (and of the offline bit allocation before it). It is used only by the
+tests, by `__graft_entry__.smoke()` and by the `cpu_baseline` / `--impl reference`
+legs of `bench.py`. The library's product path
 never imports, links or runs anything here, and nothing here imports the library:
 the two share no code, tables or constants. Only the seeded input generator
 (`quantized_linear_attention_02_b200.workload`, which holds none of the method's
