@@ -35,11 +35,13 @@
  *     non-finite updated states; those heads are still processed.
  *   - No call may list the same slot twice in one batch.
  *   - Stream capture: stq_decode_step, stq_quantize_init, stq_dequantize,
- *     stq_decode_step_host and stq_row_sq_error only enqueue work on `stream` (no
- *     allocation, no synchronisation), so they can be recorded into a CUDA graph. Make
- *     the first call of stq_dequantize and of stq_decode_step_host_static on a device
- *     outside capture (each sets itself up once per device); stq_pool_check
- *     synchronises and cannot be captured.
+ *     stq_decode_step_host, stq_row_sq_error and stq_row_error_at_widths only enqueue
+ *     work on `stream` (no allocation, no synchronisation), so they can be recorded
+ *     into a CUDA graph. Make the first call of stq_decode_step (or of a call that runs
+ *     it), stq_quantize_init, stq_dequantize and stq_decode_step_host_static on a device
+ *     outside capture: each sets itself up once per device (a kernel's shared-memory
+ *     limit, the number of CTAs the device holds at once, the static staging address).
+ *     stq_pool_check and the pipeline calls synchronise and cannot be captured.
  *   - Errors: a non-zero stq_status; stq_last_error() gives a message (thread-local).
  *   - No C++ exception crosses this boundary.
  */
@@ -112,14 +114,21 @@ typedef struct stq_pool stq_pool;
  * row is bits [b*j, b*j+b) of a little-endian bit stream, stored as
  * u = Q + 2^(b-1)); the float16 rows of its pivot units in (head, row) order; and
  * r[128], c[128] per head (float32, or binary16 when scale_bits is 16). Returns
- * STQ_ERR_INVALID_ARG on a bad description. */
+ * STQ_ERR_INVALID_ARG on a bad description. The pages fix what is stored -- integer
+ * codes of the unit's width times a row and a column scale, pivot units in FP16
+ * (bloombook section 4; ai-trend review, Method) -- and that a slot serves one request
+ * (zhichai forum reply: five slots per request); the byte layout is this library's. */
 stq_status stq_pool_layout(const stq_pool_desc* desc, stq_pool_sizes* out);
 
 /* Bind caller-allocated device buffers (sizes from stq_pool_layout) to a new pool
  * handle and upload the static metadata (offsets, widths, omega_i and the row gain
  * g_i = (omega_i / mean omega)^(-1/2)) into d_meta with a synchronous copy. The
  * state buffers are not touched: fill them with stq_quantize_init. d_pivots may be
- * NULL when the pool has no pivot rows. */
+ * NULL when the pool has no pivot rows. The widths and row influences are fixed once
+ * for all requests (ai-trend review, Method (1); singularity-lens calibration
+ * paragraph); the row gain is the omega_i^(-1/2) factor of the row scale (bloombook
+ * section 4). Errors: STQ_ERR_INVALID_ARG (description, NULL buffers),
+ * STQ_ERR_ALIGNMENT, STQ_ERR_CUDA (the metadata copy). */
 stq_status stq_pool_create(const stq_pool_desc* desc, void* d_codes, void* d_scales,
                            void* d_pivots, void* d_meta, stq_pool** out);
 
@@ -133,8 +142,9 @@ void stq_pool_destroy(stq_pool* pool);
 stq_status stq_quantize_init(stq_pool* pool, const int32_t* d_slots, int B,
                              const float* d_S, void* stream);
 
-/* One decode step for B requests (THE hot path). For request b and head h, with
- * slot s = d_slots[b]:
+/* One decode step for B requests (THE hot path; the fused decode kernel of bloombook
+ * section 4 and the decode order of the singularity-lens summary). For request b and
+ * head h, with slot s = d_slots[b]:
  *   restore S' = D_t * dequantised state of (s, h), update with the gated delta rule,
  *   write out[b, h, :] = S_t^T q (float32, from the updated unquantised state), refit
  *   the scales and store S_t back into slot s packed.
@@ -159,6 +169,49 @@ stq_status stq_decode_step_host(stq_pool* pool, const int32_t* d_slots, int B,
                                 const float* h_gate, const float* h_beta, float* h_out,
                                 void* d_staging, size_t staging_bytes, void* stream);
 
+/* ---- The host-buffer step pipelined inside the library ---------------------------
+ * A serving loop that keeps its per-step inputs and outputs in host memory overlaps
+ * the copies with the decode: step i's inputs go up on the pipeline's upload stream
+ * while step i-1 decodes, and step i's readout comes down on its download stream while
+ * step i+1 decodes. The decode steps stay in order on the caller's stream, as the
+ * decode-order paragraph of the singularity-lens.com summary requires (each step reads
+ * the state the previous one wrote). The pipeline owns two CUDA streams and eight
+ * events (created by stq_pipeline_create, released by stq_pipeline_destroy) and no
+ * device memory: two halves of the caller's staging buffer alternate between steps. */
+typedef struct stq_pipeline stq_pipeline;
+
+/* Bytes of device staging a pipeline of B requests needs (two halves, each holding
+ * one step's q, k, v, gate, beta and readout); 0 for a NULL pool or B < 0. */
+size_t stq_pipeline_staging_bytes(const stq_pool* pool, int B);
+
+/* A pipeline for steps of B > 0 requests of `pool`, on the current device (make every
+ * later call on it with that device current). d_staging: caller-owned device buffer of
+ * staging_bytes >= stq_pipeline_staging_bytes(pool, B), 16-byte aligned, that the
+ * pipeline uses until stq_pipeline_destroy. Errors: STQ_ERR_INVALID_ARG (sizes, NULL),
+ * STQ_ERR_ALIGNMENT, STQ_ERR_CUDA (stream or event creation). */
+stq_status stq_pipeline_create(stq_pool* pool, int B, void* d_staging, size_t staging_bytes,
+                               stq_pipeline** out);
+
+/* Enqueue one decode step (stq_decode_step's operation; q, k, v, gate, beta and out
+ * have its shapes, in host memory, pinned for the copies to overlap): the inputs are
+ * copied up on the upload stream, the step runs on `stream`, its readout is copied
+ * into h_out on the download stream. Then the call waits on the host until the
+ * PREVIOUS call's readout is in that call's h_out, and returns. So on return the
+ * previous step's h_out is complete, and the host inputs and h_out of the step before
+ * it may be reused. d_slots (device, B entries) must stay unchanged until the step's
+ * decode has run. */
+stq_status stq_pipeline_step(stq_pipeline* pipe, const int32_t* d_slots, const float* h_q,
+                             const float* h_k, const float* h_v, const float* h_gate,
+                             const float* h_beta, float* h_out, void* stream);
+
+/* Wait on the host for the last step's readout, and make `stream` wait for it too
+ * (work enqueued on `stream` afterwards follows every pipelined copy). */
+stq_status stq_pipeline_finish(stq_pipeline* pipe, void* stream);
+
+/* Synchronise the pipeline's streams and release them and its events. NULL is
+ * ignored. The staging buffer stays the caller's. */
+void stq_pipeline_destroy(stq_pipeline* pipe);
+
 /* Bytes of the library's own device staging array used by
  * stq_decode_step_host_static (8 MiB). */
 #define STQ_STATIC_STAGING_BYTES (8u << 20)
@@ -178,7 +231,10 @@ stq_status stq_decode_step_host(stq_pool* pool, const int32_t* d_slots, int B,
  *   - Calls no cudaMalloc/cudaFree and no allocating routine.
  *   - The first call on each device looks up the array's device address (once per
  *     device, with that device current); make that first call before any stream
- *     capture on the device.
+ *     capture on the device. The address is kept per device ordinal for the life of
+ *     the process: it belongs to the device's primary context, so do not call this
+ *     entry point after cudaDeviceReset on that device, nor with a context other than
+ *     the primary one current (use stq_decode_step_host then).
  *   - All calls share the one array, which keeps the last call's contents (nothing in
  *     it needs to start at zero: each call writes every byte it reads). Calls whose
  *     work overlaps on the GPU (other streams, other host threads) race on it: order
@@ -189,7 +245,10 @@ stq_status stq_decode_step_host_static(stq_pool* pool, const int32_t* d_slots, i
                                        void* stream);
 
 /* Dequantise slots d_slots[0..B) into d_S_out [B, H, 128, 128] float32:
- * S_ij = (Q_ij * r_i) * c_j, pivot rows float32(h_ij). */
+ * S_ij = (Q_ij * r_i) * c_j, pivot rows float32(h_ij) -- the restored state
+ * X_ij = r_i c_j z_ij of bloombook section 4, without the decay of a step. Errors as
+ * stq_decode_step; the first call on a device raises the kernel's shared-memory limit
+ * (make it outside stream capture). */
 stq_status stq_dequantize(stq_pool* pool, const int32_t* d_slots, int B, float* d_S_out,
                           void* stream);
 
@@ -216,6 +275,23 @@ stq_status stq_fp32_decode_step(int kind, int B, int H, int d, float* d_S,
  * aligned; n_states >= 0. Enqueued on `stream`. */
 stq_status stq_row_sq_error(const float* d_S, const float* d_S_hat, int n_states, float* d_err,
                             int accumulate, void* stream);
+
+/* In-head distortion of every row at candidate widths, for the allocation of per-row
+ * widths (KDA): the rows of a head share the column scales c_j, so a row's width only
+ * sets how far its codes reach. For b < B, head h, row i and candidate k, with
+ * S = d_S[b] ([H, 128, 128] float32) and c the column scales stored in slot
+ * d_slots[b] (fill the slot with stq_quantize_init of the same states first):
+ *   r_i = the refit's row scale of S's row i (computed for every row, pivot rows too;
+ *         rounded to binary16 in a compact pool, as the refit stores it),
+ *   Q_ij = clamp(rint((S_ij * fl(1/r_i)) * fl(1/c_j)), +-(2^(b_k-1) - 1)),
+ *   d_err[((b H + h) 128 + i) n_cand + k] = tree sum_j (S_ij - (Q_ij r_i) c_j)^2
+ * (the tree of stq_row_sq_error). h_cand_bits: 1 to 4 widths from {2,4,6,8} (host).
+ * At a row's own width this is the row's error in the quantised slot. Device pointers
+ * 16-byte aligned; enqueued on `stream`; a slot outside the pool is flagged as in
+ * stq_decode_step. (bloombook section 4, budgeted allocation; singularity-lens
+ * calibration paragraph: per-row squared error for KDA units.) */
+stq_status stq_row_error_at_widths(stq_pool* pool, const int32_t* d_slots, int B, const float* d_S,
+                                   const int* h_cand_bits, int n_cand, float* d_err, void* stream);
 
 /* Lifetime weights L_u = sum_{j=0}^{horizon-1} exp(2 j ell_u) of n units, ell_u the
  * unit's mean log-retention (<= 0), summed term by term in double. Host arrays. */

@@ -63,6 +63,49 @@ def allocate(kind, omega, states, ell_units, budget, pivot_frac=0.02, horizon=10
     return bits, {"lifetime": life, "distortion": dist, "candidates": cand, "n_pivots": n_piv}
 
 
+def in_head_distortions(kind, omega, states, unit_bits, cand_bits, stream=None):
+    """D_u(b) of every KDA row measured inside the heads of a pool of widths unit_bits:
+    the calibration states are quantised into that pool, and each row's error at every
+    candidate width is taken with the column scales its head got
+    (stq_row_error_at_widths). Returns [H*128, n_cand] float64."""
+    import torch
+    N, H = states.shape[0], states.shape[1]
+    om = np.ascontiguousarray(omega, dtype=np.float32)
+    slots = torch.arange(N, dtype=torch.int32, device=states.device)
+    pool = stq.Pool(kind, N, unit_bits, om, device=states.device)
+    pool.quantize_init(slots, states, stream)
+    err = torch.empty((N, H, D, len(cand_bits)), dtype=torch.float32, device=states.device)
+    pool.row_error_at_widths(slots, states, cand_bits, err, stream)
+    pool.check(stream)
+    e = err.cpu().numpy()
+    pool.close()
+    return np.stack([stq.unit_distortion(kind, np.ascontiguousarray(e[..., k]), om)
+                     for k in range(len(cand_bits))], axis=1)
+
+
+def allocate_in_head(kind, omega, states, ell_units, budget, pivot_frac=0.02, horizon=1024, rounds=3,
+                     cand_bits=None):
+    """allocate(), then for per-row widths (KDA) up to `rounds` re-allocations on the
+    rows' in-head distortions under the previous allocation (a row's width sets only the
+    reach of its codes when its head shares column scales), stopping when no width
+    changes. GDN heads have one width each, so the uniform-width distortions are already
+    in-head ones and the first allocation stands. Returns (unit_bits, details)."""
+    bits, info = allocate(kind, omega, states, ell_units, budget, pivot_frac, horizon, cand_bits)
+    info["rounds"] = 0
+    if kind == "gdn":
+        return bits, info
+    cand = info["candidates"]
+    for k in range(rounds):
+        dist = in_head_distortions(kind, omega, states, bits, cand)
+        new = stq.allocate_bits(info["lifetime"], dist, cand, budget, info["n_pivots"])
+        info["rounds"] = k + 1
+        info["distortion"] = dist
+        if np.array_equal(new, bits):
+            break
+        bits = new
+    return bits, info
+
+
 def calibration_states(w, n_seq, steps, device="cuda"):
     """FP32 states after `steps` synthetic calibration steps from zero (FP32 step kernel)."""
     import torch
@@ -91,16 +134,20 @@ def main():
     ap.add_argument("--calib-steps", type=int, default=256)
     ap.add_argument("--eval-steps", type=int, default=1024)
     ap.add_argument("--eval-sequences", type=int, default=4)
+    ap.add_argument("--in-head-rounds", type=int, default=3,
+                    help="re-allocations of per-row (KDA) widths on in-head distortions (0: none)")
     a = ap.parse_args()
     build.build()
     w = W.WORKLOADS[a.workload]
     om = W.omega(w)
     S = calibration_states(w, a.sequences, a.calib_steps)
-    bits, info = allocate(w.kind, om, S, W.calibration_log_retention(w), a.budget)
+    bits, info = allocate_in_head(w.kind, om, S, W.calibration_log_retention(w), a.budget,
+                                  rounds=a.in_head_rounds)
     del S
     hist = {str(b): int((bits == b).sum()) for b in sorted(set(bits.tolist()))}
     res = {"workload": w.name, "budget": a.budget, "calibration": f"{a.sequences} sequences x {a.calib_steps} steps",
            "evaluation": f"{a.eval_sequences} other sequences x {a.eval_steps} steps",
+           "in_head_rounds": info["rounds"],
            "widths": hist, "mean_bits_non_pivot": float(bits[bits != 16].mean()),
            "mean_bits_with_pivots": float(bits.mean())}
     uniform = np.full_like(bits, a.budget)

@@ -126,6 +126,11 @@ stq_status build_layout(const stq_pool_desc* desc, HostLayout& L) {
     const int hb = int(in_head + piv_in_head * D * 2);
     if (hb > L.max_head_bytes) L.max_head_bytes = hb;
   }
+  if (off > 0xFFFFFFFFull)
+    return fail(STQ_ERR_INVALID_ARG, "packed codes of one slot exceed 4 GiB (%llu bytes)",
+                static_cast<unsigned long long>(off));
+  if (piv >= (1 << 24))
+    return fail(STQ_ERR_INVALID_ARG, "too many FP16 pivot rows per slot: %d (limit %d)", piv, (1 << 24) - 1);
   L.slot_code_bytes = off;
   L.n_pivot_rows = piv;
   return STQ_OK;
@@ -144,6 +149,7 @@ MetaLayout meta_layout(int H) {
   m.head_piv_count = o;  o = up16(o + size_t(H) * 4);
   m.head_bits = o;       o = up16(o + size_t(H) * 4);
   m.warp_code_off = o;   o = up16(o + size_t(H) * 8 * 4);
+  m.warp_rec = o;        o = up16(o + size_t(H) * 8 * 16);
   m.row_info = o;        o = up16(o + size_t(H) * D * 4);
   m.g = o;               o = up16(o + size_t(H) * D * 4);
   m.omega = o;           o = up16(o + size_t(H) * D * 4);
@@ -223,6 +229,19 @@ stq_status stq_pool_create(const stq_pool_desc* desc, void* d_codes, void* d_sca
   put(m.head_piv_count, L.head_piv_count.data(), L.H * 4);
   put(m.head_bits, L.head_bits.data(), L.H * 4);
   put(m.warp_code_off, L.warp_code_off.data(), L.warp_code_off.size() * 4);
+  {
+    std::vector<uint32_t> rec(size_t(L.H) * 8 * 4);
+    for (int h = 0; h < L.H; ++h)
+      for (int w = 0; w < 8; ++w) {
+        const size_t hw = size_t(h) * 8 + w;
+        const uint32_t end = (w + 1 < 8) ? L.warp_code_off[hw + 1] : L.head_code_bytes[h];
+        rec[4 * hw + 0] = L.head_code_off[h];
+        rec[4 * hw + 1] = L.warp_code_off[hw];
+        rec[4 * hw + 2] = end - L.warp_code_off[hw];
+        rec[4 * hw + 3] = L.head_bits[h] | (L.head_piv_first[h] << 8);
+      }
+    put(m.warp_rec, rec.data(), rec.size() * 4);
+  }
   put(m.row_info, L.row_info.data(), L.row_info.size() * 4);
   put(m.g, L.g.data(), L.g.size() * 4);
   put(m.omega, L.omega.data(), L.omega.size() * 4);
@@ -246,6 +265,7 @@ stq_status stq_pool_create(const stq_pool_desc* desc, void* d_codes, void* d_sca
   dv.head_piv_count = reinterpret_cast<const uint32_t*>(mb + m.head_piv_count);
   dv.head_bits = reinterpret_cast<const uint32_t*>(mb + m.head_bits);
   dv.warp_code_off = reinterpret_cast<const uint32_t*>(mb + m.warp_code_off);
+  dv.warp_rec = reinterpret_cast<const uint4*>(mb + m.warp_rec);
   dv.row_info = reinterpret_cast<const uint32_t*>(mb + m.row_info);
   dv.g = reinterpret_cast<const float*>(mb + m.g);
   dv.omega = reinterpret_cast<const float*>(mb + m.omega);
@@ -261,13 +281,42 @@ stq_status stq_pool_create(const stq_pool_desc* desc, void* d_codes, void* d_sca
 
 void stq_pool_destroy(stq_pool* pool) { delete pool; }
 
-static stq_status check_batch(const stq_pool* pool, const int32_t* d_slots, int B) {
+}  // extern "C"
+
+namespace stq {
+
+int check_batch(const ::stq_pool* pool, const int32_t* d_slots, int B) {
   if (pool == nullptr) return fail(STQ_ERR_INVALID_ARG, "pool is NULL");
   if (B < 0) return fail(STQ_ERR_INVALID_ARG, "B must be >= 0, got %d", B);
   if (int64_t(B) * pool->L.H > (int64_t(1) << 31) - 1)
     return fail(STQ_ERR_INVALID_ARG, "B * H too large: %d * %d", B, pool->L.H);
   if (B > 0 && d_slots == nullptr) return fail(STQ_ERR_INVALID_ARG, "d_slots is NULL");
   return STQ_OK;
+}
+
+StagingLayout staging_layout(const PoolDev& P, int B) {
+  StagingLayout s;
+  const size_t BH = size_t(B) * size_t(P.H);
+  s.n_vec = BH * STQ_D;
+  s.n_gate = (P.kind == STQ_GDN) ? BH : BH * STQ_D;
+  s.n_beta = BH;
+  size_t o = 0;
+  s.q = o;    o = up16(o + s.n_vec * 4);
+  s.k = o;    o = up16(o + s.n_vec * 4);
+  s.v = o;    o = up16(o + s.n_vec * 4);
+  s.gate = o; o = up16(o + s.n_gate * 4);
+  s.beta = o; o = up16(o + s.n_beta * 4);
+  s.out = o;  o = up16(o + s.n_vec * 4);
+  s.total = o;
+  return s;
+}
+
+}  // namespace stq
+
+extern "C" {
+
+static stq_status check_batch(const stq_pool* pool, const int32_t* d_slots, int B) {
+  return static_cast<stq_status>(stq::check_batch(pool, d_slots, B));
 }
 
 static stq_status check_ptrs(std::initializer_list<const void*> ps) {
@@ -304,32 +353,9 @@ stq_status stq_decode_step(stq_pool* pool, const int32_t* d_slots, int B, const 
   return ok();
 }
 
-namespace {
-struct StagingLayout {
-  size_t q, k, v, gate, beta, out, total;
-  size_t n_vec, n_gate, n_beta;
-};
-StagingLayout staging_layout(const stq_pool* pool, int B) {
-  StagingLayout s;
-  const size_t BH = size_t(B) * size_t(pool->L.H);
-  s.n_vec = BH * STQ_D;
-  s.n_gate = (pool->L.kind == STQ_GDN) ? BH : BH * STQ_D;
-  s.n_beta = BH;
-  size_t o = 0;
-  s.q = o;    o = up16(o + s.n_vec * 4);
-  s.k = o;    o = up16(o + s.n_vec * 4);
-  s.v = o;    o = up16(o + s.n_vec * 4);
-  s.gate = o; o = up16(o + s.n_gate * 4);
-  s.beta = o; o = up16(o + s.n_beta * 4);
-  s.out = o;  o = up16(o + s.n_vec * 4);
-  s.total = o;
-  return s;
-}
-}  // namespace
-
 size_t stq_decode_step_host_staging_bytes(const stq_pool* pool, int B) {
   if (pool == nullptr || B < 0) return 0;
-  return staging_layout(pool, B).total;
+  return stq::staging_layout(pool->dev, B).total;
 }
 
 stq_status stq_decode_step_host(stq_pool* pool, const int32_t* d_slots, int B, const float* h_q,
@@ -343,7 +369,7 @@ stq_status stq_decode_step_host(stq_pool* pool, const int32_t* d_slots, int B, c
     return fail(STQ_ERR_INVALID_ARG, "a host pointer is NULL");
   st = check_ptrs({d_staging});
   if (st != STQ_OK) return st;
-  const StagingLayout L = staging_layout(pool, B);
+  const stq::StagingLayout L = stq::staging_layout(pool->dev, B);
   if (staging_bytes < L.total)
     return fail(STQ_ERR_INVALID_ARG, "staging_bytes %zu < required %zu", staging_bytes, L.total);
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -14,8 +14,9 @@ namespace {
 struct AbsmaxStore {
   template <int BITS, class Sc>
   static __device__ __forceinline__ void store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], const Sc& sc,
-                                               uint8_t* codes_global, int warp_code_start, float* o_global) {
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+                                               uint8_t* codes_global, int warp_code_start, float* o_global,
+                                               uint8_t* /*stage*/) {
+    const int w = group_tid() >> 5, lane = group_tid() & 31;
     const int r0 = w * RPW;
 
     // --- row maxima of |S| (exact in any order): 4 columns per lane, then a
@@ -109,7 +110,7 @@ struct AbsmaxStore {
 
     // --- readout from the per-warp partials the caller left in red[1][0] ------------
     if (o_global != nullptr) {
-      __syncthreads();
+      group_sync();
       if (w == 0) {
         f2 lo, hi;
         warp_tree(cs.red[1][0], lane, lo, hi);
@@ -125,23 +126,23 @@ cudaError_t launch_decode_absmax(const PoolDev& P, const int32_t* slots, int B, 
                                  const float* k, const float* v, const float* gate,
                                  const float* beta, float* out, cudaStream_t s) {
   if (B == 0) return cudaSuccess;
-  const unsigned grid = unsigned(B) * unsigned(P.H);
+  const unsigned n = unsigned(B) * unsigned(P.H);
+  constexpr int SM = 2 * sizeof(DecodeSmem);
   if (P.scale16) {
-    if (P.any_mixed) decode_kernel<AbsmaxStore, true, true><<<grid, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
-    else decode_kernel<AbsmaxStore, false, true><<<grid, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
-  } else {
-    if (P.any_mixed) decode_kernel<AbsmaxStore, true, false><<<grid, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
-    else decode_kernel<AbsmaxStore, false, false><<<grid, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+    if (P.any_mixed) return launch_persistent<decode_kernel<AbsmaxStore, true, true>>(n, SM, s, P, slots, B, q, k, v, gate, beta, out);
+    return launch_persistent<decode_kernel<AbsmaxStore, false, true>>(n, SM, s, P, slots, B, q, k, v, gate, beta, out);
   }
-  return cudaGetLastError();
+  if (P.any_mixed) return launch_persistent<decode_kernel<AbsmaxStore, true, false>>(n, SM, s, P, slots, B, q, k, v, gate, beta, out);
+  return launch_persistent<decode_kernel<AbsmaxStore, false, false>>(n, SM, s, P, slots, B, q, k, v, gate, beta, out);
 }
 
 cudaError_t launch_quantize_absmax(const PoolDev& P, const int32_t* slots, int B, const float* S,
                                    cudaStream_t s) {
   if (B == 0) return cudaSuccess;
-  if (P.scale16) quantize_kernel<AbsmaxStore, true><<<B * P.H, NT, 0, s>>>(P, slots, B, S);
-  else quantize_kernel<AbsmaxStore, false><<<B * P.H, NT, 0, s>>>(P, slots, B, S);
-  return cudaGetLastError();
+  const unsigned n = unsigned(B) * unsigned(P.H);
+  constexpr int SM = sizeof(CtaSmem);
+  if (P.scale16) return launch_items<quantize_kernel<AbsmaxStore, true>>(n, SM, s, P, slots, B, S);
+  return launch_items<quantize_kernel<AbsmaxStore, false>>(n, SM, s, P, slots, B, S);
 }
 
 }  // namespace stq

@@ -8,6 +8,8 @@
 #include <limits>
 #include <vector>
 
+#include <cuda_fp16.h>
+
 #include "stq.h"
 #include "stq_internal.h"
 
@@ -33,6 +35,73 @@ row_sq_error_kernel(const float4* __restrict__ S, const float4* __restrict__ S_h
 #pragma unroll
   for (int m = 1; m < 32; m <<= 1) e = __fadd_rn(e, __shfl_xor_sync(0xffffffffu, e, m));
   if (lane == 0) err[row] = accumulate ? __fadd_rn(err[row], e) : e;
+}
+
+// In-head distortion of a row at candidate widths: one warp per row of one (state, head)
+// of a quantised pool. The row keeps the refit's row scale r_i (computed here from S for
+// every row, pivot rows included) and the head's stored column scales c_j; only the
+// reach of its codes changes with the width: Q = clamp(rint((S r^-1) c^-1), +-qmax_b)
+// on the exact product, S_hat = (Q r) c, and the error is the tree sum of the squared
+// differences (the row_sq_error_kernel's tree).
+struct CandWidths {
+  int n;
+  float qmax[4];
+};
+
+template <bool H16>
+__global__ void __launch_bounds__(256)
+row_error_at_widths_kernel(stq::PoolDev P, const int32_t* __restrict__ slots, int B,
+                           const float4* __restrict__ S, CandWidths cw, float* __restrict__ err) {
+  constexpr float kMagic = 12582912.0f;            // 1.5 * 2^23
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const long long n_rows = (long long)B * P.H * kD;
+  if (row >= n_rows) return;
+  const long long hs = row / kD;                   // (state, head)
+  const int i = int(row - hs * kD);
+  const int n = int(hs / P.H), h = int(hs - (long long)n * P.H);
+  const int slot = slots[n];
+  if (slot < 0 || slot >= P.n_slots) {
+    if (lane == 0 && i == 0) atomicOr(P.err, stq::ERR_SLOT_RANGE);
+    return;
+  }
+  const size_t cbase = (size_t(slot) * P.H + h) * 2 * kD + kD + 4 * lane;
+  float c[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    if constexpr (H16) c[e] = __half2float(static_cast<const __half*>(P.scales)[cbase + e]);
+    else c[e] = static_cast<const float*>(P.scales)[cbase + e];
+  }
+  const float4 x = S[row * 32 + lane];
+  const float sv[4] = {x.x, x.y, x.z, x.w};
+  float a = __fadd_rn(__fadd_rn(fabsf(sv[0]), fabsf(sv[1])), __fadd_rn(fabsf(sv[2]), fabsf(sv[3])));
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, m));
+  float r = __fmul_rn(__fmul_rn(a, 0.0078125f), P.g[h * kD + i]);
+  if constexpr (H16) r = __half2float(__float2half_rn(r));   // a compact pool stores r as binary16
+  const float tiny = 1.17549435e-38f;              // scales below 2^-126 count as zero
+  const float ir = r >= tiny ? __frcp_rn(r) : 0.0f;
+  float y[4], ic[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    y[e] = __fmul_rn(sv[e], ir);
+    ic[e] = c[e] >= tiny ? __frcp_rn(c[e]) : 0.0f;
+  }
+  for (int ci = 0; ci < cw.n; ++ci) {
+    const float lo = kMagic - cw.qmax[ci], hi = kMagic + cw.qmax[ci];
+    float d2[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float t = fminf(fmaxf(__fmaf_rn(y[e], ic[e], kMagic), lo), hi);
+      const float q = __fadd_rn(t, -kMagic);
+      const float d = __fsub_rn(sv[e], __fmul_rn(__fmul_rn(q, r), c[e]));
+      d2[e] = __fmul_rn(d, d);
+    }
+    float ev = __fadd_rn(__fadd_rn(d2[0], d2[1]), __fadd_rn(d2[2], d2[3]));
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) ev = __fadd_rn(ev, __shfl_xor_sync(0xffffffffu, ev, m));
+    if (lane == 0) err[row * cw.n + ci] = ev;
+  }
 }
 
 stq_status fail(stq_status st, const char* msg) {
@@ -66,6 +135,41 @@ extern "C" stq_status stq_row_sq_error(const float* d_S, const float* d_S_hat, i
   if (e != cudaSuccess) {
     char buf[256];
     snprintf(buf, sizeof(buf), "stq_row_sq_error launch: %s", cudaGetErrorString(e));
+    return fail(STQ_ERR_CUDA, buf);
+  }
+  return ok();
+}
+
+extern "C" stq_status stq_row_error_at_widths(stq_pool* pool, const int32_t* d_slots, int B,
+                                              const float* d_S, const int* h_cand_bits, int n_cand,
+                                              float* d_err, void* stream) {
+  const int st = stq::check_batch(pool, d_slots, B);
+  if (st != STQ_OK) return static_cast<stq_status>(st);
+  if (h_cand_bits == nullptr || n_cand < 1 || n_cand > 4)
+    return fail(STQ_ERR_INVALID_ARG, "need 1 to 4 candidate widths");
+  CandWidths cw;
+  cw.n = n_cand;
+  for (int k = 0; k < n_cand; ++k) {
+    const int b = h_cand_bits[k];
+    if (b != 2 && b != 4 && b != 6 && b != 8) return fail(STQ_ERR_INVALID_ARG, "candidate width not in {2,4,6,8}");
+    cw.qmax[k] = float((1 << (b - 1)) - 1);
+  }
+  for (int k = n_cand; k < 4; ++k) cw.qmax[k] = 0.0f;
+  if (B == 0) return ok();
+  if (!d_S || !d_err) return fail(STQ_ERR_INVALID_ARG, "a device pointer is NULL");
+  if (!aligned16(d_S) || !aligned16(d_err)) return fail(STQ_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+  const stq::PoolDev* P = stq::pool_dev(pool);
+  const long long n_rows = (long long)B * P->H * kD;
+  const long long blocks = (n_rows + 7) / 8;
+  if (blocks > 0x7fffffffLL) return fail(STQ_ERR_INVALID_ARG, "B too large");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const float4* S4 = reinterpret_cast<const float4*>(d_S);
+  if (P->scale16) row_error_at_widths_kernel<true><<<unsigned(blocks), 256, 0, s>>>(*P, d_slots, B, S4, cw, d_err);
+  else row_error_at_widths_kernel<false><<<unsigned(blocks), 256, 0, s>>>(*P, d_slots, B, S4, cw, d_err);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    char buf[256];
+    snprintf(buf, sizeof(buf), "stq_row_error_at_widths launch: %s", cudaGetErrorString(e));
     return fail(STQ_ERR_CUDA, buf);
   }
   return ok();

@@ -4,10 +4,11 @@
 // policy `Store` with
 //   template <int BITS> static __device__ void store(CtaSmem&, WarpRows&,
 //       f2 (&s)[RPW][2], const Scales<H16>& sc, uint8_t* codes, int warp_code_start,
-//       float* o);
+//       float* o, uint8_t* stage);
 // which quantises the warp's 16 rows s (float32 state), writes codes and scales (r at
-// Scales index i, c at D + j) and, when
-// o is not null, the readout whose per-warp partials are in red[1][0].
+// Scales index i, c at D + j) and, when o is not null, the readout whose per-warp
+// partials are in red[1][0]. `stage` is the warp's consumed code staging area (its
+// rows' bytes), free for the store to use.
 // The float32 evaluation order is described at the top of stq_kernels.cu.
 #pragma once
 
@@ -313,8 +314,32 @@ struct __align__(16) WarpRows {
   float dec[RPW];                  // row retention
   float g[RPW], om[RPW];           // row gain and omega
   float qm[RPW], iq[RPW], mb[RPW];   // per-row width constants (mixed heads)
+  uint4 rk[RPW];                   // mixed heads, unpack of row i (width b, pivot rows 0):
+                                   //   {M = 2^b - 1, M << b, exponent bits of a code at
+                                   //   bit b, 4b | 2b << 8}
+  f2 roff[RPW];                    // -(2^23 + 2^(b-1)), -(2^(23-b) + 2^(b-1))
+  f2 clampb[RPW];                  // least-squares clamp: 1.5*2^23 -+ qmax
   uint32_t info[RPW];              // bits | offset << 8
-  uint8_t codes[RPW * D];          // this warp's rows of packed codes
+  uint8_t codes[2][RPW * D];       // this warp's rows of packed codes: the item being
+                                   // decoded and the next one (arriving asynchronously)
+  uint32_t tail[4];                // the last row may read one word past its codes
+};
+
+// The inputs of one (request, head) item that a warp needs, as they arrive from global
+// memory by asynchronous copies issued while the warp works on the item before it.
+struct __align__(16) WarpRaw {
+  float k[RPW], q[RPW];            // k_i, q_i of rows 16w..16w+15
+  float gate[RPW];                 // per-row retention (KDA)
+  float v[RPW];                    // v_j of the columns 16w..16w+15 that lanes 0..15 own
+  uint32_t info[RPW];              // row_info of the rows
+  float g[RPW], om[RPW];           // row gain and omega of the rows
+  uint32_t r[RPW];                 // r_i of the rows (float32; binary16 in the first 32 bytes)
+  uint32_t c[D];                   // c_j (float32; binary16 in the first 256 bytes)
+  float beta, gate_s;              // beta and the GDN retention of the item
+  int32_t next_slot;               // slot of the warp's next item
+  int32_t slot;                    // slot of this item
+  uint4 next_rec;                  // warp_rec of the next item
+  uint4 rec;                       // warp_rec of this item
 };
 
 struct __align__(16) CtaSmem {
@@ -322,13 +347,37 @@ struct __align__(16) CtaSmem {
   float col_ic[D];                 // 1/c_j of the current column scale, from its owner
   float col_delta[D];              // delta_j = beta (v_j - u_j), from its owner
   WarpRows wr[NW];
-  uint32_t tail[4];                // the last warp's last row may read one word past its codes
+};
+
+struct __align__(16) DecodeSmem {
+  CtaSmem cs;
+  WarpRaw raw[NW];
+  const uint8_t* ptab[8];          // base pointers of the prefetched row arrays
 };
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
                "l"(src)
                : "memory");
+}
+
+// The 256 threads (8 warps) that work on one (request, head) item meet at a named
+// barrier of their own: 1 for threads 0..255, 2 for 256..511 (a decode CTA runs two such
+// groups on separate items; a 256-thread CTA is one group).
+__device__ __forceinline__ int group_id() { return int(threadIdx.x) >> 8; }
+__device__ __forceinline__ int group_tid() { return int(threadIdx.x) & (NT - 1); }
+__device__ __forceinline__ void group_sync() {
+  asm volatile("bar.sync %0, 256;" ::"r"(1 + group_id()) : "memory");
+}
+__device__ __forceinline__ int group_sync_or(int pred) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\tbar.red.or.pred q, %2, 256, p;\n\t"
+      "selp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred), "r"(1 + group_id())
+      : "memory");
+  return r;
 }
 
 // Per-row constants of a width (2/4/6/8, 16 = pivot).
@@ -343,6 +392,24 @@ __device__ __forceinline__ void width_consts(int bits, float& qm, float& iq, flo
   }
 }
 
+// Lane l < 16 of a warp: every per-row constant of its row (width `bits`) that the
+// mixed-width paths read.
+__device__ __forceinline__ void mixed_row_consts(WarpRows& wr, int l, int bits) {
+  float qm, iq, mb;
+  width_consts(bits, qm, iq, mb);
+  wr.qm[l] = qm; wr.iq[l] = iq; wr.mb[l] = mb;
+  wr.clampb[l] = make_float2(MAGIC - qm, MAGIC + qm);
+  if (bits == PIVOT) {
+    wr.rk[l] = make_uint4(0u, 0u, 0u, 0u);
+    wr.roff[l] = make_float2(0.0f, 0.0f);
+  } else {
+    const uint32_t M = (1u << bits) - 1u;
+    const float bias = float(1 << (bits - 1));
+    wr.rk[l] = make_uint4(M, M << bits, uint32_t(150 - bits) << 23, uint32_t(4 * bits) | (uint32_t(2 * bits) << 8));
+    wr.roff[l] = make_float2(-(8388608.0f + bias), -(float(1u << (23 - bits)) + bias));
+  }
+}
+
 // Lanes 0..15 of warp w: the per-row data of rows 16w..16w+15 of head h.
 template <bool H16>
 __device__ __forceinline__ void load_warp_rows(const PoolDev& P, int h, WarpRows& wr, int lane, int r0,
@@ -354,9 +421,7 @@ __device__ __forceinline__ void load_warp_rows(const PoolDev& P, int h, WarpRows
     wr.info[lane] = info;
     wr.g[lane] = P.g[h * D + i];
     wr.om[lane] = P.omega[h * D + i];
-    float qm, iq, mb;
-    width_consts(row_bits(info), qm, iq, mb);
-    wr.qm[lane] = qm; wr.iq[lane] = iq; wr.mb[lane] = mb;
+    mixed_row_consts(wr, lane, row_bits(info));
     if (k_vec != nullptr) {
       const float dec = gate_rows != nullptr ? gate_rows[i] : gate_s;
       const float kv = k_vec[i], qv = q_vec[i];
@@ -376,22 +441,22 @@ __device__ __forceinline__ void load_warp_rows(const PoolDev& P, int h, WarpRows
 // u_j = (k^T S')_j in the tree ((w0+w1)+(w2+w3))+((w4+w5)+(w6+w7)) and publishes
 // delta_j = beta (v_j - u_j) through shared memory.
 __device__ __forceinline__ void publish_delta(CtaSmem& cs, int lane, int w, float v_own, float beta_s) {
-  if (lane < 16) {
-    const int j = 16 * w + lane;
-    const float* part = reinterpret_cast<const float*>(cs.red[0][0][0]);
-    float x[NW];
+  // lanes 16..31 repeat the work of lanes 0..15 (no divergent branch); only 0..15 store
+  const int j = 16 * w + (lane & 15);
+  const float* part = reinterpret_cast<const float*>(cs.red[0][0][0]);
+  float x[NW];
 #pragma unroll
-    for (int ww = 0; ww < NW; ++ww) x[ww] = part[ww * D + j];
-    const float u = fadd(fadd(fadd(x[0], x[1]), fadd(x[2], x[3])), fadd(fadd(x[4], x[5]), fadd(x[6], x[7])));
-    cs.col_delta[j] = fmul(beta_s, fadd(v_own, -u));
-  }
+  for (int ww = 0; ww < NW; ++ww) x[ww] = part[ww * D + j];
+  const float u = fadd(fadd(fadd(x[0], x[1]), fadd(x[2], x[3])), fadd(fadd(x[4], x[5]), fadd(x[6], x[7])));
+  const float dl = fmul(beta_s, fadd(v_own, -u));
+  if (lane < 16) cs.col_delta[j] = dl;
 }
 
 template <int BITS, class Store, bool H16>
 __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const HeadRef<H16>& hr, int warp_code_start,
-                                            const f2 (&cin)[2], float v_own, float beta_s,
+                                            uint8_t* wcodes, const f2 (&cin)[2], float v_own, float beta_s,
                                             float* o_out) {
-  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int tid = group_tid(), w = tid >> 5, lane = tid & 31;
   f2 s[RPW][2];
 #ifdef STQ_CHECKS
   bool zero_code = false;   // a stored code 0: never written by the quantiser
@@ -402,43 +467,36 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
   for (int rr = 0; rr < RPW; ++rr) {
     if constexpr (BITS == MIXED) {
       const uint32_t info = wr.info[rr];
-      const int bits = row_bits(info);
-      const uint8_t* row = wr.codes + (row_off(info) - warp_code_start);
-      const float rd = wr.rdd[rr].x;
-      switch (bits) {
-        case 2: case 4: case 6: case 8: {
-          // any width b: the lane's 4b bits start at bit 4 b l of the row; the word after
-          // them is inside the staging area (the next row, the next warp's rows or `tail`)
-          const uint32_t* wp = reinterpret_cast<const uint32_t*>(row);
-          const int bitpos = 4 * bits * lane;
-          const uint32_t f = __funnelshift_r(wp[bitpos >> 5], wp[(bitpos >> 5) + 1], bitpos & 31);
-          const uint32_t M = (1u << bits) - 1u;
+      if (row_bits(info) != PIVOT) {
+        // any width b: the lane's 4b bits start at bit 4 b l of the row (the word after them
+        // is inside the staging area: the next row, the other buffer or `tail`); codes 0
+        // and 2 sit at bit 0 of f and fh, codes 1 and 3 at bit b, each unpacked in place
+        // into a float's mantissa (2^23 + u, 2^(23-b) + u)
+        const uint4 K = wr.rk[rr];
+        const f2 off = wr.roff[rr];
+        const uint32_t* wp = reinterpret_cast<const uint32_t*>(wcodes + (row_off(info) - warp_code_start));
+        const int bitpos = int(K.w & 0xFFu) * lane;
+        const uint32_t f = __funnelshift_r(wp[bitpos >> 5], wp[(bitpos >> 5) + 1], bitpos & 31);
+        const uint32_t fh = f >> (K.w >> 8);
 #ifdef STQ_CHECKS
-          zero_code |= (f & M) == 0 || ((f >> bits) & M) == 0 || ((f >> (2 * bits)) & M) == 0 ||
-                       ((f >> (3 * bits)) & M) == 0;
+        zero_code |= (f & K.x) == 0 || (f & K.y) == 0 || (fh & K.x) == 0 || (fh & K.y) == 0;
 #endif
-          // 2^23 + bias as a float: the bias sits in the mantissa
-          const f2 ntb = dup(-__uint_as_float(FLOAT_2P23 | (1u << (bits - 1))));
-          const f2 q01 = add2(make_float2(__uint_as_float((f & M) | FLOAT_2P23),
-                                          __uint_as_float(((f >> bits) & M) | FLOAT_2P23)), ntb);
-          const f2 q23 = add2(make_float2(__uint_as_float(((f >> (2 * bits)) & M) | FLOAT_2P23),
-                                          __uint_as_float(((f >> (3 * bits)) & M) | FLOAT_2P23)), ntb);
-          s[rr][0] = mul2(mul2(q01, dup(rd)), cin[0]);
-          s[rr][1] = mul2(mul2(q23, dup(rd)), cin[1]);
-          break;
-        }
-        default: {
-          const uint2 hv = *reinterpret_cast<const uint2*>(hr.pivots + row_off(info) * D + 4 * lane);
-          f2 x, y;
-          half4_floats(hv, x, y);
-          const f2 dd = dup(wr.dec[rr]);
-          s[rr][0] = mul2(dd, x);
-          s[rr][1] = mul2(dd, y);
-        }
+        const f2 q01 = add2(make_float2(__uint_as_float((f & K.x) | FLOAT_2P23), __uint_as_float((f & K.y) | K.z)), off);
+        const f2 q23 = add2(make_float2(__uint_as_float((fh & K.x) | FLOAT_2P23), __uint_as_float((fh & K.y) | K.z)), off);
+        const f2 rd = dup(wr.rdd[rr].x);
+        s[rr][0] = mul2(mul2(q01, rd), cin[0]);
+        s[rr][1] = mul2(mul2(q23, rd), cin[1]);
+      } else {
+        const uint2 hv = *reinterpret_cast<const uint2*>(hr.pivots + row_off(info) * D + 4 * lane);
+        f2 x, y;
+        half4_floats(hv, x, y);
+        const f2 dd = dup(wr.dec[rr]);
+        s[rr][0] = mul2(dd, x);
+        s[rr][1] = mul2(dd, y);
       }
     } else {
       uint32_t cd[4];
-      load_codes<BITS>(wr.codes + rr * (D * BITS / 8), lane, cd);
+      load_codes<BITS>(wcodes + rr * (D * BITS / 8), lane, cd);
 #ifdef STQ_CHECKS
       // the mantissa of an unpacked code holds u << pos: zero exactly when u = 0
       zero_code |= ((cd[0] & 0x7FFFFFu) == 0) || ((cd[1] & 0x7FFFFFu) == 0) ||
@@ -463,34 +521,37 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
     });
     put_partial(cs.red[0][0], w, lane, u.x[0], u.x[1]);
   }
-  __syncthreads();
+  group_sync();
 
   // ---- delta_j = beta (v_j - u_j) by its column owner; S = S' + k delta^T; readout ----
   f2 delta[2];
   publish_delta(cs, lane, w, v_own, beta_s);
-  __syncthreads();
+  group_sync();
   {
     const float4 d4 = *reinterpret_cast<const float4*>(&cs.col_delta[4 * lane]);
     delta[0] = make_float2(d4.x, d4.y);
     delta[1] = make_float2(d4.z, d4.w);
   }
   {
-    V2<2> o = tree<0, RPW / 2, 2>([&](int m) {
+    // S = S' + k delta^T and the readout partials sum_i q_i S_ij of this warp's rows (the
+    // readout is compared within a tolerance, not bit for bit: plain running sums, even
+    // and odd rows apart)
+    f2 o[2][2] = {{make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)}, {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)}};
+#pragma unroll
+    for (int m = 0; m < RPW / 2; ++m) {
       const float4 k2 = *reinterpret_cast<const float4*>(&wr.kk[2 * m]);
       const float4 q2 = *reinterpret_cast<const float4*>(&wr.qq[2 * m]);
       const f2 kp[2] = {make_float2(k2.x, k2.y), make_float2(k2.z, k2.w)};
+      const f2 qp[2] = {make_float2(q2.x, q2.y), make_float2(q2.z, q2.w)};
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         s[2 * m + e][0] = fma2(kp[e], delta[0], s[2 * m + e][0]);
         s[2 * m + e][1] = fma2(kp[e], delta[1], s[2 * m + e][1]);
+        o[e][0] = fma2(qp[e], s[2 * m + e][0], o[e][0]);
+        o[e][1] = fma2(qp[e], s[2 * m + e][1], o[e][1]);
       }
-      const f2 qe = make_float2(q2.x, q2.y), qo = make_float2(q2.z, q2.w);
-      V2<2> leaf;
-      leaf.x[0] = fma2(qe, s[2 * m][0], mul2(qo, s[2 * m + 1][0]));
-      leaf.x[1] = fma2(qe, s[2 * m][1], mul2(qo, s[2 * m + 1][1]));
-      return leaf;
-    });
-    put_partial(cs.red[1][0], w, lane, o.x[0], o.x[1]);
+    }
+    put_partial(cs.red[1][0], w, lane, add2(o[0][0], o[1][0]), add2(o[0][1], o[1][1]));
   }
   if constexpr (BITS == MIXED) {
     // pivot rows: store float16(S) now (they take no part in the refit)
@@ -513,14 +574,14 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
     if (lane == 0 && bits) atomicOr(hr.err, bits);
   }
 #endif
-  Store::template store<BITS>(cs, wr, s, hr.sc, hr.codes, warp_code_start, o_out);
+  Store::template store<BITS>(cs, wr, s, hr.sc, hr.codes, warp_code_start, o_out, wcodes);
 }
 
 // A head whose rows are all FP16 pivots: decay, update, readout, store float16; r = c = 0.
 template <bool H16>
 __device__ __forceinline__ void decode_pivot_warp(CtaSmem& cs, WarpRows& wr, const HeadRef<H16>& hr,
                                                   float v_own, float beta_s, float* o_out) {
-  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int tid = group_tid(), w = tid >> 5, lane = tid & 31;
   const int r0 = w * RPW;
   f2 s[RPW][2];
 #pragma unroll
@@ -543,10 +604,10 @@ __device__ __forceinline__ void decode_pivot_warp(CtaSmem& cs, WarpRows& wr, con
     });
     put_partial(cs.red[0][0], w, lane, u.x[0], u.x[1]);
   }
-  __syncthreads();
+  group_sync();
   f2 delta[2];
   publish_delta(cs, lane, w, v_own, beta_s);
-  __syncthreads();
+  group_sync();
   {
     const float4 d4 = *reinterpret_cast<const float4*>(&cs.col_delta[4 * lane]);
     delta[0] = make_float2(d4.x, d4.y);
@@ -571,7 +632,7 @@ __device__ __forceinline__ void decode_pivot_warp(CtaSmem& cs, WarpRows& wr, con
 #pragma unroll
   for (int rr = 0; rr < RPW; ++rr)
     *reinterpret_cast<uint2*>(hr.pivots + (r0 + rr) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
-  __syncthreads();
+  group_sync();
   if (w == 0) {
     f2 lo, hi;
     warp_tree(cs.red[1][0], lane, lo, hi);
@@ -580,55 +641,180 @@ __device__ __forceinline__ void decode_pivot_warp(CtaSmem& cs, WarpRows& wr, con
   if (tid < 2 * D) hr.sc.put(tid, 0.0f);
 }
 
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+
+// Warp w's asynchronous copies of the inputs of item (h, bq): its packed rows into
+// `codes_dst`, its rows' k, q, gate, row data and r, the column scales c and the v_j of
+// its owned columns into `raw`; and, when there is a following item (hn, bn), that
+// item's slot and warp_rec. The slot and warp_rec of (h, bq) itself came from the
+// previous copies and are stored into `raw` as they are. A slot outside [0, n_slots)
+// gets no copies (the item is skipped and flagged when its turn comes).
+// `ptab` holds the eight 64-byte row arrays' base pointers: k, q, gate, v, row_info, g,
+// omega, scales.
+template <bool H16>
+__device__ __forceinline__ void prefetch_item(const PoolDev& P, const int32_t* __restrict__ slots,
+                                              const float* __restrict__ beta, const float* __restrict__ gate,
+                                              const uint8_t* const* ptab, WarpRaw& raw, uint8_t* codes_dst,
+                                              int h, int bq, int slot, uint4 rec, bool has_next, int hn,
+                                              int bn, int w, int lane) {
+  constexpr int ES = H16 ? 2 : 4;   // bytes per stored scale
+  const int r0 = w * RPW;
+  if (lane == 0) {
+    raw.slot = slot;
+    raw.rec = rec;
+  }
+  if (slot >= 0 && slot < P.n_slots) {
+    const uint64_t vi = uint64_t(bq) * P.H + h;
+    const uint64_t soff = (uint64_t(slot) * P.H + h) * (2 * D * ES);
+    const uint8_t* cg = P.codes + uint64_t(slot) * P.slot_code_bytes + rec.x + rec.y;
+#pragma unroll
+    for (int j = 0; j < (RPW * D) / (16 * 32); ++j) {
+      const int o = 16 * lane + 16 * 32 * j;
+      if (o < int(rec.z)) cp_async16(codes_dst + o, cg + o);
+    }
+    // eight 64-byte row arrays, four lanes each; v of the 16 columns the warp owns shares
+    // the rows' offset (r0 = 16 w)
+    const int grp = lane >> 2, part = 16 * (lane & 3);
+    const uint64_t off = grp < 4 ? (vi * D + r0) * 4 : grp < 7 ? (uint64_t(h) * D + r0) * 4 : soff + r0 * ES;
+    const bool valid = (grp != 2 || P.kind != 0) && (grp != 7 || part < RPW * ES);
+    if (valid) cp_async16(reinterpret_cast<uint8_t*>(&raw) + 64 * grp + part, ptab[grp] + off + part);
+    if (16 * lane < D * ES)
+      cp_async16(reinterpret_cast<uint8_t*>(raw.c) + 16 * lane, ptab[7] + soff + D * ES + 16 * lane);
+    if (lane == 4) cp_async4(&raw.beta, beta + vi);
+    if (lane == 5 && P.kind == 0) cp_async4(&raw.gate_s, gate + vi);
+  }
+  if (has_next) {
+    if (lane == 6) cp_async4(&raw.next_slot, slots + bn);
+    if (lane == 7) cp_async16(&raw.next_rec, P.warp_rec + hn * NW + w);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------------
-// stq_decode_step: one CTA per (head, request) item, numbered head-major so that the
-// CTAs resident on an SM at the same time mostly run the same width's code path. Each
-// warp stages its own 16 rows (asynchronous 16-byte copies) and writes its own codes
-// back, so the CTA synchronises only for the five column exchanges.
+// stq_decode_step: persistent CTAs, each taking the (head, request) items
+// blockIdx.x, blockIdx.x + gridDim.x, ... of a head-major numbering (the CTAs resident
+// on an SM at the same time mostly run the same width's code path). Each warp copies
+// the inputs of its next item into shared memory asynchronously while it decodes the
+// current one, so no global load is waited for inside the loop; it writes its own
+// codes back, so the CTA synchronises only for the column exchanges.
 // ---------------------------------------------------------------------------------
 template <class Store, bool kMixed, bool H16>
-__global__ void __launch_bounds__(NT, 2)
+__global__ void __launch_bounds__(2 * NT, 1)
 decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* __restrict__ q,
               const float* __restrict__ k, const float* __restrict__ v,
               const float* __restrict__ gate, const float* __restrict__ beta,
               float* __restrict__ out) {
-  __shared__ CtaSmem cs;
-  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  const int r0 = w * RPW;
-  const int h = blockIdx.x / B, bq = blockIdx.x - h * B;
-  const int slot = slots[bq];
-  if (slot < 0 || slot >= P.n_slots) {
-    if (tid == 0) atomicOr(P.err, ERR_SLOT_RANGE);
-    return;
-  }
-  const HeadRef<H16> hr = head_ref<H16>(P, slot, h);
-  const int vi = bq * P.H + h;
-  const uint64_t vec = uint64_t(vi) * D;
+  extern __shared__ __align__(16) uint8_t smem_bytes[];
+  const int grp = group_id();
+  DecodeSmem& sm = reinterpret_cast<DecodeSmem*>(smem_bytes)[grp];
+  CtaSmem& cs = sm.cs;
+  const int tid = group_tid(), w = tid >> 5, lane = tid & 31;
   WarpRows& wr = cs.wr[w];
-  // this warp's packed rows -> shared memory (16-byte asynchronous copies)
-  const int wstart = int(P.warp_code_off[h * NW + w]);
-  const int wend = (w + 1 < NW) ? int(P.warp_code_off[h * NW + w + 1]) : hr.code_bytes;
-  for (int o = 16 * lane; o < wend - wstart; o += 16 * 32) cp_async16(wr.codes + o, hr.codes + wstart + o);
-  asm volatile("cp.async.commit_group;" ::: "memory");
-  const float gate_s = (P.kind == 0) ? gate[vi] : 0.0f;
-  load_warp_rows(P, h, wr, lane, r0, k + vec, q + vec, &hr.sc, P.kind == 0 ? nullptr : gate + vec, gate_s);
-  const float beta_s = beta[vi];
-  const float4 c4 = hr.sc.get4(D + 4 * lane);
-  const f2 cin[2] = {make_float2(c4.x, c4.y), make_float2(c4.z, c4.w)};
-  const float v_own = v[vec + 16 * w + (lane & 15)];
-  asm volatile("cp.async.wait_all;" ::: "memory");
-  __syncwarp();
-  float* o_out = out + vec;
-  switch (hr.bits) {
-    case 2: decode_warp<2, Store, H16>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
-    case 4: decode_warp<4, Store, H16>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
-    case 6: decode_warp<6, Store, H16>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
-    case 8: decode_warp<8, Store, H16>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out); break;
-    case PIVOT: decode_pivot_warp(cs, wr, hr, v_own, beta_s, o_out); break;
-    default:
-      // heads whose rows have different widths (only pools with such heads launch this)
-      if constexpr (kMixed) decode_warp<MIXED, Store, H16>(cs, wr, hr, wstart, cin, v_own, beta_s, o_out);
-      break;
+  WarpRaw& raw = sm.raw[w];
+  if (tid < 8) {
+    const void* base = tid == 0 ? static_cast<const void*>(k) : tid == 1 ? static_cast<const void*>(q)
+                     : tid == 2 ? static_cast<const void*>(gate) : tid == 3 ? static_cast<const void*>(v)
+                     : tid == 4 ? static_cast<const void*>(P.row_info) : tid == 5 ? static_cast<const void*>(P.g)
+                     : tid == 6 ? static_cast<const void*>(P.omega) : static_cast<const void*>(P.scales);
+    sm.ptab[tid] = static_cast<const uint8_t*>(base);
+  }
+  group_sync();
+  // group g of CTA b takes the items m = 2 b + g, 2 b + g + 2 gridDim.x, ..., with
+  // m = h * B + bq; the next one is reached by adding (dh, db) with one carry (no
+  // division inside the loop)
+  const int G = 2 * int(gridDim.x);
+  const int dh = G / B, db = G - dh * B;
+  const int m0 = 2 * int(blockIdx.x) + grp;
+  int h = m0 / B, bq = m0 - h * B;
+  if (h >= P.H) return;
+  // the second group starts about half an item later, so that the two groups sharing
+  // the SM are mostly in different phases of the step (a bounded, one-time wait)
+  if (grp == 1)
+    for (int i = 0; i < 8; ++i) __nanosleep(500);
+  {
+    int hn = h + dh, bn = bq + db;
+    if (bn >= B) { bn -= B; ++hn; }
+    prefetch_item<H16>(P, slots, beta, gate, sm.ptab, raw, wr.codes[0], h, bq, slots[bq],
+                       P.warp_rec[h * NW + w], hn < P.H, hn, bn, w, lane);
+  }
+  for (int cur = 0; h < P.H; cur ^= 1) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncwarp();
+    const int slot = raw.slot;
+    const uint4 rec = raw.rec;
+    // this item's row data -> the working area (lanes 0..15, one row each)
+    if (lane < RPW) {
+      const uint32_t info = raw.info[lane];
+      wr.info[lane] = info;
+      wr.g[lane] = raw.g[lane];
+      wr.om[lane] = raw.om[lane];
+      if constexpr (kMixed) mixed_row_consts(wr, lane, row_bits(info));
+      const float dec = (P.kind == 0) ? raw.gate_s : raw.gate[lane];
+      float r_in;
+      if constexpr (H16) r_in = __half2float(reinterpret_cast<const __half*>(raw.r)[lane]);
+      else r_in = __uint_as_float(raw.r[lane]);
+      const float rd = fmul(dec, r_in);
+      const float kv = raw.k[lane], qv = raw.q[lane];
+      wr.dec[lane] = dec;
+      wr.kk[lane] = make_float2(kv, kv);
+      wr.qq[lane] = make_float2(qv, qv);
+      wr.rdd[lane] = make_float2(rd, rd);
+    }
+    const float beta_s = raw.beta;
+    f2 cin[2];
+    if constexpr (H16) {
+      const uint2 hb = reinterpret_cast<const uint2*>(raw.c)[lane];
+      half4_floats(hb, cin[0], cin[1]);
+    } else {
+      const float4 c4 = reinterpret_cast<const float4*>(raw.c)[lane];
+      cin[0] = make_float2(c4.x, c4.y);
+      cin[1] = make_float2(c4.z, c4.w);
+    }
+    const float v_own = raw.v[lane & 15];
+    int hn = h + dh, bn = bq + db;
+    if (bn >= B) { bn -= B; ++hn; }
+    if (hn < P.H) {
+      const int next_slot = raw.next_slot;
+      const uint4 next_rec = raw.next_rec;
+      int hnn = hn + dh, bnn = bn + db;
+      if (bnn >= B) { bnn -= B; ++hnn; }
+      __syncwarp();   // the raw area is consumed: the next item's copies may overwrite it
+      prefetch_item<H16>(P, slots, beta, gate, sm.ptab, raw, wr.codes[cur ^ 1], hn, bn, next_slot, next_rec,
+                         hnn < P.H, hnn, bnn, w, lane);
+    }
+    if (slot >= 0 && slot < P.n_slots) {
+      HeadRef<H16> hr;
+      hr.err = P.err;
+      hr.codes = P.codes + uint64_t(slot) * P.slot_code_bytes + rec.x;
+      hr.pivots = P.pivots + (uint64_t(slot) * P.n_pivot_rows + (rec.w >> 8)) * D;
+      hr.sc.p = static_cast<uint8_t*>(P.scales) + (uint64_t(slot) * P.H + h) * 2 * D * (H16 ? 2 : 4);
+      hr.bits = int(rec.w & 0xFFu);
+      hr.code_bytes = 0;     // not used by the decode step
+      hr.piv_count = 0;
+      hr.piv_stage_off = 0;
+      const int wstart = int(rec.y);
+      uint8_t* wcodes = wr.codes[cur];
+      float* o_out = out + (uint64_t(bq) * P.H + h) * D;
+      switch (hr.bits) {
+        case 2: decode_warp<2, Store, H16>(cs, wr, hr, wstart, wcodes, cin, v_own, beta_s, o_out); break;
+        case 4: decode_warp<4, Store, H16>(cs, wr, hr, wstart, wcodes, cin, v_own, beta_s, o_out); break;
+        case 6: decode_warp<6, Store, H16>(cs, wr, hr, wstart, wcodes, cin, v_own, beta_s, o_out); break;
+        case 8: decode_warp<8, Store, H16>(cs, wr, hr, wstart, wcodes, cin, v_own, beta_s, o_out); break;
+        case PIVOT: decode_pivot_warp(cs, wr, hr, v_own, beta_s, o_out); break;
+        default:
+          // heads whose rows have different widths (only pools with such heads launch this)
+          if constexpr (kMixed) decode_warp<MIXED, Store, H16>(cs, wr, hr, wstart, wcodes, cin, v_own, beta_s, o_out);
+          break;
+      }
+    } else if (tid == 0) {
+      atomicOr(P.err, ERR_SLOT_RANGE);
+    }
+    h = hn;
+    bq = bn;
   }
 }
 
@@ -638,7 +824,7 @@ decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* 
 template <int BITS, class Store, bool H16>
 __device__ __forceinline__ void quantize_warp(CtaSmem& cs, WarpRows& wr, const HeadRef<H16>& hr, int warp_code_start,
                                               const float* src) {
-  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int tid = group_tid(), w = tid >> 5, lane = tid & 31;
   const int r0 = w * RPW;
   f2 s[RPW][2];
 #pragma unroll
@@ -652,13 +838,14 @@ __device__ __forceinline__ void quantize_warp(CtaSmem& cs, WarpRows& wr, const H
         *reinterpret_cast<uint2*>(hr.pivots + row_off(info) * D + 4 * lane) = half4_bits(s[rr][0], s[rr][1]);
     }
   }
-  Store::template store<BITS>(cs, wr, s, hr.sc, hr.codes, warp_code_start, nullptr);
+  Store::template store<BITS>(cs, wr, s, hr.sc, hr.codes, warp_code_start, nullptr, wr.codes[0]);
 }
 
 template <class Store, bool H16>
 __global__ void __launch_bounds__(NT, 2)
 quantize_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* __restrict__ S) {
-  __shared__ CtaSmem cs;
+  extern __shared__ __align__(16) uint8_t smem_bytes[];
+  CtaSmem& cs = *reinterpret_cast<CtaSmem*>(smem_bytes);
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int r0 = w * RPW;
   const int item = blockIdx.x;
@@ -691,6 +878,58 @@ quantize_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float
       break;
     default: quantize_warp<MIXED, Store, H16>(cs, wr, hr, wstart, src); break;
   }
+}
+
+// ---------------------------------------------------------------------------------
+// Launch helpers. Kernels whose shared memory exceeds the default 48 KB raise their
+// limit once per device; the persistent decode kernel runs as many CTAs as fit on the
+// device at once (SM count x resident CTAs per SM, also found once per device).
+// ---------------------------------------------------------------------------------
+constexpr int kMaxDevices = 64;
+
+template <auto Kern>
+cudaError_t kernel_setup(int smem, int* per_device_cap, int threads = NT) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static int cap_cache[kMaxDevices];
+  int cap = (dev >= 0 && dev < kMaxDevices) ? cap_cache[dev] : 0;
+  if (cap == 0) {
+    e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int nsm = 0, per = 0;
+    e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, Kern, threads, smem);
+    if (e != cudaSuccess) return e;
+    cap = nsm * (per > 0 ? per : 1);
+    if (dev >= 0 && dev < kMaxDevices) cap_cache[dev] = cap;
+  }
+  *per_device_cap = cap;
+  return cudaSuccess;
+}
+
+// One CTA per item (grid = n_items), dynamic shared memory `smem`.
+template <auto Kern, class... Args>
+cudaError_t launch_items(unsigned n_items, int smem, cudaStream_t s, Args... args) {
+  int cap = 0;
+  cudaError_t e = kernel_setup<Kern>(smem, &cap);
+  if (e != cudaSuccess) return e;
+  Kern<<<n_items, NT, smem, s>>>(args...);
+  return cudaGetLastError();
+}
+
+// Persistent decode CTAs of two 256-thread groups, each on its own items: grid =
+// min(ceil(n_items / 2), CTAs resident on the device at once).
+template <auto Kern, class... Args>
+cudaError_t launch_persistent(unsigned n_items, int smem, cudaStream_t s, Args... args) {
+  int cap = 0;
+  cudaError_t e = kernel_setup<Kern>(smem, &cap, 2 * NT);
+  if (e != cudaSuccess) return e;
+  const unsigned pairs = (n_items + 1) / 2;
+  const unsigned grid = pairs < unsigned(cap) ? pairs : unsigned(cap);
+  Kern<<<grid, 2 * NT, smem, s>>>(args...);
+  return cudaGetLastError();
 }
 
 }  // namespace

@@ -44,6 +44,11 @@ struct PoolDev {
   const uint32_t* head_bits;        // [H] the width shared by all rows of head h
                                     //   (2/4/6/8, or 16 if all rows are pivots), 0 if mixed
   const uint32_t* warp_code_off;    // [H*8] byte offset in head h where rows 16w.. start
+  const uint4* warp_rec;            // [H*8] what the decode step prefetches for warp w of
+                                    //   head h: {x: byte offset of head h in a slot,
+                                    //   y: byte offset of rows 16w.. in head h, z: their
+                                    //   code bytes, w: head width (low 8 bits, 0 if mixed)
+                                    //   | index of the head's first pivot row << 8}
   const uint32_t* row_info;         // [H*D] bits (low 8) | byte offset in head << 8
                                     //   (pivot rows: index in head's pivot block << 8)
   const float* g;                   // [H*D] row gain (omega_i / mean omega)^(-1/2)
@@ -57,12 +62,13 @@ struct PoolDev {
 // Byte layout of the meta buffer, computed on the host.
 struct MetaLayout {
   size_t head_code_off, head_code_bytes, head_piv_first, head_piv_count, head_bits;
-  size_t warp_code_off, row_info, g, omega, err, total;
+  size_t warp_code_off, warp_rec, row_info, g, omega, err, total;
 };
 
 MetaLayout meta_layout(int H);
 
-// Launchers (stq_kernels.cu). They return the cudaGetLastError() of the launch.
+// Launchers (stq_kernels.cu). They return the cudaGetLastError() of the launch (or of
+// the one-time set-up of the kernel's shared-memory size and the device's SM count).
 cudaError_t launch_decode(const PoolDev& P, const int32_t* slots, int B, const float* q,
                           const float* k, const float* v, const float* gate,
                           const float* beta, float* out, cudaStream_t s);
@@ -80,6 +86,20 @@ cudaError_t launch_quantize_absmax(const PoolDev& P, const int32_t* slots, int B
 cudaError_t launch_fp32_step(int kind, int B, int H, float* S, const float* q,
                              const float* k, const float* v, const float* gate,
                              const float* beta, float* out, cudaStream_t s);
+
+// Device staging of one host-buffer decode step for B requests: q, k, v, gate, beta and
+// the readout, each 16-byte aligned (byte offsets; element counts). Used by
+// stq_decode_step_host, stq_decode_step_host_static and the pipeline (stq_abi.cpp).
+struct StagingLayout {
+  size_t q, k, v, gate, beta, out, total;
+  size_t n_vec, n_gate, n_beta;
+};
+StagingLayout staging_layout(const PoolDev& P, int B);
+
+// The argument checks every batched entry point makes (pool not NULL, 0 <= B,
+// B * H < 2^31, d_slots not NULL when B > 0). Returns an stq_status (0 = STQ_OK) and
+// sets the thread's last error message on failure.
+int check_batch(const struct ::stq_pool* pool, const int32_t* d_slots, int B);
 
 // Accessors for entry points that live outside stq_abi.cpp.
 const PoolDev* pool_dev(const struct ::stq_pool* pool);

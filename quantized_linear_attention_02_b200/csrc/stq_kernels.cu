@@ -44,8 +44,9 @@ namespace {
 // ---------------------------------------------------------------------------------
 template <int BITS, class Sc>
 __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], const Sc& sc,
-                                            uint8_t* codes_global, int warp_code_start, float* o_global) {
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+                                            uint8_t* codes_global, int warp_code_start, float* o_global,
+                                            uint8_t* stage) {
+  const int w = group_tid() >> 5, lane = group_tid() & 31;
   const int r0 = w * RPW;
 
   // --- row scale r_i = (tree sum_j |S_ij|) / 128 * g_i -------------------------------
@@ -106,11 +107,13 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
     s[rr][0] = mul2(s[rr][0], ir);
     s[rr][1] = mul2(s[rr][1], ir);
     if constexpr (BITS == MIXED) {
-      const float iq = wr.iq[rr];
-      mx[0] = fmaxf(mx[0], fmul(fabsf(s[rr][0].x), iq));
-      mx[1] = fmaxf(mx[1], fmul(fabsf(s[rr][0].y), iq));
-      mx[2] = fmaxf(mx[2], fmul(fabsf(s[rr][1].x), iq));
-      mx[3] = fmaxf(mx[3], fmul(fabsf(s[rr][1].y), iq));
+      // |y| / qmax_i as |y * fl(1/qmax_i)| (rounding is symmetric)
+      const f2 iq = dup(wr.iq[rr]);
+      const f2 p01 = mul2(s[rr][0], iq), p23 = mul2(s[rr][1], iq);
+      mx[0] = fmaxf(mx[0], fabsf(p01.x));
+      mx[1] = fmaxf(mx[1], fabsf(p01.y));
+      mx[2] = fmaxf(mx[2], fabsf(p23.x));
+      mx[3] = fmaxf(mx[3], fabsf(p23.y));
     } else {
       mx[0] = fmaxf(mx[0], fabsf(s[rr][0].x));
       mx[1] = fmaxf(mx[1], fabsf(s[rr][0].y));
@@ -119,7 +122,7 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
     }
   }
   cs.red[1][1][w][lane] = make_float4(mx[0], mx[1], mx[2], mx[3]);
-  __syncthreads();
+  group_sync();
 
   if (o_global != nullptr && w == 0) {
     f2 lo, hi;
@@ -141,11 +144,12 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
       m = fmul(m, __frcp_rn(QM));
     }
     c_own = m;
-    if (lane < 16) cs.col_ic[jown] = recip_scale(c_own);
+    const float ic0 = recip_scale(c_own);
+    if (lane < 16) cs.col_ic[jown] = ic0;
   }
   const float c0 = c_own;
   int wide = 0, any_wide = 0;
-  __syncthreads();
+  group_sync();
 
   // --- two least-squares steps: c_j <- sum_i p y / sum_i p Q, p = b_i Q_ij -------------
 #pragma unroll
@@ -166,8 +170,9 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
         const f2 bb = e == 0 ? make_float2(b2.x, b2.y) : make_float2(b2.z, b2.w);
         float lo_b, hi_b;
         if constexpr (BITS == MIXED) {
-          lo_b = MAGIC - wr.qm[rr];
-          hi_b = MAGIC + wr.qm[rr];
+          const f2 cb = wr.clampb[rr];
+          lo_b = cb.x;
+          hi_b = cb.y;
         } else {
           lo_b = MAGIC - float((1 << (BITS - 1)) - 1);
           hi_b = MAGIC + float((1 << (BITS - 1)) - 1);
@@ -193,7 +198,7 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
     });
     put_partial(cs.red[it][0], w, lane, nd.x[0], nd.x[1]);
     put_partial(cs.red[it][1], w, lane, nd.x[2], nd.x[3]);
-    __syncthreads();
+    group_sync();
     {
       // lanes 0..15: numerator of column jown, lanes 16..31: its denominator
       const float* part = reinterpret_cast<const float*>(cs.red[it][lane >> 4][0]);
@@ -202,19 +207,19 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
       for (int ww = 0; ww < NW; ++ww) x[ww] = part[ww * D + jown];
       const float sum = fadd(fadd(fadd(x[0], x[1]), fadd(x[2], x[3])), fadd(fadd(x[4], x[5]), fadd(x[6], x[7])));
       const float den = __shfl_down_sync(0xffffffffu, sum, 16);
-      if (lane < 16) {
-        if (den > 0.0f) c_own = __fdiv_rn(sum, den);
-        if (it == 1) c_own = sc.stored(c_own);   // the final c as the pool will hold it
-        const float icn = recip_scale(c_own);
-        cs.col_ic[jown] = icn;
-        // every least-squares step keeps c >= c_before / 2 (each term Q y >= c Q^2 / 2),
-        // so |n| = |rint(y / c)| <= qmax c0 / c + 1/2 < 2^15 unless rounding at the bottom
-        // of the float32 range broke that; then the column takes the float clamp
-        if (it == 1) wide = !(fmul(c0, icn) < 128.0f);
-      }
+      // lanes 16..31 compute a value they never store (no divergent branch)
+      const float q = __fdiv_rn(sum, den);
+      if (den > 0.0f) c_own = q;
+      if (it == 1) c_own = sc.stored(c_own);   // the final c as the pool will hold it
+      const float icn = recip_scale(c_own);
+      if (lane < 16) cs.col_ic[jown] = icn;
+      // every least-squares step keeps c >= c_before / 2 (each term Q y >= c Q^2 / 2),
+      // so |n| = |rint(y / c)| <= qmax c0 / c + 1/2 < 2^15 unless rounding at the bottom
+      // of the float32 range broke that; then the column takes the float clamp
+      if (it == 1) wide = lane < 16 && !(fmul(c0, icn) < 128.0f);
     }
-    if (it == 1) any_wide = __syncthreads_or(wide);
-    else __syncthreads();
+    if (it == 1) any_wide = group_sync_or(wide);
+    else group_sync();
   }
 
   // --- final codes with the final c, stored straight into the pool -------------------
@@ -242,7 +247,6 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
       // Mixed widths: clamp in 16-bit lanes, pack any width without a branch, and put
       // each lane's b/2 bytes into the warp's staging area (the staged codes are consumed
       // by now; it has the pool's layout), then copy the area out with 16-byte stores.
-      uint8_t* stage = wr.codes;
 #pragma unroll
       for (int rr = 0; rr < RPW; ++rr) {
         const uint32_t info = wr.info[rr];
@@ -311,8 +315,8 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
 struct StepQuantStore {
   template <int BITS, class Sc>
   static __device__ __forceinline__ void store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], const Sc& sc,
-                                               uint8_t* codes, int warp_code_start, float* o) {
-    refit_store<BITS>(cs, wr, s, sc, codes, warp_code_start, o);
+                                               uint8_t* codes, int warp_code_start, float* o, uint8_t* stage) {
+    refit_store<BITS>(cs, wr, s, sc, codes, warp_code_start, o, stage);
   }
 };
 
@@ -472,24 +476,24 @@ cudaError_t launch_decode(const PoolDev& P, const int32_t* slots, int B, const f
                           const float* beta, float* out, cudaStream_t s) {
   if (B == 0) return cudaSuccess;
   if (P.scheme == SCHEME_ROW_ABSMAX) return launch_decode_absmax(P, slots, B, q, k, v, gate, beta, out, s);
-  const unsigned grid = unsigned(B) * unsigned(P.H);
+  const unsigned n = unsigned(B) * unsigned(P.H);
+  constexpr int SM = 2 * sizeof(DecodeSmem);
   if (P.scale16) {
-    if (P.any_mixed) decode_kernel<StepQuantStore, true, true><<<grid, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
-    else decode_kernel<StepQuantStore, false, true><<<grid, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
-  } else {
-    if (P.any_mixed) decode_kernel<StepQuantStore, true, false><<<grid, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
-    else decode_kernel<StepQuantStore, false, false><<<grid, NT, 0, s>>>(P, slots, B, q, k, v, gate, beta, out);
+    if (P.any_mixed) return launch_persistent<decode_kernel<StepQuantStore, true, true>>(n, SM, s, P, slots, B, q, k, v, gate, beta, out);
+    return launch_persistent<decode_kernel<StepQuantStore, false, true>>(n, SM, s, P, slots, B, q, k, v, gate, beta, out);
   }
-  return cudaGetLastError();
+  if (P.any_mixed) return launch_persistent<decode_kernel<StepQuantStore, true, false>>(n, SM, s, P, slots, B, q, k, v, gate, beta, out);
+  return launch_persistent<decode_kernel<StepQuantStore, false, false>>(n, SM, s, P, slots, B, q, k, v, gate, beta, out);
 }
 
 cudaError_t launch_quantize(const PoolDev& P, const int32_t* slots, int B, const float* S,
                             cudaStream_t s) {
   if (B == 0) return cudaSuccess;
   if (P.scheme == SCHEME_ROW_ABSMAX) return launch_quantize_absmax(P, slots, B, S, s);
-  if (P.scale16) quantize_kernel<StepQuantStore, true><<<B * P.H, NT, 0, s>>>(P, slots, B, S);
-  else quantize_kernel<StepQuantStore, false><<<B * P.H, NT, 0, s>>>(P, slots, B, S);
-  return cudaGetLastError();
+  const unsigned n = unsigned(B) * unsigned(P.H);
+  constexpr int SM = sizeof(CtaSmem);
+  if (P.scale16) return launch_items<quantize_kernel<StepQuantStore, true>>(n, SM, s, P, slots, B, S);
+  return launch_items<quantize_kernel<StepQuantStore, false>>(n, SM, s, P, slots, B, S);
 }
 
 cudaError_t launch_dequantize(const PoolDev& P, const int32_t* slots, int B, float* S_out,

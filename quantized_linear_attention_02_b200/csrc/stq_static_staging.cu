@@ -17,8 +17,6 @@ constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 void* g_staging_addr[kMaxDevices];   // device address of g_static_staging, per device
 
-size_t up16(size_t x) { return (x + 15) & ~size_t(15); }
-
 // Device address of the staging array on the current device (looked up once per device).
 cudaError_t staging_address(void** out) {
   int dev = 0;
@@ -48,31 +46,21 @@ extern "C" stq_status stq_decode_step_host_static(stq_pool* pool, const int32_t*
                                                   const float* h_v, const float* h_gate,
                                                   const float* h_beta, float* h_out,
                                                   void* stream) {
-  const stq::PoolDev* P = stq::pool_dev(pool);
-  if (P == nullptr) return fail(STQ_ERR_INVALID_ARG, "pool is NULL");
-  if (B < 0) return fail(STQ_ERR_INVALID_ARG, "B must be >= 0");
+  const int st = stq::check_batch(pool, d_slots, B);
+  if (st != STQ_OK) return static_cast<stq_status>(st);
   if (B == 0) {
     stq::clear_last_error();
     return STQ_OK;
   }
-  if (d_slots == nullptr) return fail(STQ_ERR_INVALID_ARG, "d_slots is NULL");
   if (!h_q || !h_k || !h_v || !h_gate || !h_beta || !h_out)
     return fail(STQ_ERR_INVALID_ARG, "a host pointer is NULL");
-  const size_t BH = size_t(B) * size_t(P->H);
-  const size_t n_vec = BH * stq::D;
-  const size_t n_gate = (P->kind == STQ_GDN) ? BH : n_vec;
-  size_t o = 0;
-  const size_t oq = o;    o = up16(o + n_vec * 4);
-  const size_t ok = o;    o = up16(o + n_vec * 4);
-  const size_t ov = o;    o = up16(o + n_vec * 4);
-  const size_t og = o;    o = up16(o + n_gate * 4);
-  const size_t ob = o;    o = up16(o + BH * 4);
-  const size_t oo = o;    o = up16(o + n_vec * 4);
-  if (o > STQ_STATIC_STAGING_BYTES) {
+  const stq::PoolDev* P = stq::pool_dev(pool);
+  const stq::StagingLayout L = stq::staging_layout(*P, B);
+  if (L.total > STQ_STATIC_STAGING_BYTES) {
     char msg[256];
     snprintf(msg, sizeof(msg),
              "B=%d x H=%d needs %zu bytes of staging, more than the static %u; "
-             "use stq_decode_step_host with a caller buffer", B, P->H, o,
+             "use stq_decode_step_host with a caller buffer", B, P->H, L.total,
              unsigned(STQ_STATIC_STAGING_BYTES));
     return fail(STQ_ERR_INVALID_ARG, msg);
   }
@@ -85,15 +73,15 @@ extern "C" stq_status stq_decode_step_host_static(stq_pool* pool, const int32_t*
   }
   uint8_t* base = static_cast<uint8_t*>(base_v);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  float* dq = reinterpret_cast<float*>(base + oq);
-  float* dk = reinterpret_cast<float*>(base + ok);
-  float* dv = reinterpret_cast<float*>(base + ov);
-  float* dg = reinterpret_cast<float*>(base + og);
-  float* db = reinterpret_cast<float*>(base + ob);
-  float* dout = reinterpret_cast<float*>(base + oo);
+  float* dq = reinterpret_cast<float*>(base + L.q);
+  float* dk = reinterpret_cast<float*>(base + L.k);
+  float* dv = reinterpret_cast<float*>(base + L.v);
+  float* dg = reinterpret_cast<float*>(base + L.gate);
+  float* db = reinterpret_cast<float*>(base + L.beta);
+  float* dout = reinterpret_cast<float*>(base + L.out);
   struct Copy { void* dst; const void* src; size_t n; };
-  const Copy in[] = {{dq, h_q, n_vec * 4}, {dk, h_k, n_vec * 4}, {dv, h_v, n_vec * 4},
-                     {dg, h_gate, n_gate * 4}, {db, h_beta, BH * 4}};
+  const Copy in[] = {{dq, h_q, L.n_vec * 4}, {dk, h_k, L.n_vec * 4}, {dv, h_v, L.n_vec * 4},
+                     {dg, h_gate, L.n_gate * 4}, {db, h_beta, L.n_beta * 4}};
   for (const Copy& c : in) {
     e = cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) {
@@ -108,7 +96,7 @@ extern "C" stq_status stq_decode_step_host_static(stq_pool* pool, const int32_t*
     snprintf(msg, sizeof(msg), "stq_decode_step launch: %s", cudaGetErrorString(e));
     return fail(STQ_ERR_CUDA, msg);
   }
-  e = cudaMemcpyAsync(h_out, dout, n_vec * 4, cudaMemcpyDeviceToHost, s);
+  e = cudaMemcpyAsync(h_out, dout, L.n_vec * 4, cudaMemcpyDeviceToHost, s);
   if (e != cudaSuccess) {
     char msg[256];
     snprintf(msg, sizeof(msg), "device-to-host copy of the readout: %s", cudaGetErrorString(e));

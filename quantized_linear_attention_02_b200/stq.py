@@ -15,6 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libstq.so")
 
 STQ_GDN, STQ_KDA = 0, 1
+STATIC_STAGING_BYTES = 8 << 20     # STQ_STATIC_STAGING_BYTES of include/stq.h
 D = 128
 PIVOT_BITS = 16
 KINDS = {"gdn": STQ_GDN, "kda": STQ_KDA}
@@ -67,10 +68,16 @@ def lib():
         "stq_decode_step_host": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                       ctypes.c_size_t, _vp]),
         "stq_decode_step_host_static": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+        "stq_pipeline_staging_bytes": (ctypes.c_size_t, [_vp, _i]),
+        "stq_pipeline_create": (_i, [_vp, _i, _vp, ctypes.c_size_t, ctypes.POINTER(_vp)]),
+        "stq_pipeline_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+        "stq_pipeline_finish": (_i, [_vp, _vp]),
+        "stq_pipeline_destroy": (None, [_vp]),
         "stq_dequantize": (_i, [_vp, _vp, _i, _vp, _vp]),
         "stq_fp32_decode_step": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
         "stq_pool_check": (_i, [_vp, _vp]),
         "stq_row_sq_error": (_i, [_vp, _vp, _i, _vp, _i, _vp]),
+        "stq_row_error_at_widths": (_i, [_vp, _vp, _i, _vp, _vp, _i, _vp, _vp]),
         "stq_lifetime_weights": (_i, [_vp, _i, _i, _vp]),
         "stq_unit_distortion": (_i, [_i, _i, _i, _vp, _vp, _vp]),
         "stq_allocate_bits": (_i, [_i, _i, _vp, _vp, _vp, ctypes.c_double, _i, _vp]),
@@ -234,6 +241,21 @@ class Pool:
             ctypes.c_void_p(h_gate.data_ptr()), ctypes.c_void_p(h_beta.data_ptr()),
             ctypes.c_void_p(h_out.data_ptr()), _stream(stream)))
 
+    def row_error_at_widths(self, slots, S, cand_bits, err, stream=None):
+        """In-head row errors at candidate widths (stq_row_error_at_widths): S [B, H, 128,
+        128] float32 CUDA, err [B, H, 128, len(cand_bits)] float32 CUDA."""
+        import torch
+        B = slots.numel()
+        cb = np.ascontiguousarray(cand_bits, dtype=np.int32)
+        _check(lib().stq_row_error_at_widths(
+            self.handle, self._slots(slots), B, _ptr(S, torch.float32, "S", B * self.H * D * D),
+            cb.ctypes.data_as(ctypes.c_void_p), int(cb.size),
+            _ptr(err, torch.float32, "err", B * self.H * D * cb.size), _stream(stream)))
+
+    def pipeline(self, B, staging=None):
+        """A Pipeline of host-buffer decode steps of B requests (see Pipeline)."""
+        return Pipeline(self, B, staging)
+
     def dequantize(self, slots, S_out, stream=None):
         import torch
         B = slots.numel()
@@ -304,3 +326,50 @@ def allocate_bits(lifetime, dist, cand_bits, budget, n_pivots):
     _check(lib().stq_allocate_bits(L.size, cb.size, cb.ctypes.data, L.ctypes.data, Dm.ctypes.data,
                                    float(budget), int(n_pivots), out.ctypes.data))
     return out
+
+
+class Pipeline:
+    """stq_pipeline_* of include/stq.h: host-buffer decode steps whose copies overlap the
+    previous and next steps inside the library. `step` enqueues one step and returns once
+    the previous step's readout is in its host tensor; `finish` waits for the last one.
+    The staging buffer (a uint8 CUDA tensor, allocated here if not given) and the pool
+    must outlive the pipeline."""
+
+    def __init__(self, pool, B, staging=None):
+        import torch
+        self.pool, self.B = pool, int(B)
+        need = int(lib().stq_pipeline_staging_bytes(pool.handle, self.B))
+        if staging is None:
+            staging = torch.empty(need, dtype=torch.uint8, device=pool.codes.device)
+        self.staging = staging
+        h = ctypes.c_void_p()
+        _check(lib().stq_pipeline_create(pool.handle, self.B, _ptr(staging, torch.uint8, "staging"),
+                                         ctypes.c_size_t(staging.numel()), ctypes.byref(h)))
+        self.handle = h
+
+    def step(self, slots, h_q, h_k, h_v, h_gate, h_beta, h_out, stream=None):
+        import torch
+        if slots.numel() != self.B:
+            raise ValueError(f"the pipeline runs {self.B} requests, got {slots.numel()} slots")
+        for name, t in (("q", h_q), ("k", h_k), ("v", h_v), ("gate", h_gate), ("beta", h_beta), ("out", h_out)):
+            if t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+                raise ValueError(f"host {name} must be a contiguous float32 CPU tensor")
+        _check(lib().stq_pipeline_step(
+            self.handle, self.pool._slots(slots), ctypes.c_void_p(h_q.data_ptr()),
+            ctypes.c_void_p(h_k.data_ptr()), ctypes.c_void_p(h_v.data_ptr()),
+            ctypes.c_void_p(h_gate.data_ptr()), ctypes.c_void_p(h_beta.data_ptr()),
+            ctypes.c_void_p(h_out.data_ptr()), _stream(stream)))
+
+    def finish(self, stream=None):
+        _check(lib().stq_pipeline_finish(self.handle, _stream(stream)))
+
+    def close(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            lib().stq_pipeline_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # pragma: no cover - interpreter shutdown
+            pass
