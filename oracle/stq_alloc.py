@@ -107,3 +107,38 @@ def allocate(lifetime, dist, cand_bits, budget, n_pivots):
         bits[rest[t]] = cand[ci]
         s -= ks[ci]
     return bits
+
+
+def row_error_at_widths(S, c, omega, cand_bits, scale16=False):
+    """Distortion of every row at every candidate width inside a head whose column scales
+    are fixed: the head's rows share c_j, so a row's width b only sets how far its codes
+    reach (+-qmax_b steps of r_i c_j). For state n, head h, row i and candidate b:
+      r_i   = (tree sum_j |S_ij|) * (1/d) * g_i, the refit's row scale (every row, pivot
+              rows included: the width they would get is what is measured);
+      Q_ij  = clamp(rint((S_ij * fl(1/r_i)) * fl(1/c_j)), -qmax_b, qmax_b) on the exact
+              product, 0 when r_i or c_j is below 2^-126;
+      e_i(b) = tree sum_j (S_ij - (Q_ij r_i) c_j)^2 in float32, as row_sq_error.
+    S [N, H, d, d] float32; c [N, H, d] float32 (the allocated pool's column scales);
+    omega [H, d]; scale16: r rounded to binary16 as a compact pool stores it; returns
+    [N, H, d, n_cand] float32.
+    Reading (the pages name a per-row squared error for KDA units but not the scales it
+    is taken under): the allocation is iterated with these in-head errors, since a KDA
+    row quantised alone at width b gets a column scale it would not have in a head of
+    mixed widths."""
+    from .stq_oracle import _recip, row_gain, qmax_of
+    S = np.asarray(S, dtype=F32)
+    c = np.asarray(c, dtype=F32)
+    d = S.shape[-1]
+    g = row_gain(omega)
+    r = (tree_sum(np.abs(S), axis=-1) * F32(1.0 / d) * g).astype(F32)
+    if scale16:
+        r = r.astype(np.float16).astype(F32)
+    y = (S * _recip(r)[..., :, None]).astype(F32)
+    x = y.astype(F64) * _recip(c).astype(F64)[..., None, :]
+    out = np.empty(S.shape[:-1] + (len(cand_bits),), F32)
+    for ci, b in enumerate(cand_bits):
+        qm = float(qmax_of(b))
+        Q = np.clip(np.rint(x), -qm, qm).astype(F32)
+        S_hat = ((Q * r[..., :, None]).astype(F32) * c[..., None, :]).astype(F32)
+        out[..., ci] = row_sq_error(S, S_hat)
+    return out

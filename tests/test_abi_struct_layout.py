@@ -99,3 +99,11 @@ def test_plain_c_caller(tmp_path):
     assert int(ok[4]) == 3 * 128 * 128 * 2 and int(ok[5]) == 128
     bad = out[2].split(maxsplit=2)
     assert bad[1] == "1" and len(bad) == 3 and bad[2]     # STQ_ERR_INVALID_ARG with a message
+
+
+def test_static_staging_size_matches_header():
+    import re
+    txt = open(os.path.join(ROOT, "include", "stq.h")).read()
+    m = re.search(r"#define\s+STQ_STATIC_STAGING_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", txt)
+    assert m, "STQ_STATIC_STAGING_BYTES not found in include/stq.h"
+    assert int(m.group(1)) << int(m.group(2)) == stq.STATIC_STAGING_BYTES

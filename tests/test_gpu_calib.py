@@ -112,3 +112,26 @@ def test_error_lifetime_diagnostic_matches_oracle(widx):
     err = rows.sum(axis=1) if w.kind == "gdn" else rows.reshape(-1)
     assert np.allclose(r["accumulated_sq_error"], err, rtol=1e-3, atol=1e-30)
     assert np.allclose(r["half_life"], np.log(0.5) / W.calibration_log_retention(w).reshape(-1))
+
+
+@pytest.mark.parametrize("scale_bits", [32, 16])
+def test_row_error_at_widths_matches_oracle(scale_bits):
+    """The in-head row errors (stq_row_error_at_widths) equal the oracle's bit for bit:
+    a KDA pool of mixed per-row widths with a pivot row, quantised from random states."""
+    rng = np.random.default_rng(5)
+    H, N = 3, 4
+    S = (rng.standard_normal((N, H, D, D)) * rng.lognormal(0, 1, (N, H, D, 1))).astype(F32)
+    om = rng.lognormal(0, 1, (H, D)).astype(F32)
+    rb = rng.choice([2, 4, 6, 8], size=(H, D))
+    rb[1, 9] = 16
+    pool = stq.Pool("kda", N + 2, rb.reshape(-1).astype(np.uint8), om, scale_bits=scale_bits)
+    slots = torch.tensor([2, 0, 5, 3], dtype=torch.int32, device="cuda")
+    Sg = dev(S)
+    pool.quantize_init(slots, Sg)
+    cand = (2, 4, 6, 8)
+    err = torch.empty((N, H, D, len(cand)), device="cuda")
+    pool.row_error_at_widths(slots, Sg, cand, err)
+    pool.check()
+    c = pool.scales_view()[slots.long(), :, 1].float().cpu().numpy()
+    ref = A.row_error_at_widths(S, c, om, cand, scale16=scale_bits == 16)
+    assert np.array_equal(err.cpu().numpy(), ref)

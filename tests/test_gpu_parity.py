@@ -90,9 +90,8 @@ def test_quantize_init_matches_oracle(widx):
     pool.check()
     ug, rg, cg, pg = T.read_pool_state(pool, L, [W.slot_of_request(b) for b in reqs])
     rb = W.row_bits(w)
-    n = T.compare_codes(ug, u, S0, r, c, rb, "quantize_init")
-    if n == 0:
-        assert np.array_equal(rg, r) and np.array_equal(cg, c)
+    n = T.compare_codes(ug, u, S0, r, c, rb, "quantize_init", config=w.name)
+    T.check_scales(rg, r, cg, c, n, "quantize_init")
     piv_rows = (rb == 16)
     assert np.array_equal(pg[:, piv_rows], piv[:, piv_rows])
 
@@ -112,10 +111,8 @@ def _single_step(w, reqs, t, pool, L):
     pool.decode_step(slots_t(reqs), dev(x.q), dev(x.k), dev(x.v), dev(x.gate), dev(x.beta), out)
     pool.check()
     ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
-    n = T.compare_codes(ug, u2, X, r2, c2, rb, f"{w.name} step {t}")
-    if n == 0:
-        assert np.array_equal(rg, r2), "row scales differ"
-        assert np.array_equal(cg, c2), "column scales differ"
+    n = T.compare_codes(ug, u2, X, r2, c2, rb, f"{w.name} step {t}", config=w.name)
+    T.check_scales(rg, r2, cg, c2, n, f"{w.name} step {t}")
     piv_rows = rb == 16
     assert np.array_equal(pg[:, piv_rows], p2[:, piv_rows])
     assert T.per_vector_rel_l2(out.cpu().numpy(), o).max() <= T.OUT_REL_L2
@@ -162,46 +159,94 @@ def test_decode_chain(widx, steps):
 # ---------------------------------------------------------------------------------
 # full-size workloads in the launch configuration the bench times
 # ---------------------------------------------------------------------------------
+def _full_size_start(w, pool, L, sample):
+    """Quantise every request's state (random ones, oracle-built warm states for the
+    sampled requests) and check the sample against the oracle's quantiser; then put the
+    oracle's packed state into the sampled slots so that later steps start identical.
+    Returns the oracle's packed state of the sample."""
+    om, rb = W.omega(w), W.row_bits(w)
+    g = torch.Generator(device="cuda").manual_seed(1234 + w.index)
+    S_all = torch.randn((w.B, w.H, D, D), device="cuda", generator=g) * 0.05
+    S0 = T.warm_states(w.index, sample)
+    S_all[sample] = dev(S0)
+    pool.quantize_init(slots_t(range(w.B)), S_all)
+    del S_all
+    pool.check()
+    u, r, c, piv = O.refit(S0, om, rb)
+    slots = [W.slot_of_request(b) for b in sample]
+    ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
+    n = T.compare_codes(ug, u, S0, r, c, rb, "full-size quantize_init", config=w.name)
+    T.check_scales(rg, r, cg, c, n, "full-size quantize_init")
+    T.write_oracle_state(pool, L, slots, u, r, c, piv)
+    return u, r, c, piv
+
+
+def _full_size_inputs(w, t, sample, gen):
+    """Inputs of step t for all B requests: the recipe's distributions from the device
+    RNG, with the sampled requests' inputs from their seeded NumPy streams."""
+    xin = dict(zip(("q", "k", "v", "gate", "beta"), W.torch_step_inputs(w, w.B, gen, "cuda")))
+    xs = T.inputs_for(w, "decode", t, sample)
+    for name in xin:
+        xin[name][sample] = dev(getattr(xs, name))
+    return xin, xs
+
+
 @pytest.mark.parametrize("widx", [3, 4])
 def test_full_size_sampled(widx):
     w = W.WORKLOADS[widx]
     pool, L, om = make_pool(w)
     sample = [int(b) for b in W.parity_sample(w, 8)]
-    # every request gets a state; the sampled ones get oracle-built ones
-    g = torch.Generator(device="cuda").manual_seed(1234 + widx)
-    S_all = torch.randn((w.B, w.H, D, D), device="cuda", generator=g) * 0.05
-    S0 = T.warm_states(widx, sample)
-    S_all[sample] = dev(S0)
-    all_slots = slots_t(range(w.B))
-    pool.quantize_init(all_slots, S_all)
-    del S_all
-    pool.check()
-    u, r, c, piv = O.refit(S0, om, W.row_bits(w))
-    ug, rg, cg, pg = T.read_pool_state(pool, L, [W.slot_of_request(b) for b in sample])
-    T.compare_codes(ug, u, S0, r, c, W.row_bits(w), "full-size quantize_init")
-    # one decode step over all B requests: random inputs, the sampled requests' from
-    # the seeded generator
+    u, r, c, piv = _full_size_start(w, pool, L, sample)
     gen = torch.Generator(device="cuda").manual_seed(99)
-    xin = {
-        "q": torch.nn.functional.normalize(torch.randn((w.B, w.H, D), device="cuda", generator=gen), dim=-1),
-        "k": torch.nn.functional.normalize(torch.randn((w.B, w.H, D), device="cuda", generator=gen), dim=-1),
-        "v": torch.randn((w.B, w.H, D), device="cuda", generator=gen),
-        "gate": torch.exp(torch.empty((w.B, w.H) if w.kind == "gdn" else (w.B, w.H, D),
-                                      device="cuda").uniform_(w.gate_low, w.gate_high, generator=gen)),
-        "beta": torch.sigmoid(torch.randn((w.B, w.H), device="cuda", generator=gen)),
-    }
-    xs = T.inputs_for(w, "decode", 0, sample)
-    for name in xin:
-        xin[name][sample] = dev(getattr(xs, name))
+    xin, xs = _full_size_inputs(w, 0, sample, gen)
     out = torch.empty((w.B, w.H, D), device="cuda")
-    pool.decode_step(all_slots, xin["q"], xin["k"], xin["v"], xin["gate"], xin["beta"], out)
+    pool.decode_step(slots_t(range(w.B)), xin["q"], xin["k"], xin["v"], xin["gate"], xin["beta"], out)
     pool.check()
     u2, r2, c2, p2, o, X = O.decode_step(u, r, c, piv, W.row_bits(w), om, xs.q, xs.k, xs.v,
                                          O.gate_rows(xs.gate, w.kind, D), xs.beta)
     ug, rg, cg, pg = T.read_pool_state(pool, L, [W.slot_of_request(b) for b in sample])
-    T.compare_codes(ug, u2, X, r2, c2, W.row_bits(w), "full-size decode")
+    n = T.compare_codes(ug, u2, X, r2, c2, W.row_bits(w), "full-size decode", config=w.name)
+    T.check_scales(rg, r2, cg, c2, n, "full-size decode")
     assert T.per_vector_rel_l2(out[sample].cpu().numpy(), o).max() <= T.OUT_REL_L2
     assert torch.isfinite(out).all()
+
+
+@pytest.mark.parametrize("widx", [3, 4])
+def test_full_size_chained(widx):
+    """64 chained steps of the full-B launch; the 8 sampled requests run on their own
+    on both sides from one packed start: every step's readout and the final
+    dequantised states are compared with the oracle's chains."""
+    w = W.WORKLOADS[widx]
+    steps = 64
+    pool, L, om = make_pool(w)
+    rb = W.row_bits(w)
+    sample = [int(b) for b in W.parity_sample(w, 8)]
+    start = _full_size_start(w, pool, L, sample)
+    chains = T.oracle_chains(widx, sample, start, 0, steps)
+    gen = torch.Generator(device="cuda").manual_seed(199 + widx)
+    all_slots = slots_t(range(w.B))
+    out = torch.empty((w.B, w.H, D), device="cuda")
+    worst_o = 0.0
+    for t in range(steps):
+        xin, _ = _full_size_inputs(w, t, sample, gen)
+        pool.decode_step(all_slots, xin["q"], xin["k"], xin["v"], xin["gate"], xin["beta"], out)
+        o_or = np.stack([ch[0][t] for ch in chains])
+        worst_o = max(worst_o, T.per_vector_rel_l2(out[sample].cpu().numpy(), o_or).max())
+    pool.check()
+    assert torch.isfinite(out).all()
+    Sg = torch.empty((len(sample), w.H, D, D), device="cuda")
+    pool.dequantize(slots_t(sample), Sg)
+    fin = [ch[1] for ch in chains]
+    S_or = np.concatenate([O.dequantize(*st, rb) for st in fin], 0)
+    rel = T.rel_l2(Sg.cpu().numpy(), S_or)
+    ug = T.read_pool_state(pool, L, [W.slot_of_request(b) for b in sample])[0]
+    u_or = np.concatenate([st[0] for st in fin], 0)
+    quant = np.broadcast_to((rb != 16)[..., None], u_or.shape)
+    T.REPORTS[f"{w.name} 64 chained steps, 8 sampled requests"] = (
+        f"state rel L2 {rel:.3g}, worst readout rel L2 {worst_o:.3g}, "
+        f"final codes differing {int(((ug != u_or) & quant).sum())} of {int(quant.sum())}")
+    assert rel <= T.CHAIN_REL_L2
+    assert worst_o <= T.OUT_REL_L2
 
 
 # ---------------------------------------------------------------------------------
@@ -263,7 +308,8 @@ def test_zero_state_stays_zero_and_all_pivot_kda_head():
     pool.check()
     u2, r2, c2, p2, o, X = O.decode_step(u, r, c, piv, rb, om, k, k, v, gate, beta)
     ug, rg, cg, pg = T.read_pool_state(pool, L, [1])
-    T.compare_codes(ug, u2, X, r2, c2, rb, "pivot head")
+    n = T.compare_codes(ug, u2, X, r2, c2, rb, "pivot head", config="kda_all_pivot_head")
+    T.check_scales(rg, r2, cg, c2, n, "pivot head")
     assert np.array_equal(pg[:, rb == 16], p2[:, rb == 16])
     assert T.per_vector_rel_l2(out.cpu().numpy(), o).max() <= T.OUT_REL_L2
 
@@ -291,6 +337,44 @@ def test_host_entry_point_matches_device_entry_point():
     assert torch.equal(h_out, out_dev.cpu())
 
 
+@pytest.mark.parametrize("widx", [1, 2])
+def test_pipelined_host_steps_match_serial_host_steps(widx):
+    """The pipelined host-buffer steps (copies overlapping the neighbouring steps inside
+    the library) give bit for bit the readouts and states of stq_decode_step_host."""
+    w = W.WORKLOADS[widx]
+    reqs = [0, 1, 2, 3, 4]
+    steps = 4
+    pool, L, _ = make_pool(w)
+    S0, u, r, c, piv = oracle_quantised(w, reqs)
+    slots = [W.slot_of_request(b) for b in reqs]
+    st = slots_t(reqs)
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    xs = [[pin(getattr(T.inputs_for(w, "decode", t, reqs), n)) for n in ("q", "k", "v", "gate", "beta")]
+          for t in range(steps)]
+    T.write_oracle_state(pool, L, slots, u, r, c, piv)
+    staging = torch.empty(pool.host_staging_bytes(len(reqs)), dtype=torch.uint8, device="cuda")
+    ref = []
+    for x in xs:
+        h_out = torch.empty((len(reqs), w.H, D)).pin_memory()
+        pool.decode_step_host(st, *x, h_out, staging)
+        torch.cuda.synchronize()
+        ref.append(h_out)
+    pool.check()
+    codes_ref, scales_ref = pool.codes.clone(), pool.scales.clone()
+    T.write_oracle_state(pool, L, slots, u, r, c, piv)
+    pipe = pool.pipeline(len(reqs))
+    outs = [torch.full((len(reqs), w.H, D), float("nan")).pin_memory() for _ in range(steps)]
+    for t, x in enumerate(xs):
+        pipe.step(st, *x, outs[t])
+        if t >= 1:      # on return the previous step's readout is on the host
+            assert torch.equal(outs[t - 1], ref[t - 1]), f"step {t - 1}"
+    pipe.finish()
+    assert torch.equal(outs[-1], ref[-1])
+    pipe.close()
+    pool.check()
+    assert torch.equal(pool.codes, codes_ref) and torch.equal(pool.scales, scales_ref)
+
+
 # ---------------------------------------------------------------------------------
 # the uniform baseline scheme: symmetric per-key-row absmax (same kernels, other
 # quantiser)
@@ -311,7 +395,7 @@ def test_absmax_quantize_init_matches_oracle(widx, bits):
     pool.quantize_init(slots_t(reqs), dev(S0))
     pool.check()
     ug, rg, cg, pg = T.read_pool_state(pool, L, [W.slot_of_request(b) for b in reqs])
-    T.compare_codes(ug, u, S0, r, c, rb, "absmax quantize_init")
+    T.compare_codes(ug, u, S0, r, c, rb, "absmax quantize_init", config=f"{w.name} row_absmax")
     assert np.array_equal(rg, r) and np.array_equal(cg, c)
     assert np.array_equal(pg[:, rb == 16], piv[:, rb == 16])
 
@@ -332,7 +416,7 @@ def test_absmax_decode_step_teacher_forced(widx, t, bits):
     pool.decode_step(slots_t(reqs), dev(x.q), dev(x.k), dev(x.v), dev(x.gate), dev(x.beta), out)
     pool.check()
     ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
-    T.compare_codes(ug, u2, X, r2, c2, rb, f"absmax {w.name} step {t}")
+    T.compare_codes(ug, u2, X, r2, c2, rb, f"absmax {w.name} step {t}", config=f"{w.name} row_absmax")
     assert np.array_equal(rg, r2) and np.array_equal(cg, c2)
     assert np.array_equal(pg[:, rb == 16], p2[:, rb == 16])
     assert T.per_vector_rel_l2(out.cpu().numpy(), o).max() <= T.OUT_REL_L2
@@ -385,8 +469,8 @@ def test_scale16_quantize_step_and_chain(widx, scheme):
     pool.quantize_init(slots_t(reqs), dev(S0))
     pool.check()
     ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
-    if T.compare_codes(ug, u, S0, r, c, rb, "scale16 quantize_init") == 0:
-        assert np.array_equal(rg, r) and np.array_equal(cg, c)
+    n = T.compare_codes(ug, u, S0, r, c, rb, "scale16 quantize_init", config=f"{w.name} {scheme} scale16")
+    T.check_scales(rg, r, cg, c, n, "scale16 quantize_init", c_rel=2.0 ** -10)
     # chained steps from the oracle's packed state
     T.write_oracle_state(pool, L, slots, u, r, c, piv)
     out = torch.empty((len(reqs), w.H, D), device="cuda")
@@ -399,8 +483,8 @@ def test_scale16_quantize_step_and_chain(widx, scheme):
         assert T.per_vector_rel_l2(out.cpu().numpy(), o).max() <= T.OUT_REL_L2, f"step {t}"
         if t == 0:     # teacher-forced first step: the step rule itself
             ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
-            if T.compare_codes(ug, u2, X, r2, c2, rb, "scale16 step") == 0:
-                assert np.array_equal(rg, r2) and np.array_equal(cg, c2)
+            n = T.compare_codes(ug, u2, X, r2, c2, rb, "scale16 step", config=f"{w.name} {scheme} scale16")
+            T.check_scales(rg, r2, cg, c2, n, "scale16 step", c_rel=2.0 ** -10)
         u, r, c, piv = u2, r2, c2, p2
     pool.check()
     ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
@@ -430,8 +514,8 @@ def test_uniform_width_paths_step(widx, bits):
     pool.quantize_init(torch.tensor(slots, dtype=torch.int32, device="cuda"), dev(S0))
     pool.check()
     ug, rg, cg, _ = T.read_pool_state(pool, L, slots)
-    if T.compare_codes(ug, u, S0, r, c, rb, f"{bits}-bit quantize") == 0:
-        assert np.array_equal(rg, r) and np.array_equal(cg, c)
+    n = T.compare_codes(ug, u, S0, r, c, rb, f"{bits}-bit quantize", config=f"{w.kind} uniform {bits}-bit")
+    T.check_scales(rg, r, cg, c, n, f"{bits}-bit quantize")
     T.write_oracle_state(pool, L, slots, u, r, c, piv)
     x = T.inputs_for(w, "decode", 3, reqs)
     u2, r2, c2, p2, o, X = O.decode_step(u, r, c, piv, rb, om, x.q, x.k, x.v,
@@ -441,8 +525,8 @@ def test_uniform_width_paths_step(widx, bits):
                      dev(x.gate), dev(x.beta), out)
     pool.check()
     ug, rg, cg, _ = T.read_pool_state(pool, L, slots)
-    if T.compare_codes(ug, u2, X, r2, c2, rb, f"{bits}-bit step") == 0:
-        assert np.array_equal(rg, r2) and np.array_equal(cg, c2)
+    n = T.compare_codes(ug, u2, X, r2, c2, rb, f"{bits}-bit step", config=f"{w.kind} uniform {bits}-bit")
+    T.check_scales(rg, r2, cg, c2, n, f"{bits}-bit step")
     assert T.per_vector_rel_l2(out.cpu().numpy(), o).max() <= T.OUT_REL_L2
 
 
@@ -480,8 +564,8 @@ def test_degenerate_rows_and_columns(widx, scheme):
     pool.quantize_init(slots_t(reqs), dev(S0))
     pool.check()
     ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
-    if T.compare_codes(ug, u, S0, r, c, rb, "degenerate quantize_init") == 0:
-        assert np.array_equal(rg, r) and np.array_equal(cg, c)
+    n = T.compare_codes(ug, u, S0, r, c, rb, "degenerate quantize_init", config=f"{w.kind} degenerate {scheme}")
+    T.check_scales(rg, r, cg, c, n, "degenerate quantize_init")
     piv_rows = rb == 16
     assert np.array_equal(pg[:, piv_rows], piv[:, piv_rows])
     # one step from the oracle's packed state; k_i = 0 keeps the zero rows zero and
@@ -499,7 +583,7 @@ def test_degenerate_rows_and_columns(widx, scheme):
     pool.decode_step(slots_t(reqs), dev(x.q), dev(k), dev(v), dev(x.gate), dev(x.beta), out)
     pool.check()
     ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
-    if T.compare_codes(ug, u2, X, r2, c2, rb, "degenerate step") == 0:
-        assert np.array_equal(rg, r2) and np.array_equal(cg, c2)
+    n = T.compare_codes(ug, u2, X, r2, c2, rb, "degenerate step", config=f"{w.kind} degenerate {scheme}")
+    T.check_scales(rg, r2, cg, c2, n, "degenerate step")
     assert np.array_equal(pg[:, piv_rows], p2[:, piv_rows])
     assert T.per_vector_rel_l2(out.cpu().numpy(), o).max() <= T.OUT_REL_L2

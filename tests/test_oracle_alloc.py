@@ -123,3 +123,57 @@ def test_distortion_shrinks_with_width():
         e = A.row_sq_error(S, O.dequantize(u, r, c, piv, rb))
         ds.append(A.unit_distortion("gdn", e, om)[0])
     assert ds[0] > ds[1] > ds[2] > ds[3] > 0
+
+
+def _mixed_head_state(seed, H=3, N=2):
+    rng = np.random.default_rng(seed)
+    S = (rng.standard_normal((N, H, 128, 128)) * rng.lognormal(0, 1, (N, H, 128, 1))
+         * rng.lognormal(0, 0.5, (N, H, 1, 128))).astype(F32)
+    om = rng.lognormal(0, 1, (H, 128)).astype(F32)
+    rb = rng.choice([2, 4, 6, 8], size=(H, 128))
+    rb[0, 5] = 16                                   # a pivot row
+    return S, om, rb
+
+
+def test_in_head_error_at_own_width_is_the_pools_error():
+    # a row's in-head error at the width it has in the pool is its reconstruction error
+    # in that pool (refit, dequantise, row error: each pinned on its own)
+    S, om, rb = _mixed_head_state(1)
+    u, r, c, piv = O.refit(S, om, rb)
+    cand = (2, 4, 6, 8)
+    e = A.row_error_at_widths(S, c, om, cand)
+    own = A.row_sq_error(S, O.dequantize(u, r, c, piv, rb))
+    quant = rb != 16
+    for k, b in enumerate(cand):
+        sel = np.broadcast_to((rb == b)[None], own.shape)
+        assert np.array_equal(e[..., k][sel], own[sel])
+    assert quant.sum() < rb.size
+
+
+def test_in_head_error_never_grows_with_width_and_stops_at_full_reach():
+    S, om, rb = _mixed_head_state(2)
+    _, r, c, _ = O.refit(S, om, rb)
+    cand = (2, 4, 6, 8)
+    e = A.row_error_at_widths(S, c, om, cand).astype(np.float64)
+    assert np.all(np.diff(e, axis=-1) <= 1e-6 * e[..., :1])
+    # a row none of whose codes reaches +-qmax_b at width b gains nothing from more bits:
+    # the codes are rint of the same exact quotients
+    rr = (A.tree_sum(np.abs(S), axis=-1) * F32(1 / 128) * O.row_gain(om)).astype(F32)
+    y = (S * O._recip(rr)[..., :, None]).astype(F32)
+    x = np.abs(y.astype(np.float64) * O._recip(c).astype(np.float64)[..., None, :]).max(axis=-1)
+    fits = x < 31.5                                  # within reach at 6 bits
+    assert fits.any()
+    assert np.array_equal(e[..., 2][fits], e[..., 3][fits])
+
+
+def test_in_head_error_of_a_uniform_head_matches_uniform_measure_at_its_width():
+    # in a head of one width the in-head error at that width is the uniform-width
+    # distortion measure the first allocation uses
+    rng = np.random.default_rng(3)
+    S = (rng.standard_normal((2, 2, 128, 128)) * rng.lognormal(0, 1, (2, 2, 128, 1))).astype(F32)
+    om = rng.lognormal(0, 1, (2, 128)).astype(F32)
+    for b in (2, 4, 6, 8):
+        rb = np.full((2, 128), b)
+        u, r, c, piv = O.refit(S, om, rb)
+        e = A.row_error_at_widths(S, c, om, (b,))[..., 0]
+        assert np.array_equal(e, A.row_sq_error(S, O.dequantize(u, r, c, piv, rb)))
