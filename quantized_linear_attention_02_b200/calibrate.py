@@ -84,17 +84,21 @@ def in_head_distortions(kind, omega, states, unit_bits, cand_bits, stream=None):
 
 
 def allocate_in_head(kind, omega, states, ell_units, budget, pivot_frac=0.02, horizon=1024, rounds=3,
-                     cand_bits=None):
+                     cand_bits=None, start="allocated"):
     """allocate(), then for per-row widths (KDA) up to `rounds` re-allocations on the
     rows' in-head distortions under the previous allocation (a row's width sets only the
     reach of its codes when its head shares column scales), stopping when no width
-    changes. GDN heads have one width each, so the uniform-width distortions are already
-    in-head ones and the first allocation stands. Returns (unit_bits, details)."""
+    changes. start="uniform" takes the first in-head distortions under a pool of the
+    budget width instead of under allocate()'s widths. GDN heads have one width each, so
+    the uniform-width distortions are already in-head ones and the first allocation
+    stands. Returns (unit_bits, details)."""
     bits, info = allocate(kind, omega, states, ell_units, budget, pivot_frac, horizon, cand_bits)
     info["rounds"] = 0
     if kind == "gdn":
         return bits, info
     cand = info["candidates"]
+    if start == "uniform":
+        bits = np.full_like(bits, int(budget))
     for k in range(rounds):
         dist = in_head_distortions(kind, omega, states, bits, cand)
         new = stq.allocate_bits(info["lifetime"], dist, cand, budget, info["n_pivots"])
@@ -136,18 +140,20 @@ def main():
     ap.add_argument("--eval-sequences", type=int, default=4)
     ap.add_argument("--in-head-rounds", type=int, default=3,
                     help="re-allocations of per-row (KDA) widths on in-head distortions (0: none)")
+    ap.add_argument("--in-head-start", choices=["allocated", "uniform"], default="allocated",
+                    help="pool whose column scales the first in-head distortions are taken under")
     a = ap.parse_args()
     build.build()
     w = W.WORKLOADS[a.workload]
     om = W.omega(w)
     S = calibration_states(w, a.sequences, a.calib_steps)
     bits, info = allocate_in_head(w.kind, om, S, W.calibration_log_retention(w), a.budget,
-                                  rounds=a.in_head_rounds)
+                                  rounds=a.in_head_rounds, start=a.in_head_start)
     del S
     hist = {str(b): int((bits == b).sum()) for b in sorted(set(bits.tolist()))}
     res = {"workload": w.name, "budget": a.budget, "calibration": f"{a.sequences} sequences x {a.calib_steps} steps",
            "evaluation": f"{a.eval_sequences} other sequences x {a.eval_steps} steps",
-           "in_head_rounds": info["rounds"],
+           "in_head_rounds": info["rounds"], "in_head_start": a.in_head_start,
            "widths": hist, "mean_bits_non_pivot": float(bits[bits != 16].mean()),
            "mean_bits_with_pivots": float(bits.mean())}
     uniform = np.full_like(bits, a.budget)
