@@ -84,12 +84,13 @@ def in_head_distortions(kind, omega, states, unit_bits, cand_bits, stream=None):
 
 
 def allocate_in_head(kind, omega, states, ell_units, budget, pivot_frac=0.02, horizon=1024, rounds=3,
-                     cand_bits=None, start="allocated"):
+                     cand_bits=None, start="uniform"):
     """allocate(), then for per-row widths (KDA) up to `rounds` re-allocations on the
     rows' in-head distortions under the previous allocation (a row's width sets only the
     reach of its codes when its head shares column scales), stopping when no width
-    changes. start="uniform" takes the first in-head distortions under a pool of the
-    budget width instead of under allocate()'s widths. GDN heads have one width each, so
+    changes. The first in-head distortions are taken under a pool of the budget width
+    (start="uniform", which reaches the better widths) or under allocate()'s widths
+    (start="allocated"). GDN heads have one width each, so
     the uniform-width distortions are already in-head ones and the first allocation
     stands. Returns (unit_bits, details)."""
     bits, info = allocate(kind, omega, states, ell_units, budget, pivot_frac, horizon, cand_bits)
@@ -140,7 +141,7 @@ def main():
     ap.add_argument("--eval-sequences", type=int, default=4)
     ap.add_argument("--in-head-rounds", type=int, default=3,
                     help="re-allocations of per-row (KDA) widths on in-head distortions (0: none)")
-    ap.add_argument("--in-head-start", choices=["allocated", "uniform"], default="allocated",
+    ap.add_argument("--in-head-start", choices=["allocated", "uniform"], default="uniform",
                     help="pool whose column scales the first in-head distortions are taken under")
     a = ap.parse_args()
     build.build()

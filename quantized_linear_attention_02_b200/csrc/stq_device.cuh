@@ -316,7 +316,8 @@ struct __align__(16) WarpRows {
   float qm[RPW], iq[RPW], mb[RPW];   // per-row width constants (mixed heads)
   uint4 rk[RPW];                   // mixed heads, unpack of row i (width b, pivot rows 0):
                                    //   {M = 2^b - 1, M << b, exponent bits of a code at
-                                   //   bit b, 4b | 2b << 8}
+                                   //   bit b, 4b | 2b << 8 | byte offset of the row in the
+                                   //   warp's codes << 16}
   f2 roff[RPW];                    // -(2^23 + 2^(b-1)), -(2^(23-b) + 2^(b-1))
   f2 clampb[RPW];                  // least-squares clamp: 1.5*2^23 -+ qmax
   uint32_t info[RPW];              // bits | offset << 8
@@ -392,9 +393,10 @@ __device__ __forceinline__ void width_consts(int bits, float& qm, float& iq, flo
   }
 }
 
-// Lane l < 16 of a warp: every per-row constant of its row (width `bits`) that the
-// mixed-width paths read.
-__device__ __forceinline__ void mixed_row_consts(WarpRows& wr, int l, int bits) {
+// Lane l < 16 of a warp: every per-row constant of its row (width `bits`, codes at byte
+// `code_off` of the warp's codes) that the mixed-width paths read. A pivot row gets zero
+// unpack constants and offset 0, so that it can run the code path harmlessly.
+__device__ __forceinline__ void mixed_row_consts(WarpRows& wr, int l, int bits, uint32_t code_off) {
   float qm, iq, mb;
   width_consts(bits, qm, iq, mb);
   wr.qm[l] = qm; wr.iq[l] = iq; wr.mb[l] = mb;
@@ -405,7 +407,8 @@ __device__ __forceinline__ void mixed_row_consts(WarpRows& wr, int l, int bits) 
   } else {
     const uint32_t M = (1u << bits) - 1u;
     const float bias = float(1 << (bits - 1));
-    wr.rk[l] = make_uint4(M, M << bits, uint32_t(150 - bits) << 23, uint32_t(4 * bits) | (uint32_t(2 * bits) << 8));
+    wr.rk[l] = make_uint4(M, M << bits, uint32_t(150 - bits) << 23,
+                          uint32_t(4 * bits) | (uint32_t(2 * bits) << 8) | (code_off << 16));
     wr.roff[l] = make_float2(-(8388608.0f + bias), -(float(1u << (23 - bits)) + bias));
   }
 }
@@ -421,7 +424,7 @@ __device__ __forceinline__ void load_warp_rows(const PoolDev& P, int h, WarpRows
     wr.info[lane] = info;
     wr.g[lane] = P.g[h * D + i];
     wr.om[lane] = P.omega[h * D + i];
-    mixed_row_consts(wr, lane, row_bits(info));
+    mixed_row_consts(wr, lane, row_bits(info), uint32_t(row_off(info)) - P.warp_code_off[h * NW + r0 / RPW]);
     if (k_vec != nullptr) {
       const float dec = gate_rows != nullptr ? gate_rows[i] : gate_s;
       const float kv = k_vec[i], qv = q_vec[i];
@@ -466,34 +469,27 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
 #pragma unroll
   for (int rr = 0; rr < RPW; ++rr) {
     if constexpr (BITS == MIXED) {
-      const uint32_t info = wr.info[rr];
-      if (row_bits(info) != PIVOT) {
-        // any width b: the lane's 4b bits start at bit 4 b l of the row (the word after them
-        // is inside the staging area: the next row, the other buffer or `tail`); codes 0
-        // and 2 sit at bit 0 of f and fh, codes 1 and 3 at bit b, each unpacked in place
-        // into a float's mantissa (2^23 + u, 2^(23-b) + u)
-        const uint4 K = wr.rk[rr];
-        const f2 off = wr.roff[rr];
-        const uint32_t* wp = reinterpret_cast<const uint32_t*>(wcodes + (row_off(info) - warp_code_start));
-        const int bitpos = int(K.w & 0xFFu) * lane;
-        const uint32_t f = __funnelshift_r(wp[bitpos >> 5], wp[(bitpos >> 5) + 1], bitpos & 31);
-        const uint32_t fh = f >> (K.w >> 8);
+      // any width b: the lane's 4b bits start at bit 4 b l of the row (the word after them
+      // is inside the staging area: the next row, the other buffer or `tail`); codes 0
+      // and 2 sit at bit 0 of f and fh, codes 1 and 3 at bit b, each unpacked in place
+      // into a float's mantissa (2^23 + u, 2^(23-b) + u). Every row runs this path: a
+      // pivot row's zero constants and zero stored row scale make it 0 here, and the
+      // fix-up after the loop replaces it.
+      const uint4 K = wr.rk[rr];
+      const f2 off = wr.roff[rr];
+      const uint32_t* wp = reinterpret_cast<const uint32_t*>(wcodes + (K.w >> 16));
+      const int bitpos = int(K.w & 0xFFu) * lane;
+      const uint32_t f = __funnelshift_r(wp[bitpos >> 5], wp[(bitpos >> 5) + 1], bitpos & 31);
+      const uint32_t fh = f >> ((K.w >> 8) & 0xFFu);
 #ifdef STQ_CHECKS
-        zero_code |= (f & K.x) == 0 || (f & K.y) == 0 || (fh & K.x) == 0 || (fh & K.y) == 0;
+      zero_code |= row_bits(wr.info[rr]) != PIVOT &&
+                   ((f & K.x) == 0 || (f & K.y) == 0 || (fh & K.x) == 0 || (fh & K.y) == 0);
 #endif
-        const f2 q01 = add2(make_float2(__uint_as_float((f & K.x) | FLOAT_2P23), __uint_as_float((f & K.y) | K.z)), off);
-        const f2 q23 = add2(make_float2(__uint_as_float((fh & K.x) | FLOAT_2P23), __uint_as_float((fh & K.y) | K.z)), off);
-        const f2 rd = dup(wr.rdd[rr].x);
-        s[rr][0] = mul2(mul2(q01, rd), cin[0]);
-        s[rr][1] = mul2(mul2(q23, rd), cin[1]);
-      } else {
-        const uint2 hv = *reinterpret_cast<const uint2*>(hr.pivots + row_off(info) * D + 4 * lane);
-        f2 x, y;
-        half4_floats(hv, x, y);
-        const f2 dd = dup(wr.dec[rr]);
-        s[rr][0] = mul2(dd, x);
-        s[rr][1] = mul2(dd, y);
-      }
+      const f2 q01 = add2(make_float2(__uint_as_float((f & K.x) | FLOAT_2P23), __uint_as_float((f & K.y) | K.z)), off);
+      const f2 q23 = add2(make_float2(__uint_as_float((fh & K.x) | FLOAT_2P23), __uint_as_float((fh & K.y) | K.z)), off);
+      const f2 rd = dup(wr.rdd[rr].x);
+      s[rr][0] = mul2(mul2(q01, rd), cin[0]);
+      s[rr][1] = mul2(mul2(q23, rd), cin[1]);
     } else {
       uint32_t cd[4];
       load_codes<BITS>(wcodes + rr * (D * BITS / 8), lane, cd);
@@ -508,6 +504,21 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
       codes_to_q<BITS>(cd, q01, q23);
       s[rr][0] = mul2(mul2(q01, rd), cin[0]);
       s[rr][1] = mul2(mul2(q23, rd), cin[1]);
+    }
+  }
+  if (BITS == MIXED && hr.piv_count) {
+    // FP16 pivot rows: S' = D h
+#pragma unroll
+    for (int rr = 0; rr < RPW; ++rr) {
+      const uint32_t info = wr.info[rr];
+      if (row_bits(info) == PIVOT) {
+        const uint2 hv = *reinterpret_cast<const uint2*>(hr.pivots + row_off(info) * D + 4 * lane);
+        f2 x, y;
+        half4_floats(hv, x, y);
+        const f2 dd = dup(wr.dec[rr]);
+        s[rr][0] = mul2(dd, x);
+        s[rr][1] = mul2(dd, y);
+      }
     }
   }
   {
@@ -553,7 +564,7 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
     }
     put_partial(cs.red[1][0], w, lane, add2(o[0][0], o[1][0]), add2(o[0][1], o[1][1]));
   }
-  if constexpr (BITS == MIXED) {
+  if (BITS == MIXED && hr.piv_count) {
     // pivot rows: store float16(S) now (they take no part in the refit)
 #pragma unroll
     for (int rr = 0; rr < RPW; ++rr) {
@@ -752,7 +763,7 @@ decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* 
       wr.info[lane] = info;
       wr.g[lane] = raw.g[lane];
       wr.om[lane] = raw.om[lane];
-      if constexpr (kMixed) mixed_row_consts(wr, lane, row_bits(info));
+      if constexpr (kMixed) mixed_row_consts(wr, lane, row_bits(info), uint32_t(row_off(info)) - rec.y);
       const float dec = (P.kind == 0) ? raw.gate_s : raw.gate[lane];
       float r_in;
       if constexpr (H16) r_in = __half2float(reinterpret_cast<const __half*>(raw.r)[lane]);
@@ -775,6 +786,8 @@ decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* 
       cin[1] = make_float2(c4.z, c4.w);
     }
     const float v_own = raw.v[lane & 15];
+    // this warp's pivot rows (warp-uniform): mixed-width warps without any skip the fix-ups
+    const int npiv = __popc(__ballot_sync(0xffffffffu, lane < RPW && row_bits(raw.info[lane]) == PIVOT));
     int hn = h + dh, bn = bq + db;
     if (bn >= B) { bn -= B; ++hn; }
     if (hn < P.H) {
@@ -794,7 +807,7 @@ decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* 
       hr.sc.p = static_cast<uint8_t*>(P.scales) + (uint64_t(slot) * P.H + h) * 2 * D * (H16 ? 2 : 4);
       hr.bits = int(rec.w & 0xFFu);
       hr.code_bytes = 0;     // not used by the decode step
-      hr.piv_count = 0;
+      hr.piv_count = npiv;   // pivot rows among this warp's rows
       hr.piv_stage_off = 0;
       const int wstart = int(rec.y);
       uint8_t* wcodes = wr.codes[cur];
