@@ -135,3 +135,19 @@ def test_null_arguments(lib):
     lib.stq_pool_destroy(None)
     assert lib.stq_fp32_decode_step(3, 1, 1, 128, None, None, None, None, None, None, None, None) == 1
     assert lib.stq_fp32_decode_step(0, 1, 1, 64, None, None, None, None, None, None, None, None) == 1
+
+
+def test_pipeline_and_in_head_error_reject_bad_arguments_without_a_gpu(lib):
+    # argument checks come before any CUDA call, so they run here
+    vp = ctypes.c_void_p
+    assert lib.stq_pipeline_staging_bytes(None, 4) == 0
+    out = vp(123)
+    st = lib.stq_pipeline_create(None, 4, vp(16), ctypes.c_size_t(1 << 20), ctypes.byref(out))
+    assert st == 1 and out.value is None and lib.stq_last_error()
+    st = lib.stq_pipeline_step(None, vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), None)
+    assert st == 1 and b"pipeline" in lib.stq_last_error()
+    assert lib.stq_pipeline_finish(None, None) == 1
+    lib.stq_pipeline_destroy(None)                       # NULL is ignored
+    cand = (ctypes.c_int * 1)(6)
+    st = lib.stq_row_error_at_widths(None, vp(16), 1, vp(16), ctypes.cast(cand, vp), 1, vp(16), None)
+    assert st == 1 and b"pool" in lib.stq_last_error()
