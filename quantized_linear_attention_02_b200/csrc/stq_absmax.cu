@@ -15,46 +15,36 @@ struct AbsmaxStore {
   template <int BITS, class Sc>
   static __device__ __forceinline__ void store(CtaSmem& cs, WarpRows& wr, f2 (&s)[RPW][2], const Sc& sc,
                                                uint8_t* codes_global, int warp_code_start, float* o_global,
-                                               uint8_t* /*stage*/) {
+                                               uint8_t* stage) {
     const int w = group_tid() >> 5, lane = group_tid() & 31;
     const int r0 = w * RPW;
 
-    // --- row maxima of |S| (exact in any order): 4 columns per lane, then a
-    // reduce-scatter over the lanes that leaves row R(l) in lane l -----------------
+    // --- row maxima of |S| (exact in any order): 4 columns per lane, then across the
+    // lanes -------------------------------------------------------------------------
     float a[RPW];
 #pragma unroll
     for (int rr = 0; rr < RPW; ++rr)
       a[rr] = fmaxf(fmaxf(fabsf(s[rr][0].x), fabsf(s[rr][0].y)), fmaxf(fabsf(s[rr][1].x), fabsf(s[rr][1].y)));
+    // through the warp's consumed code staging area, as the refit's row sums: lane l
+    // writes its 16 row maxima at tr[rr][l ^ 4 (rr & 7)], lane L takes row L & 15 over
+    // lanes 16 (L >> 4) .. +15, and the two halves meet in one shuffle
+    float* tr = reinterpret_cast<float*>(stage);
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const bool up = lane & 1;
-      const float send = up ? a[t] : a[t + 8];
-      const float keep = up ? a[t + 8] : a[t];
-      a[t] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 1));
-    }
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const bool up = lane & 2;
-      const float send = up ? a[t] : a[t + 4];
-      const float keep = up ? a[t + 4] : a[t];
-      a[t] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
-    }
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const bool up = lane & 4;
-      const float send = up ? a[t] : a[t + 2];
-      const float keep = up ? a[t + 2] : a[t];
-      a[t] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 4));
-    }
+    for (int rr = 0; rr < RPW; ++rr) tr[rr * 32 + (lane ^ (4 * (rr & 7)))] = a[rr];
+    __syncwarp();
     {
-      const bool up = lane & 8;
-      const float send = up ? a[0] : a[1];
-      const float keep = up ? a[1] : a[0];
-      a[0] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+      const int Rr = lane & 15, hh = lane >> 4;
+      float m = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 v = *reinterpret_cast<const float4*>(tr + Rr * 32 + ((16 * hh + 4 * j) ^ (4 * (Rr & 7))));
+        m = fmaxf(m, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+      }
+      a[0] = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
     }
-    a[0] = fmaxf(a[0], __shfl_xor_sync(0xffffffffu, a[0], 16));
+    __syncwarp();   // the staging area is free again
     {
-      const int R = ((lane & 1) << 3) | ((lane & 2) << 1) | ((lane & 4) >> 1) | ((lane & 8) >> 3);
+      const int R = lane & 15;   // lane l holds the maximum of row l & 15
       float iq;
       bool pivot = false;
       if constexpr (BITS == MIXED) {

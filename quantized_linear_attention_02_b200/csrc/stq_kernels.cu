@@ -54,38 +54,33 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
 #pragma unroll
   for (int rr = 0; rr < RPW; ++rr)
     a[rr] = fadd(fadd(fabsf(s[rr][0].x), fabsf(s[rr][0].y)), fadd(fabsf(s[rr][1].x), fabsf(s[rr][1].y)));
-  // reduce-scatter over lanes: step m keeps half of the rows and pairs lane l with l^m
+  // Row sums through the warp's consumed code staging area: lane l writes its 16 row
+  // partials at tr[rr][l ^ 4 (rr & 7)] (the swizzle keeps every group of 4 lanes whole and
+  // spreads the rows over the banks); lane L then adds row L & 15 over lanes 16 (L >> 4)
+  // .. +15 as a balanced tree, and the two halves meet in one shuffle: the same tree over
+  // the 128 columns as lane pairs xor 1, 2, 4, 8, 16 would make.
+  float* tr = reinterpret_cast<float*>(stage);
 #pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    const bool up = lane & 1;
-    const float send = up ? a[t] : a[t + 8];
-    const float keep = up ? a[t + 8] : a[t];
-    a[t] = fadd(keep, __shfl_xor_sync(0xffffffffu, send, 1));
-  }
-#pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    const bool up = lane & 2;
-    const float send = up ? a[t] : a[t + 4];
-    const float keep = up ? a[t + 4] : a[t];
-    a[t] = fadd(keep, __shfl_xor_sync(0xffffffffu, send, 2));
-  }
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const bool up = lane & 4;
-    const float send = up ? a[t] : a[t + 2];
-    const float keep = up ? a[t + 2] : a[t];
-    a[t] = fadd(keep, __shfl_xor_sync(0xffffffffu, send, 4));
-  }
+  for (int rr = 0; rr < RPW; ++rr) tr[rr * 32 + (lane ^ (4 * (rr & 7)))] = a[rr];
+  __syncwarp();
   {
-    const bool up = lane & 8;
-    const float send = up ? a[0] : a[1];
-    const float keep = up ? a[1] : a[0];
-    a[0] = fadd(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+    const int Rr = lane & 15, hh = lane >> 4;
+    float p[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 v = *reinterpret_cast<const float4*>(tr + Rr * 32 + ((16 * hh + 4 * j) ^ (4 * (Rr & 7))));
+      p[4 * j] = v.x; p[4 * j + 1] = v.y; p[4 * j + 2] = v.z; p[4 * j + 3] = v.w;
+    }
+#pragma unroll
+    for (int m = 1; m < 16; m <<= 1)
+#pragma unroll
+      for (int t = 0; t < 16; t += 2 * m) p[t] = fadd(p[t], p[t + m]);
+    a[0] = fadd(p[0], __shfl_xor_sync(0xffffffffu, p[0], 16));
   }
-  a[0] = fadd(a[0], __shfl_xor_sync(0xffffffffu, a[0], 16));
+  __syncwarp();   // the staging area is free again
   {
-    // lane l now holds the sum of row R(l): bits 0..3 of l chose halves 8, 4, 2, 1
-    const int R = ((lane & 1) << 3) | ((lane & 2) << 1) | ((lane & 4) >> 1) | ((lane & 8) >> 3);
+    // lane l holds the sum of row l & 15
+    const int R = lane & 15;
     const bool pivot = (BITS == MIXED) ? (row_bits(wr.info[R]) == PIVOT) : false;
     // a compact pool rounds r to binary16 here: y, the weights and the codes use it
     const float r = sc.stored(pivot ? 0.0f : fmul(fmul(a[0], 0.0078125f), wr.g[R]));
