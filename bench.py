@@ -45,8 +45,8 @@ FP32_LANES_PER_SM = 128
 # ncu dram bytes (read + write) per launch of decode_kernel on the default workload
 # (GDN B = 512, dual-axis refit), and the sha256 of the kernel sources they were taken
 # with (a changed kernel voids them).
-TRAFFIC = {"bytes": 2 * (193_588_224 + 125_869_056),
-           "kernel_sha256": "2ad6efd24633b532a10e2838cd245eb107475318a261dfa4a3b9781e371c0814",
+TRAFFIC = {"bytes": 2 * (193_409_536 + 126_277_376),
+           "kernel_sha256": "859456e5c98609cf3d04375811fdc9abaebdd35d0cde1f0058f6f013640a3e45",
            "source": "profiles/decode_kernel_gdn_b256_h48_nominal6.md: dram read + write of one "
                      "B = 256 launch, doubled for B = 512 (traffic grows with B)"}
 

@@ -318,7 +318,11 @@ struct __align__(16) WarpRows {
                                    //   {M = 2^b - 1, M << b, exponent bits of a code at
                                    //   bit b, 4b | 2b << 8 | byte offset of the row in the
                                    //   warp's codes << 16}
-  f2 roff[RPW];                    // -(2^23 + 2^(b-1)), -(2^(23-b) + 2^(b-1))
+  float4 rp[RPW];                  // restore of row i: -(2^23 + 2^(b-1)), -(2^(23-b) +
+                                   //   2^(b-1)), dec_i r_i, 0 (pivot rows: 0, 0, dec_i r_i, 0)
+  uint4 st[RPW];                   // final codes of row i: {bits of 1.5*2^23 + 2^(b-1),
+                                   //   (2^b - 1) * 0x10001, 2b | row offset << 16, b}
+                                   //   (pivot rows: {.., 0, 0, 16})
   f2 clampb[RPW];                  // least-squares clamp: 1.5*2^23 -+ qmax
   uint32_t info[RPW];              // bits | offset << 8
   uint8_t codes[2][RPW * D];       // this warp's rows of packed codes: the item being
@@ -394,22 +398,26 @@ __device__ __forceinline__ void width_consts(int bits, float& qm, float& iq, flo
 }
 
 // Lane l < 16 of a warp: every per-row constant of its row (width `bits`, codes at byte
-// `code_off` of the warp's codes) that the mixed-width paths read. A pivot row gets zero
-// unpack constants and offset 0, so that it can run the code path harmlessly.
-__device__ __forceinline__ void mixed_row_consts(WarpRows& wr, int l, int bits, uint32_t code_off) {
+// `code_off` of the warp's codes, decay times stored row scale `rd`) that the mixed-width
+// paths read, packed per phase. A pivot row gets zero unpack and store constants and
+// offset 0, so that it can run the code path harmlessly.
+__device__ __forceinline__ void mixed_row_consts(WarpRows& wr, int l, int bits, uint32_t code_off, float rd) {
   float qm, iq, mb;
   width_consts(bits, qm, iq, mb);
   wr.qm[l] = qm; wr.iq[l] = iq; wr.mb[l] = mb;
   wr.clampb[l] = make_float2(MAGIC - qm, MAGIC + qm);
   if (bits == PIVOT) {
     wr.rk[l] = make_uint4(0u, 0u, 0u, 0u);
-    wr.roff[l] = make_float2(0.0f, 0.0f);
+    wr.rp[l] = make_float4(0.0f, 0.0f, rd, 0.0f);
+    wr.st[l] = make_uint4(__float_as_uint(mb), 0u, 0u, uint32_t(PIVOT));
   } else {
     const uint32_t M = (1u << bits) - 1u;
     const float bias = float(1 << (bits - 1));
     wr.rk[l] = make_uint4(M, M << bits, uint32_t(150 - bits) << 23,
                           uint32_t(4 * bits) | (uint32_t(2 * bits) << 8) | (code_off << 16));
-    wr.roff[l] = make_float2(-(8388608.0f + bias), -(float(1u << (23 - bits)) + bias));
+    wr.rp[l] = make_float4(-(8388608.0f + bias), -(float(1u << (23 - bits)) + bias), rd, 0.0f);
+    wr.st[l] = make_uint4(__float_as_uint(mb), M * 0x00010001u, uint32_t(2 * bits) | (code_off << 16),
+                          uint32_t(bits));
   }
 }
 
@@ -424,7 +432,7 @@ __device__ __forceinline__ void load_warp_rows(const PoolDev& P, int h, WarpRows
     wr.info[lane] = info;
     wr.g[lane] = P.g[h * D + i];
     wr.om[lane] = P.omega[h * D + i];
-    mixed_row_consts(wr, lane, row_bits(info), uint32_t(row_off(info)) - P.warp_code_off[h * NW + r0 / RPW]);
+    mixed_row_consts(wr, lane, row_bits(info), uint32_t(row_off(info)) - P.warp_code_off[h * NW + r0 / RPW], 0.0f);
     if (k_vec != nullptr) {
       const float dec = gate_rows != nullptr ? gate_rows[i] : gate_s;
       const float kv = k_vec[i], qv = q_vec[i];
@@ -476,7 +484,8 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
       // pivot row's zero constants and zero stored row scale make it 0 here, and the
       // fix-up after the loop replaces it.
       const uint4 K = wr.rk[rr];
-      const f2 off = wr.roff[rr];
+      const float4 P4 = wr.rp[rr];
+      const f2 off = make_float2(P4.x, P4.y);
       const uint32_t* wp = reinterpret_cast<const uint32_t*>(wcodes + (K.w >> 16));
       const int bitpos = int(K.w & 0xFFu) * lane;
       const uint32_t f = __funnelshift_r(wp[bitpos >> 5], wp[(bitpos >> 5) + 1], bitpos & 31);
@@ -487,7 +496,7 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
 #endif
       const f2 q01 = add2(make_float2(__uint_as_float((f & K.x) | FLOAT_2P23), __uint_as_float((f & K.y) | K.z)), off);
       const f2 q23 = add2(make_float2(__uint_as_float((fh & K.x) | FLOAT_2P23), __uint_as_float((fh & K.y) | K.z)), off);
-      const f2 rd = dup(wr.rdd[rr].x);
+      const f2 rd = dup(P4.z);
       s[rr][0] = mul2(mul2(q01, rd), cin[0]);
       s[rr][1] = mul2(mul2(q23, rd), cin[1]);
     } else {
@@ -763,12 +772,12 @@ decode_kernel(PoolDev P, const int32_t* __restrict__ slots, int B, const float* 
       wr.info[lane] = info;
       wr.g[lane] = raw.g[lane];
       wr.om[lane] = raw.om[lane];
-      if constexpr (kMixed) mixed_row_consts(wr, lane, row_bits(info), uint32_t(row_off(info)) - rec.y);
       const float dec = (P.kind == 0) ? raw.gate_s : raw.gate[lane];
       float r_in;
       if constexpr (H16) r_in = __half2float(reinterpret_cast<const __half*>(raw.r)[lane]);
       else r_in = __uint_as_float(raw.r[lane]);
       const float rd = fmul(dec, r_in);
+      if constexpr (kMixed) mixed_row_consts(wr, lane, row_bits(info), uint32_t(row_off(info)) - rec.y, rd);
       const float kv = raw.k[lane], qv = raw.q[lane];
       wr.dec[lane] = dec;
       wr.kk[lane] = make_float2(kv, kv);

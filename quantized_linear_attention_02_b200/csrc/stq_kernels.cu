@@ -244,21 +244,21 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
       // by now; it has the pool's layout), then copy the area out with 16-byte stores.
 #pragma unroll
       for (int rr = 0; rr < RPW; ++rr) {
-        // every row computes; a pivot row (zero unpack constants, offset 0) stores nothing
-        const int bits = row_bits(wr.info[rr]);
+        // every row computes; a pivot row (zero store constants, offset 0) stores nothing
+        const uint4 T = wr.st[rr];                     // 1.5*2^23 + bias, M * 0x10001, 2b | offset << 16, b
+        const int bits = int(T.w);
         const bool code_row = bits != PIVOT;
-        const uint4 K = wr.rk[rr];                     // M, .., .., 4b | 2b << 8 | offset << 16
-        const f2 mb = dup(wr.mb[rr]);
+        const f2 mb = dup(__uint_as_float(T.x));
         const f2 t01 = fma2(s[rr][0], ic[0], mb);
         const f2 t23 = fma2(s[rr][1], ic[1], mb);
-        const uint32_t M = K.x;
-        const uint32_t w01 = clamp_s16x2(__byte_perm(__float_as_uint(t01.x), __float_as_uint(t01.y), 0x5410), M * 0x00010001u);
-        const uint32_t w23 = clamp_s16x2(__byte_perm(__float_as_uint(t23.x), __float_as_uint(t23.y), 0x5410), M * 0x00010001u);
-        const uint32_t sh = (K.w >> 8) & 0xFFu;         // 2b (0 for a pivot row)
+        const uint32_t M = T.y & 0xFFFFu;
+        const uint32_t w01 = clamp_s16x2(__byte_perm(__float_as_uint(t01.x), __float_as_uint(t01.y), 0x5410), T.y);
+        const uint32_t w23 = clamp_s16x2(__byte_perm(__float_as_uint(t23.x), __float_as_uint(t23.y), 0x5410), T.y);
+        const uint32_t sh = T.z & 0xFFu;                // 2b (0 for a pivot row)
         const uint32_t x01 = (w01 & M) | (w01 >> (16 - (sh >> 1)));      // u0 | u1 << b
         const uint32_t x23 = (w23 & M) | (w23 >> (16 - (sh >> 1)));      // u2 | u3 << b
         const uint32_t f = x01 | (x23 << sh);
-        uint8_t* dst = stage + (K.w >> 16) + ((bits * lane) >> 1);
+        uint8_t* dst = stage + (T.z >> 16) + ((bits * lane) >> 1);
         if (code_row) dst[0] = static_cast<uint8_t>(f);
         if (code_row && bits >= 4) dst[1] = static_cast<uint8_t>(f >> 8);
         if (code_row && bits >= 6) dst[2] = static_cast<uint8_t>(f >> 16);
