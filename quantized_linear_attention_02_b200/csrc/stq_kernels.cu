@@ -6,17 +6,20 @@
 // summary, decode-order paragraph), dual-axis scales r_i c_j z_ij (bloombook section 4),
 // per-unit widths and FP16 pivot units (ai-trend review, Method).
 //
-// One CTA of 256 threads owns one (request, head) 128x128 state. Warp w holds key rows
-// 16w..16w+15, lane l holds value columns 4l..4l+3 as two float2 pairs, so a thread keeps
-// 64 state values in registers for the whole step. A row's width is uniform across a
-// warp instruction (KDA widths vary per key row without divergence); heads whose rows
-// share one width run a code path specialised for it.
+// A group of 256 threads (8 warps) owns one (request, head) 128x128 state at a time
+// (the decode kernel runs two such groups per CTA on separate items; the others one per
+// CTA). Warp w holds key rows 16w..16w+15, lane l holds value columns 4l..4l+3 as two
+// float2 pairs, so a thread keeps 64 state values in registers for the whole step. A
+// row's width is uniform across a warp instruction (KDA widths vary per key row without
+// divergence); heads whose rows share one width run a code path specialised for it.
 //
-// Float32 evaluation order (the CPU oracle restates the same order):
+// Float32 evaluation order of every sum that decides a code or a scale (the CPU oracle
+// restates the same order):
 //   * sums over the 128 rows of a column or the 128 columns of a row are balanced
 //     binary trees, adjacent pairs first. Column sums: a thread's 16 rows form the
 //     lower 4 levels, the 8 warps (shared memory) the top 3. Row sums: a thread's 4
-//     columns form the lower 2 levels, butterfly shuffle steps xor 1,2,...,16 the top 5;
+//     columns form the lower 2 levels, then 16 lanes' partials (a shared-memory
+//     transpose) the next 4 and one shuffle between the two halves of the warp the top;
 //   * in a sum of products a_i b_i each adjacent pair is one fused multiply-add,
 //     fma(a_2m, b_2m, a_2m+1 * b_2m+1); the state update is S = fma(k, delta, S'); every
 //     other product is rounded on its own (explicit _rn forms, --fmad=false);
@@ -25,9 +28,10 @@
 //     the low bits are the (biased) code; the least-squares step clamps in that binade,
 //     the final codes clamp in 16-bit lanes (same result, see refit_store).
 //
-// This file holds the dual-axis refit (the quantiser of the method), the dequantise and
-// FP32-state kernels and the launchers; the kernel bodies shared with the row-absmax
-// baseline are in stq_device.cuh.
+// The readout is compared within a tolerance, not bit for bit; each warp forms its
+// partials as running sums. This file holds the dual-axis refit (the quantiser of the
+// method), the dequantise and FP32-state kernels and the launchers; the kernel bodies
+// shared with the row-absmax baseline are in stq_device.cuh.
 #include "stq_device.cuh"
 
 namespace stq {
