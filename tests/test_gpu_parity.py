@@ -273,6 +273,48 @@ def test_bad_slot_is_flagged_and_skipped():
     assert torch.count_nonzero(out[1]) == 0                    # skipped request
 
 
+@pytest.mark.parametrize("kind,ub,B", [("gdn", (6,), 1), ("gdn", (2, 16, 8), 5), ("kda", 5, 3), ("kda", 7, 41)])
+def test_odd_item_counts(kind, ub, B):
+    """Batches whose (request, head) count is odd or smaller than the grid: each CTA of
+    the decode kernel runs two groups on alternate items, so the second group of the
+    last CTA may get none. Two teacher-forced steps on odd slot indices."""
+    rng = np.random.default_rng(B)
+    if kind == "gdn":
+        ub = np.array(ub, np.uint8)
+        H = ub.size
+        rb = np.repeat(ub[:, None], D, axis=1)
+    else:
+        H = ub
+        rb = rng.choice([2, 4, 6, 8, 16], size=(H, D), p=[0.2, 0.3, 0.2, 0.25, 0.05])
+        ub = rb.reshape(-1).astype(np.uint8)
+    om = rng.lognormal(0, 1, (H, D)).astype(F32)
+    pool = stq.Pool(kind, 2 * B + 1, ub, om)
+    L = O.Layout(rb)
+    slots = [2 * b + 1 for b in range(B)]
+    st = dev(np.array(slots, np.int32))
+    S0 = (rng.standard_normal((B, H, D, D)) * rng.lognormal(0, 1, (B, H, D, 1)) * 0.1).astype(F32)
+    u, r, c, piv = O.refit(S0, om, rb)
+    out = torch.empty((B, H, D), device="cuda")
+    for t in range(2):
+        q = rng.standard_normal((B, H, D))
+        k = rng.standard_normal((B, H, D))
+        q = (q / np.linalg.norm(q, axis=-1, keepdims=True)).astype(F32)
+        k = (k / np.linalg.norm(k, axis=-1, keepdims=True)).astype(F32)
+        v = rng.standard_normal((B, H, D)).astype(F32)
+        gate = np.exp(rng.uniform(-0.2, -0.001, (B, H) if kind == "gdn" else (B, H, D))).astype(F32)
+        beta = (1 / (1 + np.exp(-rng.standard_normal((B, H))))).astype(F32)
+        T.write_oracle_state(pool, L, slots, u, r, c, piv)
+        u, r, c, piv, o, X = O.decode_step(u, r, c, piv, rb, om, q, k, v, O.gate_rows(gate, kind, D), beta)
+        pool.decode_step(st, dev(q), dev(k), dev(v), dev(gate), dev(beta), out)
+        pool.check()
+        ug, rg, cg, pg = T.read_pool_state(pool, L, slots)
+        what = f"{kind} H={H} B={B} step {t}"
+        n = T.compare_codes(ug, u, X, r, c, rb, what, config=f"{kind} odd item counts")
+        T.check_scales(rg, r, cg, c, n, what)
+        assert np.array_equal(pg[:, rb == 16], piv[:, rb == 16])
+        assert T.per_vector_rel_l2(out.cpu().numpy(), o).max() <= T.OUT_REL_L2
+
+
 def test_empty_batch_is_a_no_op():
     w = W.WORKLOADS[0]
     pool, L, _ = make_pool(w, n_slots=2)
