@@ -90,8 +90,9 @@ __host__ __device__ constexpr float code_offset(int k) {
 }
 
 // The four codes of a lane as floats 2^(23 - pos_k) + u_k (exact), from a 16-byte
-// aligned row.
-template <int BITS>
+// aligned row. kStaged: the row sits in a warp's shared-memory staging buffer (sized for
+// 8-bit rows), so the word after a 6-bit row's last code may be read unconditionally.
+template <int BITS, bool kStaged = false>
 __device__ __forceinline__ void load_codes(const uint8_t* row, int lane, uint32_t (&c)[4]) {
   if constexpr (BITS == 8) {
     const uint32_t w = reinterpret_cast<const uint32_t*>(row)[lane];
@@ -114,7 +115,8 @@ __device__ __forceinline__ void load_codes(const uint8_t* row, int lane, uint32_
       const uint32_t* wp = reinterpret_cast<const uint32_t*>(row);
       const int byte = 3 * lane, wi = byte >> 2, sh = (byte & 3) * 8;
       const uint32_t lo = wp[wi];
-      const uint32_t hi = (sh > 8) ? wp[wi + 1] : 0u;  // wi + 1 <= 23 whenever sh > 8
+      // hi is used only when sh > 8, and then wi + 1 <= 23
+      const uint32_t hi = (kStaged || sh > 8) ? wp[wi + 1] : 0u;
       f = __funnelshift_r(lo, hi, sh);
       f3 = __funnelshift_r(lo, hi, sh + 1);
     }
@@ -172,27 +174,36 @@ __device__ __forceinline__ uint32_t clamp_s16x2(uint32_t x, uint32_t hi) {
   return y;
 }
 
+// The lane's codes u0..u3 (columns 4l..4l+3) clamped in two pairs of 16-bit lanes, u0 and
+// u2 in one word and u1 and u3 in the other, so that w02 | w13 << b already holds u0 | u1 << b
+// in its low half and u2 | u3 << b in its high half (2b <= 16).
+__device__ __forceinline__ void clamp_pairs(f2 t01, f2 t23, uint32_t hi, uint32_t& w02, uint32_t& w13) {
+  w02 = clamp_s16x2(__byte_perm(__float_as_uint(t01.x), __float_as_uint(t23.x), 0x5410), hi);
+  w13 = clamp_s16x2(__byte_perm(__float_as_uint(t01.y), __float_as_uint(t23.y), 0x5410), hi);
+}
+
 template <int BITS>
 __device__ __forceinline__ void store_codes_s16(uint8_t* row, int lane, f2 t01, f2 t23, uint32_t hi) {
-  const uint32_t w01 = clamp_s16x2(__byte_perm(__float_as_uint(t01.x), __float_as_uint(t01.y), 0x5410), hi);
-  const uint32_t w23 = clamp_s16x2(__byte_perm(__float_as_uint(t23.x), __float_as_uint(t23.y), 0x5410), hi);
+  uint32_t w02, w13;
+  clamp_pairs(t01, t23, hi, w02, w13);
   if constexpr (BITS == 8) {
-    reinterpret_cast<uint32_t*>(row)[lane] = __byte_perm(w01, w23, 0x6420);
-  } else if constexpr (BITS == 4) {
-    const uint32_t x01 = w01 | (w01 >> 12), x23 = w23 | (w23 >> 12);
-    reinterpret_cast<uint16_t*>(row)[lane] = static_cast<uint16_t>(__byte_perm(x01, x23, 0x0040));
-  } else if constexpr (BITS == 2) {
-    const uint32_t x = w01 | (w23 << 4);
-    row[lane] = static_cast<uint8_t>(x | (x >> 14));
+    reinterpret_cast<uint32_t*>(row)[lane] = __byte_perm(w02, w13, 0x6240);
   } else {
-    const uint32_t x01 = w01 | (w01 >> 10), x23 = w23 | (w23 >> 10);
-    const uint32_t f = (x01 & 0xFFFu) | (x23 << 12);   // bits 24.. are not stored
-    // even lanes: 16 bits at byte 3l, 8 bits at 3l + 2; odd lanes: 8 bits at 3l, 16 at 3l + 1
-    const int odd = lane & 1;
-    uint8_t* p8 = row + 3 * lane + 2 - 2 * odd;
-    uint16_t* p16 = reinterpret_cast<uint16_t*>(row + 3 * lane + odd);
-    *p8 = static_cast<uint8_t>(f >> (16 - 16 * odd));
-    *p16 = static_cast<uint16_t>(f >> (8 * odd));
+    const uint32_t x = w02 + (w13 << BITS);     // u0 | u1 << b, u2 | u3 << b at bit 16
+    if constexpr (BITS == 4) {
+      reinterpret_cast<uint16_t*>(row)[lane] = static_cast<uint16_t>(__byte_perm(x, 0u, 0x0020));
+    } else if constexpr (BITS == 2) {
+      row[lane] = static_cast<uint8_t>(x | (x >> 12));
+    } else {
+      // the high half moves down to bit 12; bits 24.. are not stored
+      const uint32_t f = (x & 0xFFFu) | ((x >> 4) & ~0xFFFu);
+      // even lanes: 16 bits at byte 3l, 8 bits at 3l + 2; odd lanes: 8 bits at 3l, 16 at 3l + 1
+      const int odd = lane & 1;
+      uint8_t* p8 = row + 3 * lane + 2 - 2 * odd;
+      uint16_t* p16 = reinterpret_cast<uint16_t*>(row + 3 * lane + odd);
+      *p8 = static_cast<uint8_t>(f >> (16 - 16 * odd));
+      *p16 = static_cast<uint16_t>(f >> (8 * odd));
+    }
   }
 }
 
@@ -321,7 +332,8 @@ struct __align__(16) WarpRows {
   float4 rp[RPW];                  // restore of row i: -(2^23 + 2^(b-1)), -(2^(23-b) +
                                    //   2^(b-1)), dec_i r_i, 0 (pivot rows: 0, 0, dec_i r_i, 0)
   uint4 st[RPW];                   // final codes of row i: {bits of 1.5*2^23 + 2^(b-1),
-                                   //   (2^b - 1) * 0x10001, 2b | row offset << 16, b}
+                                   //   (2^b - 1) * 0x10001, 2^(2b) - 1,
+                                   //   b | (16 - 2b) << 8 | row offset << 16}
                                    //   (pivot rows: {.., 0, 0, 16})
   f2 clampb[RPW];                  // least-squares clamp: 1.5*2^23 -+ qmax
   uint32_t info[RPW];              // bits | offset << 8
@@ -364,6 +376,15 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
                "l"(src)
                : "memory");
+}
+
+// The same copy issued only where `pred` holds, as a predicated instruction (no branch);
+// where it does not, nothing is read or written.
+__device__ __forceinline__ void cp_async16_if(bool pred, void* dst, const void* src) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %2, 0;\n\t@p cp.async.cg.shared.global [%0], [%1], 16;\n\t}"
+      ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))), "l"(src), "r"(int(pred))
+      : "memory");
 }
 
 // The 256 threads (8 warps) that work on one (request, head) item meet at a named
@@ -416,8 +437,8 @@ __device__ __forceinline__ void mixed_row_consts(WarpRows& wr, int l, int bits, 
     wr.rk[l] = make_uint4(M, M << bits, uint32_t(150 - bits) << 23,
                           uint32_t(4 * bits) | (uint32_t(2 * bits) << 8) | (code_off << 16));
     wr.rp[l] = make_float4(-(8388608.0f + bias), -(float(1u << (23 - bits)) + bias), rd, 0.0f);
-    wr.st[l] = make_uint4(__float_as_uint(mb), M * 0x00010001u, uint32_t(2 * bits) | (code_off << 16),
-                          uint32_t(bits));
+    wr.st[l] = make_uint4(__float_as_uint(mb), M * 0x00010001u, (1u << (2 * bits)) - 1u,
+                          uint32_t(bits) | (uint32_t(16 - 2 * bits) << 8) | (code_off << 16));
   }
 }
 
@@ -501,7 +522,7 @@ __device__ __forceinline__ void decode_warp(CtaSmem& cs, WarpRows& wr, const Hea
       s[rr][1] = mul2(mul2(q23, rd), cin[1]);
     } else {
       uint32_t cd[4];
-      load_codes<BITS>(wcodes + rr * (D * BITS / 8), lane, cd);
+      load_codes<BITS, true>(wcodes + rr * (D * BITS / 8), lane, cd);
 #ifdef STQ_CHECKS
       // the mantissa of an unpacked code holds u << pos: zero exactly when u = 0
       zero_code |= ((cd[0] & 0x7FFFFFu) == 0) || ((cd[1] & 0x7FFFFFu) == 0) ||
@@ -661,10 +682,11 @@ __device__ __forceinline__ void decode_pivot_warp(CtaSmem& cs, WarpRows& wr, con
   if (tid < 2 * D) hr.sc.put(tid, 0.0f);
 }
 
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-               "l"(src)
-               : "memory");
+__device__ __forceinline__ void cp_async4_if(bool pred, void* dst, const void* src) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %2, 0;\n\t@p cp.async.ca.shared.global [%0], [%1], 4;\n\t}"
+      ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))), "l"(src), "r"(int(pred))
+      : "memory");
 }
 
 // Warp w's asynchronous copies of the inputs of item (h, bq): its packed rows into
@@ -687,30 +709,31 @@ __device__ __forceinline__ void prefetch_item(const PoolDev& P, const int32_t* _
     raw.slot = slot;
     raw.rec = rec;
   }
-  if (slot >= 0 && slot < P.n_slots) {
-    const uint64_t vi = uint64_t(bq) * P.H + h;
-    const uint64_t soff = (uint64_t(slot) * P.H + h) * (2 * D * ES);
-    const uint8_t* cg = P.codes + uint64_t(slot) * P.slot_code_bytes + rec.x + rec.y;
+  // every copy is predicated (no branch); the addresses of a skipped item or of a
+  // missing next item are formed from index 0 and never used
+  const bool ok = slot >= 0 && slot < P.n_slots;
+  const int sl = ok ? slot : 0;
+  const uint64_t vi = uint64_t(bq) * P.H + h;
+  const uint64_t soff = (uint64_t(sl) * P.H + h) * (2 * D * ES);
+  const uint8_t* cg = P.codes + uint64_t(sl) * P.slot_code_bytes + rec.x + rec.y;
 #pragma unroll
-    for (int j = 0; j < (RPW * D) / (16 * 32); ++j) {
-      const int o = 16 * lane + 16 * 32 * j;
-      if (o < int(rec.z)) cp_async16(codes_dst + o, cg + o);
-    }
-    // eight 64-byte row arrays, four lanes each; v of the 16 columns the warp owns shares
-    // the rows' offset (r0 = 16 w)
-    const int grp = lane >> 2, part = 16 * (lane & 3);
-    const uint64_t off = grp < 4 ? (vi * D + r0) * 4 : grp < 7 ? (uint64_t(h) * D + r0) * 4 : soff + r0 * ES;
-    const bool valid = (grp != 2 || P.kind != 0) && (grp != 7 || part < RPW * ES);
-    if (valid) cp_async16(reinterpret_cast<uint8_t*>(&raw) + 64 * grp + part, ptab[grp] + off + part);
-    if (16 * lane < D * ES)
-      cp_async16(reinterpret_cast<uint8_t*>(raw.c) + 16 * lane, ptab[7] + soff + D * ES + 16 * lane);
-    if (lane == 4) cp_async4(&raw.beta, beta + vi);
-    if (lane == 5 && P.kind == 0) cp_async4(&raw.gate_s, gate + vi);
+  for (int j = 0; j < (RPW * D) / (16 * 32); ++j) {
+    const int o = 16 * lane + 16 * 32 * j;
+    cp_async16_if(ok && o < int(rec.z), codes_dst + o, cg + o);
   }
-  if (has_next) {
-    if (lane == 6) cp_async4(&raw.next_slot, slots + bn);
-    if (lane == 7) cp_async16(&raw.next_rec, P.warp_rec + hn * NW + w);
-  }
+  // eight 64-byte row arrays, four lanes each; v of the 16 columns the warp owns shares
+  // the rows' offset (r0 = 16 w)
+  const int grp = lane >> 2, part = 16 * (lane & 3);
+  const uint64_t off = grp < 4 ? (vi * D + r0) * 4 : grp < 7 ? (uint64_t(h) * D + r0) * 4 : soff + r0 * ES;
+  const bool valid = (grp != 2 || P.kind != 0) && (grp != 7 || part < RPW * ES);
+  cp_async16_if(ok && valid, reinterpret_cast<uint8_t*>(&raw) + 64 * grp + part, ptab[grp] + off + part);
+  cp_async16_if(ok && 16 * lane < D * ES, reinterpret_cast<uint8_t*>(raw.c) + 16 * lane,
+                ptab[7] + soff + D * ES + 16 * lane);
+  cp_async4_if(ok && lane == 4, &raw.beta, beta + vi);
+  cp_async4_if(ok && lane == 5 && P.kind == 0, &raw.gate_s, gate + vi);
+  const int nb = has_next ? bn : 0, nh = has_next ? hn : 0;
+  cp_async4_if(has_next && lane == 6, &raw.next_slot, slots + nb);
+  cp_async16_if(has_next && lane == 7, &raw.next_rec, P.warp_rec + nh * NW + w);
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
 

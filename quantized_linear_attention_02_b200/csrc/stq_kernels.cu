@@ -249,20 +249,18 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
 #pragma unroll
       for (int rr = 0; rr < RPW; ++rr) {
         // every row computes; a pivot row (zero store constants, offset 0) stores nothing
-        const uint4 T = wr.st[rr];                     // 1.5*2^23 + bias, M * 0x10001, 2b | offset << 16, b
-        const int bits = int(T.w);
+        const uint4 T = wr.st[rr];                     // 1.5*2^23 + bias, M * 0x10001, 2^(2b) - 1, b | (16 - 2b) << 8 | offset << 16
+        const int bits = int(T.w & 0xFFu);
         const bool code_row = bits != PIVOT;
         const f2 mb = dup(__uint_as_float(T.x));
         const f2 t01 = fma2(s[rr][0], ic[0], mb);
         const f2 t23 = fma2(s[rr][1], ic[1], mb);
-        const uint32_t M = T.y & 0xFFFFu;
-        const uint32_t w01 = clamp_s16x2(__byte_perm(__float_as_uint(t01.x), __float_as_uint(t01.y), 0x5410), T.y);
-        const uint32_t w23 = clamp_s16x2(__byte_perm(__float_as_uint(t23.x), __float_as_uint(t23.y), 0x5410), T.y);
-        const uint32_t sh = T.z & 0xFFu;                // 2b (0 for a pivot row)
-        const uint32_t x01 = (w01 & M) | (w01 >> (16 - (sh >> 1)));      // u0 | u1 << b
-        const uint32_t x23 = (w23 & M) | (w23 >> (16 - (sh >> 1)));      // u2 | u3 << b
-        const uint32_t f = x01 | (x23 << sh);
-        uint8_t* dst = stage + (T.z >> 16) + ((bits * lane) >> 1);
+        uint32_t w02, w13;
+        clamp_pairs(t01, t23, T.y, w02, w13);
+        // funnel shifts take their count mod 32: b and 16 - 2b straight from T.w
+        const uint32_t x = w02 | __funnelshift_l(0u, w13, T.w);                // u0 | u1 << b, u2 | u3 << b at 16
+        const uint32_t f = (x & T.z) | (__funnelshift_r(x, 0u, T.w >> 8) & ~T.z);
+        uint8_t* dst = stage + (T.w >> 16) + ((bits * lane) >> 1);
         if (code_row) dst[0] = static_cast<uint8_t>(f);
         if (code_row && bits >= 4) dst[1] = static_cast<uint8_t>(f >> 8);
         if (code_row && bits >= 6) dst[2] = static_cast<uint8_t>(f >> 16);
