@@ -68,28 +68,15 @@ struct AbsmaxStore {
     for (int rr = 0; rr < RPW; ++rr) {
       const float4 i2 = *reinterpret_cast<const float4*>(&wr.irr[rr & ~1]);
       const f2 ir = (rr & 1) ? make_float2(i2.z, i2.w) : make_float2(i2.x, i2.y);
+      // |S_ij| * fl(1/r_i) <= qmax (1 + 2^-22) (binary16 r: <= qmax (1 + 2^-10)), so
+      // |n| <= qmax + 1: the 16-bit lanes hold it
       if constexpr (BITS == MIXED) {
-        const uint32_t info = wr.info[rr];
-        const int bits = row_bits(info);
-        if (bits == PIVOT) continue;
-        const float mb = wr.mb[rr], q = wr.qm[rr];
-        const f2 t01 = fma2(s[rr][0], ir, dup(mb));
-        const f2 t23 = fma2(s[rr][1], ir, dup(mb));
-        const float lo_b = mb - q, hi_b = mb + q;
-        const uint32_t t[4] = {__float_as_uint(fminf(fmaxf(t01.x, lo_b), hi_b)),
-                               __float_as_uint(fminf(fmaxf(t01.y, lo_b), hi_b)),
-                               __float_as_uint(fminf(fmaxf(t23.x, lo_b), hi_b)),
-                               __float_as_uint(fminf(fmaxf(t23.y, lo_b), hi_b))};
-        uint8_t* row = codes_global + row_off(info);
-        switch (bits) {
-          case 2: store_codes<2>(row, lane, t); break;
-          case 4: store_codes<4>(row, lane, t); break;
-          case 6: store_codes<6>(row, lane, t); break;
-          default: store_codes<8>(row, lane, t); break;
-        }
+        // the refit's branch-free staged store (a pivot row stores nothing)
+        const uint4 T = wr.st[rr];
+        const f2 mb = dup(__uint_as_float(T.x));
+        stage_mixed_codes(T, fma2(s[rr][0], ir, mb), fma2(s[rr][1], ir, mb),
+                          static_cast<uint32_t>(__cvta_generic_to_shared(stage)), lane);
       } else {
-        // |S_ij| * fl(1/r_i) <= qmax (1 + 2^-22) (binary16 r: <= qmax (1 + 2^-10)), so
-        // |n| <= qmax + 1: the 16-bit lanes hold it
         constexpr float MB = MAGIC + float(1 << (BITS - 1));
         constexpr uint32_t HI = ((1u << BITS) - 1u) * 0x00010001u;
         const f2 t01 = fma2(s[rr][0], ir, dup(MB));
@@ -97,6 +84,7 @@ struct AbsmaxStore {
         store_codes_s16<BITS>(codes_global + warp_code_start + rr * (D * BITS / 8), lane, t01, t23, HI);
       }
     }
+    if constexpr (BITS == MIXED) copy_out_staged(wr, stage, codes_global + warp_code_start, lane);
 
     // --- readout from the per-warp partials the caller left in red[1][0] ------------
     if (o_global != nullptr) {

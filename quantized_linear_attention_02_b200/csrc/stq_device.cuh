@@ -378,6 +378,44 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
                : "memory");
 }
 
+// Store the low byte of v at shared-memory address `addr` where `pred` holds, as a
+// predicated instruction (no branch).
+__device__ __forceinline__ void st_shared_u8_if(bool pred, uint32_t addr, uint32_t v) {
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %2, 0;\n\t@p st.shared.u8 [%0], %1;\n\t}"
+               ::"r"(addr), "r"(v), "r"(int(pred))
+               : "memory");
+}
+
+// Mixed-width rows: pack this lane's four codes of one row (t = 1.5*2^23 + bias + n in the
+// low 16 bits, |n| < 2^15) with the row's store constants T (WarpRows::st), clamped to
+// [1, 2^b - 1] in 16-bit lanes, and store its b/2 bytes into the warp's staging area at
+// shared address `stage_s` (the area takes the pool's layout of the warp's rows). Any width
+// runs the same instructions; a pivot row (zero constants) stores nothing.
+__device__ __forceinline__ void stage_mixed_codes(uint4 T, f2 t01, f2 t23, uint32_t stage_s, int lane) {
+  const int bits = int(T.w & 0xFFu);
+  const bool code_row = bits != PIVOT;
+  uint32_t w02, w13;
+  clamp_pairs(t01, t23, T.y, w02, w13);
+  // funnel shifts take their count mod 32: b and 16 - 2b straight from T.w
+  const uint32_t x = w02 | __funnelshift_l(0u, w13, T.w);                // u0 | u1 << b, u2 | u3 << b at 16
+  const uint32_t f = (x & T.z) | (__funnelshift_r(x, 0u, T.w >> 8) & ~T.z);
+  const uint32_t dst = stage_s + (T.w >> 16) + uint32_t((bits * lane) >> 1);
+  st_shared_u8_if(code_row, dst, f);
+  st_shared_u8_if(code_row && bits >= 4, dst + 1, f >> 8);
+  st_shared_u8_if(code_row && bits >= 6, dst + 2, f >> 16);
+  st_shared_u8_if(code_row && bits >= 8, dst + 3, f >> 24);
+}
+
+// Copy the warp's staged codes (16 b bytes per quantised row, in the pool's layout) to the
+// pool at `dst` with 16-byte stores.
+__device__ __forceinline__ void copy_out_staged(const WarpRows& wr, const uint8_t* stage, uint8_t* dst, int lane) {
+  const uint32_t my = lane < RPW ? (row_bits(wr.info[lane]) == PIVOT ? 0u : 16u * row_bits(wr.info[lane])) : 0u;
+  const int bytes = int(__reduce_add_sync(0xffffffffu, my));
+  __syncwarp();
+  for (int o = 16 * lane; o < bytes; o += 16 * 32)
+    *reinterpret_cast<uint4*>(dst + o) = *reinterpret_cast<const uint4*>(stage + o);
+}
+
 // The same copy issued only where `pred` holds, as a predicated instruction (no branch);
 // where it does not, nothing is read or written.
 __device__ __forceinline__ void cp_async16_if(bool pred, void* dst, const void* src) {

@@ -245,33 +245,15 @@ __device__ __forceinline__ void refit_store(CtaSmem& cs, WarpRows& wr, f2 (&s)[R
     if (!any_wide) {
       // Mixed widths: clamp in 16-bit lanes, pack any width without a branch, and put
       // each lane's b/2 bytes into the warp's staging area (the staged codes are consumed
-      // by now; it has the pool's layout), then copy the area out with 16-byte stores.
+      // by now), then copy the area out with 16-byte stores.
+      const uint32_t stage_s = static_cast<uint32_t>(__cvta_generic_to_shared(stage));
 #pragma unroll
       for (int rr = 0; rr < RPW; ++rr) {
-        // every row computes; a pivot row (zero store constants, offset 0) stores nothing
-        const uint4 T = wr.st[rr];                     // 1.5*2^23 + bias, M * 0x10001, 2^(2b) - 1, b | (16 - 2b) << 8 | offset << 16
-        const int bits = int(T.w & 0xFFu);
-        const bool code_row = bits != PIVOT;
+        const uint4 T = wr.st[rr];
         const f2 mb = dup(__uint_as_float(T.x));
-        const f2 t01 = fma2(s[rr][0], ic[0], mb);
-        const f2 t23 = fma2(s[rr][1], ic[1], mb);
-        uint32_t w02, w13;
-        clamp_pairs(t01, t23, T.y, w02, w13);
-        // funnel shifts take their count mod 32: b and 16 - 2b straight from T.w
-        const uint32_t x = w02 | __funnelshift_l(0u, w13, T.w);                // u0 | u1 << b, u2 | u3 << b at 16
-        const uint32_t f = (x & T.z) | (__funnelshift_r(x, 0u, T.w >> 8) & ~T.z);
-        uint8_t* dst = stage + (T.w >> 16) + ((bits * lane) >> 1);
-        if (code_row) dst[0] = static_cast<uint8_t>(f);
-        if (code_row && bits >= 4) dst[1] = static_cast<uint8_t>(f >> 8);
-        if (code_row && bits >= 6) dst[2] = static_cast<uint8_t>(f >> 16);
-        if (code_row && bits >= 8) dst[3] = static_cast<uint8_t>(f >> 24);
+        stage_mixed_codes(T, fma2(s[rr][0], ic[0], mb), fma2(s[rr][1], ic[1], mb), stage_s, lane);
       }
-      // bytes of this warp's rows: 16 b per quantised row
-      const uint32_t my = lane < RPW ? (row_bits(wr.info[lane]) == PIVOT ? 0u : 16u * row_bits(wr.info[lane])) : 0u;
-      const int bytes = int(__reduce_add_sync(0xffffffffu, my));
-      __syncwarp();
-      for (int o = 16 * lane; o < bytes; o += 16 * 32)
-        *reinterpret_cast<uint4*>(codes_global + warp_code_start + o) = *reinterpret_cast<const uint4*>(stage + o);
+      copy_out_staged(wr, stage, codes_global + warp_code_start, lane);
       return;
     }
   }
