@@ -45,8 +45,8 @@ FP32_LANES_PER_SM = 128
 # ncu dram bytes (read + write) per launch of decode_kernel on the default workload
 # (GDN B = 512, dual-axis refit), and the sha256 of the kernel sources they were taken
 # with (a changed kernel voids them).
-TRAFFIC = {"bytes": 2 * (193_409_536 + 126_277_376),
-           "kernel_sha256": "859456e5c98609cf3d04375811fdc9abaebdd35d0cde1f0058f6f013640a3e45",
+TRAFFIC = {"bytes": 2 * (193_410_048 + 124_321_280),
+           "kernel_sha256": "b81b69fa4e87e99547ed6ec1e1a71ed6942a634497f4d33ed93c64c47273bd1f",
            "source": "profiles/decode_kernel_gdn_b256_h48_nominal6.md: dram read + write of one "
                      "B = 256 launch, doubled for B = 512 (traffic grows with B)"}
 
