@@ -51,6 +51,33 @@ TRAFFIC = {"bytes": 2 * (193_410_048 + 124_321_280),
                      "B = 256 launch, doubled for B = 512 (traffic grows with B)"}
 
 
+def issue_rates(stream, reps=3):
+    """Measured lane-operation rates (TFLOP/s-like units: 1e12 lane operations per second)
+    of packed and of scalar FP32 FMA (the FMA pipe) and of LOP3 (the ALU pipe) on this
+    GPU: the library's
+    issue-rate probe at full occupancy, timed with CUDA events on `stream`, best of `reps`
+    launches after one warm-up launch."""
+    import torch
+    from quantized_linear_attention_02_b200 import stq
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    blocks, iters = 4 * n_sm, 20000           # 2,048 threads per SM
+    out = torch.empty(blocks * stq.PROBE_THREADS, device="cuda")
+    rates = {}
+    for mode, name in ((0, "ffma2"), (1, "ffma"), (2, "lop3")):
+        stq.issue_rate_probe(mode, blocks, iters, out, stream)
+        best = 0.0
+        for _ in range(reps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            ops = stq.issue_rate_probe(mode, blocks, iters, out, stream)
+            e1.record(stream)
+            e1.synchronize()
+            best = max(best, ops / (e0.elapsed_time(e1) * 1e-3) / 1e12)
+        rates[name] = best
+    return rates
+
+
 def kernel_sha():
     """sha256 over the code (comments and blank lines dropped) of the sources the decode
     kernel is compiled from: a comment edit keeps the counters, a code edit voids them."""
@@ -540,6 +567,15 @@ def stq_arm(args, rank, world, local_rank):
            "frac": alu_ach / alu_peak, "traffic": traffic,
            "peak_source": f"{SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x {smax:.0f} MHz",
            "algorithmic_flops_per_launch": flops}
+    # the derived peak checked against the GPU: the issue-rate probe's packed-FMA rate
+    # (the same lane count per SM and clock if the derivation holds) and its LOP3 rate
+    rates = issue_rates(stream)
+    fma_peak = max(rates["ffma2"], rates["ffma"])
+    alu["peak_measured"] = {"value": fma_peak, "unit": "TFLOP/s",
+                            "how": "stq_issue_rate_probe, the faster of mode 0 (fma.rn.f32x2) and mode 1 "
+                                   "(fma.rn.f32) chains at 2,048 threads per SM, CUDA events, best of 3",
+                            "ffma2": rates["ffma2"], "ffma": rates["ffma"], "alu_pipe_lop3": rates["lop3"]}
+    alu["frac_of_measured"] = alu_ach / fma_peak
     roofline = alu if alu["frac"] >= hbm["frac"] else hbm
     other = hbm if roofline is alu else alu
     line = {

@@ -316,6 +316,18 @@ stq_status stq_unit_distortion(int kind, int N, int H, const float* h_row_err,
 stq_status stq_allocate_bits(int n, int n_cand, const int* cand_bits, const double* lifetime,
                              const double* dist, double budget, int n_pivots, uint8_t* out_bits);
 
+/* Issue-rate probe (a measurement aid with no counterpart in the pages): launches
+ * `blocks` CTAs of 512 threads on `stream`; each thread runs 8 independent
+ * register-only chains of `iters` instructions of one kind -- mode 0: packed
+ * fma.rn.f32x2 (2 lane operations each), 1: scalar fma.rn.f32, 2: lop3.b32 -- and
+ * writes one float per thread to d_out (device, blocks * 512 floats, caller-owned).
+ * Timed by the caller with CUDA events it gives the rate at which the GPU retires that
+ * instruction kind: blocks * 512 * 8 * iters lane operations (twice that for mode 0).
+ * The decode step is bound by instruction issue on the CUDA cores; this is the measured
+ * rate its roofline is read against. Errors: STQ_ERR_INVALID_ARG (mode, blocks outside
+ * [1, 65535], iters < 1, NULL d_out), STQ_ERR_CUDA (launch). */
+stq_status stq_issue_rate_probe(int mode, int blocks, int iters, float* d_out, void* stream);
+
 /* Synchronise `stream`, read the pool's sticky device error bits, clear them, and
  * return STQ_ERR_DEVICE_CHECK if any was set (message names the check). */
 stq_status stq_pool_check(stq_pool* pool, void* stream);

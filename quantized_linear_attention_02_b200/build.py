@@ -8,7 +8,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libstq.so")
 SOURCES = ["csrc/stq_abi.cpp", "csrc/stq_kernels.cu", "csrc/stq_absmax.cu", "csrc/stq_calib.cu",
-           "csrc/stq_static_staging.cu", "csrc/stq_pipeline.cpp"]
+           "csrc/stq_static_staging.cu", "csrc/stq_pipeline.cpp", "csrc/stq_probe.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [

@@ -81,6 +81,7 @@ def lib():
         "stq_lifetime_weights": (_i, [_vp, _i, _i, _vp]),
         "stq_unit_distortion": (_i, [_i, _i, _i, _vp, _vp, _vp]),
         "stq_allocate_bits": (_i, [_i, _i, _vp, _vp, _vp, ctypes.c_double, _i, _vp]),
+        "stq_issue_rate_probe": (_i, [_i, _i, _i, _vp, _vp]),
         "stq_last_error": (ctypes.c_char_p, []),
         "stq_version": (ctypes.c_char_p, []),
     }
@@ -293,6 +294,20 @@ def row_sq_error(S, S_hat, err, accumulate=False, stream=None):
                                   _ptr(S_hat, torch.float32, "S_hat", n * D * D), n,
                                   _ptr(err, torch.float32, "err", n * D), int(bool(accumulate)),
                                   _stream(stream)))
+
+
+PROBE_THREADS = 512     # threads per CTA of the issue-rate probe
+
+
+def issue_rate_probe(mode, blocks, iters, out, stream=None):
+    """Launch the issue-rate probe (mode 0: packed FP32 FMA, 1: scalar FP32 FMA, 2: LOP3):
+    `blocks` CTAs of 512 threads, 8 chains of `iters` instructions per thread, one float
+    per thread into `out`. Returns the lane operations the launch performs."""
+    import torch
+    _check(lib().stq_issue_rate_probe(int(mode), int(blocks), int(iters),
+                                      _ptr(out, torch.float32, "out", blocks * PROBE_THREADS),
+                                      _stream(stream)))
+    return blocks * PROBE_THREADS * 8 * iters * (2 if mode == 0 else 1)
 
 
 def _host(a, dtype):

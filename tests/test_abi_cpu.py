@@ -151,3 +151,14 @@ def test_pipeline_and_in_head_error_reject_bad_arguments_without_a_gpu(lib):
     cand = (ctypes.c_int * 1)(6)
     st = lib.stq_row_error_at_widths(None, vp(16), 1, vp(16), ctypes.cast(cand, vp), 1, vp(16), None)
     assert st == 1 and b"pool" in lib.stq_last_error()
+
+
+def test_issue_rate_probe_rejects_bad_arguments_without_a_gpu(lib):
+    vp = ctypes.c_void_p
+    assert lib.stq_issue_rate_probe(3, 1, 1, vp(16), None) == 1
+    assert b"mode" in lib.stq_last_error()
+    assert lib.stq_issue_rate_probe(0, 0, 1, vp(16), None) == 1
+    assert lib.stq_issue_rate_probe(0, 65536, 1, vp(16), None) == 1
+    assert lib.stq_issue_rate_probe(1, 1, 0, vp(16), None) == 1
+    assert lib.stq_issue_rate_probe(2, 1, 1, None, None) == 1
+    assert b"d_out" in lib.stq_last_error()
